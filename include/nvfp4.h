@@ -1,0 +1,213 @@
+/*
+ * libnvfp4 — NVFP4 two-level micro-scaling quantization and the block-scaled
+ * GEMM that consumes it, for NVIDIA B200 (sm_100a).
+ *
+ * Format (defined by the pages this library follows):
+ *   - elements: 4-bit E2M1 codes, values +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}
+ *     ("NVIDIA NVFP4 与 Micro-Scaling" section 二; "mxFP4/nvFP4 最小化知识",
+ *     nvFP4的数据结构设计), packed two per byte, first element in the low
+ *     nibble ("FP4" wiki, 技術原理: ONNX FLOAT4E2M1 packing);
+ *   - one E4M3 block scale per 16 consecutive elements along K
+ *     ("Introducing NVFP4 ...", 二级微块 scaling 策略);
+ *   - one FP32 per-tensor scale.  The library stores the encode scale
+ *     g = 2688 / amax = 1 / s_global, s_global = amax / (6 * 448)
+ *     ("low-precision-floats", section FP4 / MXFP4 / NVFP4).
+ *
+ * Quantization rule, per 16-element block with block amax ab:
+ *     s  = e4m3_rne_satfinite((ab * g) / 6)          (fp32 multiply, fp32 divide)
+ *     q  = e2m1_rne_sat((x * g) / decode(s))           (fp32 multiply, IEEE fp32 divide)
+ *   with q = 0 for every element of a block whose scale decodes to 0, and
+ *   g = 1 for an all-zero tensor.
+ *
+ * GEMM: D = alpha * (s_a (.) A)(s_b (.) B)^T, alpha = 1 / (g_a * g_b) in fp32,
+ *   FP32 accumulation in tensor memory ("NVIDIA NVFP4 与 Micro-Scaling"
+ *   section 三 scaled GEMM and section 五 data layout).  A is [M, K], B is
+ *   [N, K]; both K-major ("NT").
+ *
+ * Conventions for every entry point:
+ *   - All buffers are device memory owned and allocated by the caller, except
+ *     where a parameter says "host".  The library never allocates or frees
+ *     memory and never synchronises, except nvfp4_check_device_status().
+ *   - Work is enqueued on the caller's stream (a cudaStream_t; NULL is the
+ *     legacy default stream).  Global scales stay on the device, so a chain of
+ *     calls needs no host round trip.
+ *   - Argument, shape, alignment and architecture errors are returned before
+ *     anything is enqueued.  A failed launch returns NVFP4_ERR_CUDA.
+ *   - Errors met on the device (a bounded wait that gave up, a tensor whose
+ *     global scale is not finite) are recorded in a per-device status word,
+ *     read and cleared by nvfp4_check_device_status().
+ *   - Codes are dense: row r of a [rows, K] code matrix starts at byte
+ *     r * K / 2.  bf16 inputs have a row pitch ld (in elements).
+ *   - Pointers must be 16-byte aligned and ld must keep every row 16-byte
+ *     aligned (ld % 8 == 0).
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of the required block, M too large, ... */
+  NVFP4_ERR_MISALIGNED = 3,        /* pointer or leading dimension breaks 16-byte alignment */
+  NVFP4_ERR_ARCH = 4,              /* current device is not sm_100 */
+  NVFP4_ERR_CUDA = 5,              /* a CUDA call or kernel launch failed */
+  NVFP4_ERR_TIMEOUT = 6,           /* a bounded device wait gave up (device status) */
+  NVFP4_ERR_RANGE = 7,             /* 2688/amax not finite: non-finite input or amax < ~7.9e-36 (device status) */
+  NVFP4_ERR_WORKSPACE = 8          /* workspace smaller than nvfp4_workspace_bytes() */
+} nvfp4_status;
+
+typedef enum {
+  NVFP4_SF_ROWMAJOR = 0, /* [rows, K/16] bytes, row-major */
+  NVFP4_SF_TCGEN05 = 1   /* tensor-core scale atoms, see nvfp4_sf_bytes() */
+} nvfp4_sf_layout;
+
+typedef enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_F32 = 1 } nvfp4_out_dtype;
+
+typedef enum { NVFP4_OP_GEMV_BATCHED = 1, NVFP4_OP_GEMM_QUANT_A = 2 } nvfp4_op;
+
+/* ABI version of this header (bumped on incompatible changes). */
+NVFP4_API int nvfp4_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+/*
+ * Bytes of a block-scale array for a [rows, k] tensor.
+ *   NVFP4_SF_ROWMAJOR: rows * k/16.
+ *   NVFP4_SF_TCGEN05 : the layout the sm_100 block-scaled MMA reads through
+ *     tensor memory.  Rows are padded to a multiple of 128 and the k/16 blocks
+ *     to a multiple of 4.  The array is a sequence of 512-byte atoms, atom
+ *     (i, j) covering rows 128i..128i+127 and blocks 4j..4j+3 at byte offset
+ *     512 * (i * (padded blocks / 4) + j); inside an atom, (row r, block b)
+ *     sits at (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4).  Padding is 0.
+ *     (The pages do not describe this layout; it is the tensor core's.)
+ * Returns 0 for negative sizes or k not a multiple of 16.
+ */
+NVFP4_API size_t nvfp4_sf_bytes(int64_t rows, int64_t k, nvfp4_sf_layout layout);
+
+/*
+ * Tensor amax ("NVIDIA NVFP4 与 Micro-Scaling" section 三, step 1:
+ * |X|_max): *amax_dev = max |x| over a bf16 [rows, k] tensor with row pitch
+ * ldx.  The callee zeroes *amax_dev first (on the stream).  k % 8 == 0.
+ * Non-finite inputs propagate to *amax_dev (a later quantize reports RANGE).
+ */
+NVFP4_API nvfp4_status nvfp4_amax(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, float* amax_dev,
+                        nvfp4_stream_t stream);
+
+/*
+ * Two-level NVFP4 quantization of a bf16 [rows, k] tensor
+ * ("low-precision-floats" section FP4 / MXFP4 / NVFP4, the s_global,
+ * s_block and x_hat formulas; "Introducing NVFP4 ..." 二级微块 scaling).
+ *   codes : out, [rows, k/2] bytes (two E2M1 codes per byte, low nibble first)
+ *   sf    : out, block scales in `layout` (nvfp4_sf_bytes(rows, k, layout) bytes;
+ *           padding of the TCGEN05 layout is written as 0)
+ *   g_dev : out, one fp32, the encode scale 2688 / amax (1 for an all-zero tensor)
+ *   amax_dev : one fp32.  amax_given == 0: workspace and out, the callee
+ *           computes the tensor amax into it (two passes over x).
+ *           amax_given == 1: in, the callee uses *amax_dev as the amax (one pass).
+ * k % 16 == 0 for NVFP4_SF_ROWMAJOR, k % 64 == 0 for NVFP4_SF_TCGEN05.
+ * If 2688/amax is not finite, codes and scales are written as 0, *g_dev as 0,
+ * and the device status records NVFP4_ERR_RANGE.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                            nvfp4_sf_layout layout, float* g_dev, float* amax_dev, int amax_given,
+                            nvfp4_stream_t stream);
+
+/*
+ * Re-layout of row-major block scales [rows, k/16] into the TCGEN05 layout
+ * (see nvfp4_sf_bytes), padding written as 0.  k % 64 == 0.  Pure byte
+ * permutation; the pages are silent on the tensor core's scale layout.
+ */
+NVFP4_API nvfp4_status nvfp4_swizzle_sf(const void* sf_rowmajor, int64_t rows, int64_t k, void* sf_tcgen05,
+                              nvfp4_stream_t stream);
+
+/*
+ * Block-scaled GEMM on tcgen05.mma kind::mxf4nvf4 ("NVIDIA NVFP4 与
+ * Micro-Scaling" section 三: D = g_d((g_a s_a (.) A)(g_b s_b (.) W)); section 五:
+ * the tensor core consumes (FP4 data, FP8 block scale) pairs and accumulates
+ * in FP32).  Here D[m, n] = alpha * sum_k (s_a a)[m,k] (s_b b)[n,k] with
+ * alpha = 1 / (g_a * g_b) computed in fp32 from *g_a_dev and *g_b_dev.
+ *   a_codes [M, K/2], a_sf_tc TCGEN05 scales of A, g_a_dev one fp32 (encode scale of A)
+ *   b_codes [N, K/2], b_sf_tc TCGEN05 scales of B, g_b_dev one fp32
+ *   d: out, [M, N] with row pitch ldd elements, bf16 (round to nearest even)
+ *      or fp32 per out_dtype.
+ * K % 64 == 0, K > 0, M, N >= 1 (any value; tails are masked).
+ */
+NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_sf_tc, const float* g_a_dev, const void* b_codes,
+                        const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d,
+                        int64_t ldd, nvfp4_out_dtype out_dtype, nvfp4_stream_t stream);
+
+/* Workspace bytes needed by an op for the given sizes (0 for bad sizes). */
+NVFP4_API size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Decode batched GEMV: y[m, n] = alpha * sum_k (s_x x_q)[m,k] (s_w w)[n,k]
+ * for M <= 32 activation rows x (bf16 [M, K], pitch ldx) quantized on the fly
+ * with the same rule as nvfp4_quantize (its own amax and global scale), and
+ * pre-quantized weights w (codes [N, K/2], TCGEN05 scales, *g_w_dev).  The
+ * weight stream dominates (decode is memory-bound: "NVIDIA NVFP4 与
+ * Micro-Scaling" section 六).  y: out, bf16 [M, N], pitch ldy.
+ * workspace: device scratch of nvfp4_workspace_bytes(NVFP4_OP_GEMV_BATCHED, M, N, K)
+ *   bytes (quantized x, its scales and g, fp32 partial sums, tile counters);
+ *   every call re-initialises what it uses.  Calls sharing a workspace must not
+ *   overlap on the device.
+ * K % 64 == 0, 1 <= M <= 32.
+ */
+NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t ldx, const void* w_codes,
+                                const void* w_sf_tc, const float* g_w_dev, int64_t N, int64_t K, void* y_bf16,
+                                int64_t ldy, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
+ * Long-K GEMM whose A operand arrives in bf16: A [M, K] (pitch lda) is
+ * quantized to NVFP4 with the nvfp4_quantize rule (tensor amax first), then
+ * multiplied by pre-quantized B as in nvfp4_gemm.
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_QUANT_A, M, N, K) bytes
+ *   (A codes, A scales, g_a, amax_a).
+ * K % 64 == 0.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,
+                                const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                                nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
+                                nvfp4_stream_t stream);
+
+/*
+ * Synchronises the stream, then returns and clears the device status word of
+ * the current device: NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_RANGE (or
+ * NVFP4_ERR_CUDA if the synchronisation itself failed).
+ */
+NVFP4_API nvfp4_status nvfp4_check_device_status(nvfp4_stream_t stream);
+
+/*
+ * Limit, in nanoseconds of device global time, for every bounded wait inside
+ * the library's kernels (default 2e9).  A wait that runs out records
+ * NVFP4_ERR_TIMEOUT and its kernel returns.  Applies to later launches.
+ */
+NVFP4_API void nvfp4_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * Self-test of the bounded-wait path: one thread waits on an mbarrier that
+ * nothing arrives on, for at most limit_ns, then records NVFP4_ERR_TIMEOUT in
+ * the device status.  Nothing else is in flight, so the context stays usable.
+ */
+NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, nvfp4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

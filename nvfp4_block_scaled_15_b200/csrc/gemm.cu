@@ -1,0 +1,758 @@
+// Block-scaled NVFP4 GEMM on the sm_100 tensor core
+// (tcgen05.mma.kind::mxf4nvf4.block_scale, 16-element E4M3 scales).
+//
+// "NVIDIA NVFP4 与 Micro-Scaling" section 三 gives the contraction
+// D = g_d ((g_a s_a (.) A) @ (g_b s_b (.) W)) and says the 5th-gen tensor
+// core consumes (FP4 data, FP8 block scale) pairs, multiplying the scale into
+// each block inside the MMA and accumulating in FP32 (section 五).  Here the
+// global scales fold into alpha = 1 / (g_a g_b) applied in the epilogue.
+//
+// Kernel structure (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: A/B code tiles (128-B swizzled) and scale atoms
+//               into a STAGES-deep shared-memory ring guarded by mbarriers;
+//   warp 1      owns tensor memory; one elected thread copies each stage's
+//               scale atoms smem -> TMEM (tcgen05.cp) and issues the MMAs,
+//               committing to the ring's "empty" barriers;
+//   warps 2-9   epilogue: TMEM -> registers (tcgen05.ld), release the
+//               accumulator, scale by alpha, round, store.
+// Every wait is bounded; a wait that runs out raises a CTA abort flag and
+// records a timeout in the device status word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "quant_core.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int BM = 128;          // rows of A per tile (MMA M)
+constexpr int BK = 256;          // K elements per pipeline stage (128 B of codes per row)
+constexpr int BK_BYTES = BK / 2;
+constexpr int MMA_K = 64;        // K per tcgen05.mma for kind::mxf4nvf4
+constexpr int SF_ATOM = 512;     // bytes of one 128-row x 4-block scale atom
+constexpr uint32_t TMEM_COLS = 512;
+
+// ---------------------------------------------------------------------------
+// GEMM configuration
+// ---------------------------------------------------------------------------
+template <int BN_>
+struct GemmCfg {
+  static constexpr int BN = BN_;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK_BYTES;
+  static constexpr int B_BYTES = BN * BK_BYTES;
+  static constexpr int SFA_BYTES = 4 * SF_ATOM;
+  static constexpr int SFB_BYTES = (BN / 128) * 4 * SF_ATOM;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int ACC_BUFS = (BN == 256) ? 1 : 2;
+  static constexpr int SFB_COLS_PER_K = BN / 32;                       // TMEM columns of B scales per MMA
+  static constexpr int SF_COLS_PER_STAGE = 4 * 4 + 4 * SFB_COLS_PER_K;
+  static constexpr int TMEM_SF_BASE = ACC_BUFS * BN;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = (2 + EPI_WARPS) * 32;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static_assert(TMEM_SF_BASE + STAGES * SF_COLS_PER_STAGE <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct GemmParams {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* g_a;
+  const float* g_b;
+  void* d;
+  int64_t ldd;
+  int M, N, K;
+  int kb4;          // scale atoms along K per 128-row group (= K / 64)
+  int tiles_m, tiles_n;
+  int out_f32;
+  uint64_t wait_limit_ns;
+  int* status;
+};
+
+__host__ __device__ __forceinline__ int round_up_int(int a, int b) { return (a + b - 1) / b * b; }
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// smem descriptor of a 128-B swizzled, K-major code tile (8-row groups 1024 B apart)
+__device__ __forceinline__ uint64_t code_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
+// smem descriptor of one 512-B scale atom read as 32 rows x 16 B (no swizzle)
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int NV>
+__device__ __forceinline__ void store_row(const GemmParams& p, int row, int col0, const uint32_t (&v)[NV],
+                                          float alpha) {
+  if (row >= p.M) return;
+  if (p.out_f32) {
+    float* out = static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + col0;
+    if (col0 + NV <= p.N) {
+#pragma unroll
+      for (int i = 0; i < NV; i += 4) {
+        float4 f = make_float4(__uint_as_float(v[i]) * alpha, __uint_as_float(v[i + 1]) * alpha,
+                               __uint_as_float(v[i + 2]) * alpha, __uint_as_float(v[i + 3]) * alpha);
+        *reinterpret_cast<float4*>(out + i) = f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (col0 + i < p.N) out[i] = __uint_as_float(v[i]) * alpha;
+    }
+  } else {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + col0;
+    if (col0 + NV <= p.N) {
+#pragma unroll
+      for (int i = 0; i < NV; i += 8) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(v[i + 0]) * alpha, __uint_as_float(v[i + 1]) * alpha);
+        w.y = pack_bf16x2(__uint_as_float(v[i + 2]) * alpha, __uint_as_float(v[i + 3]) * alpha);
+        w.z = pack_bf16x2(__uint_as_float(v[i + 4]) * alpha, __uint_as_float(v[i + 5]) * alpha);
+        w.w = pack_bf16x2(__uint_as_float(v[i + 6]) * alpha, __uint_as_float(v[i + 7]) * alpha);
+        *reinterpret_cast<uint4*>(out + i) = w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (col0 + i < p.N) out[i] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmParams p) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + C::ACC_BUFS;
+  uint64_t* mma_done = acc_empty + C::ACC_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < C::ACC_BUFS; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], C::EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int num_kt = (p.K + BK - 1) / BK;
+  const int ksteps_total = p.K / MMA_K;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        const int tm = t % p.tiles_m;
+        const int tn = t / p.tiles_m;
+        const int m0 = tm * BM;
+        const int n0 = tn * BN;
+        const int n_groups = min(BN, round_up_int(p.N - n0, 128)) / 128;
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+          const int nk = min(4, ksteps_total - kt * 4);
+          const uint32_t bytes = C::A_BYTES + C::B_BYTES + nk * SF_ATOM * (1 + n_groups);
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          uint8_t* sSFA = sB + C::B_BYTES;
+          uint8_t* sSFB = sSFA + C::SFA_BYTES;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(sA, &tmA, &full[stage], kt * BK_BYTES, m0);
+          tma_load_2d(sB, &tmB, &full[stage], kt * BK_BYTES, n0);
+          bulk_load(sSFA, p.sfa + (static_cast<int64_t>(tm) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[stage]);
+          for (int g = 0; g < n_groups; ++g)
+            bulk_load(sSFB + g * 4 * SF_ATOM,
+                      p.sfb + (static_cast<int64_t>(n0 / 128 + g) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM,
+                      &full[stage]);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // never leave the CTA with copies still landing in its shared memory
+      for (int s = 0; s < C::STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          (void)mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &no_abort, p.wait_limit_ns, p.status);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        const int tn = t / p.tiles_m;
+        const int n0 = tn * BN;
+        const int n_mma = min(BN, round_up_int(p.N - n0, 128));
+        const uint32_t idesc = idesc_mxf4nvf4(BM, n_mma);
+        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, ksteps_total - kt * 4);
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sSFA = sB + C::B_BYTES;
+          const uint32_t sSFB = sSFA + C::SFA_BYTES;
+          const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE + stage * C::SF_COLS_PER_STAGE;
+          const uint32_t tsfb = tsfa + 16;
+          for (int j = 0; j < nk; ++j) {
+            tc_cp_32x128b_warpx4(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
+            for (int g = 0; g < n_mma / 128; ++g)
+              tc_cp_32x128b_warpx4(tsfb + j * C::SFB_COLS_PER_K + g * 4, sf_desc(sSFB + g * 4 * SF_ATOM + j * SF_ATOM));
+          }
+          for (int j = 0; j < nk; ++j) {
+            mma_mxf4nvf4(d_tmem, code_desc(sA + j * (MMA_K / 2)), code_desc(sB + j * (MMA_K / 2)), idesc,
+                         tsfa + j * 4, tsfb + j * C::SFB_COLS_PER_K, (kt | j) != 0);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // all tensor-core work of this CTA finished before TMEM is released
+      tc_commit(mma_done);
+      volatile int no_abort = 0;
+      (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int ew = warp - 2;
+    const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
+    const int half = ew >> 2;                  // which half of the tile's columns
+    constexpr int HALF = BN / 2;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int tm = t % p.tiles_m;
+      const int tn = t / p.tiles_m;
+      if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
+      tc_fence_after();
+      uint32_t v[HALF];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + half * HALF;
+#pragma unroll
+      for (int c = 0; c < HALF / 32; ++c) tmem_ld_32x32b_x32(taddr + c * 32, v + c * 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+      const int row = tm * BM + quad * 32 + lane;
+      const int col0 = tn * BN + half * HALF;
+      if (col0 < p.N) store_row<HALF>(p, row, col0, v, alpha);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode GEMV: swap-AB (weights are the 128-row MMA operand, the <= 32
+// activation rows the N = 32 operand) with stream-K over (row tile, K stage)
+// units so all SMs stream weights evenly.  Partial sums meet in an fp32
+// workspace; the CTA that completes a row tile writes its bf16 outputs.
+// ---------------------------------------------------------------------------
+constexpr int GV_N = 32;                      // MMA N (activation rows, zero-padded)
+constexpr int GV_STAGES = 8;
+constexpr int GV_A_BYTES = BM * BK_BYTES;     // weights
+constexpr int GV_B_BYTES = GV_N * BK_BYTES;   // activations
+constexpr int GV_STAGE_BYTES = GV_A_BYTES + GV_B_BYTES + 2 * 4 * SF_ATOM;
+constexpr int GV_ACC_BUFS = 2;
+constexpr int GV_SF_BASE = GV_ACC_BUFS * GV_N;
+constexpr int GV_SF_COLS_PER_STAGE = 32;      // 16 for A, 16 for B (one 4-column atom per MMA-K)
+constexpr int GV_EPI_WARPS = 4;
+constexpr int GV_THREADS = (2 + GV_EPI_WARPS) * 32;
+constexpr int GV_SMEM_BYTES = GV_STAGES * GV_STAGE_BYTES + 256 + 1024;
+static_assert(GV_SF_BASE + GV_STAGES * GV_SF_COLS_PER_STAGE <= (int)TMEM_COLS, "TMEM budget");
+
+struct GemvParams {
+  const uint8_t* wsf;      // weight scales, tensor-core layout
+  const uint8_t* xsf;      // activation scales, tensor-core layout (128 padded rows)
+  const float* g_w;
+  const float* g_x;
+  float* y32;              // [M, N] fp32 partial sums (zeroed by the prologue)
+  int* counters;           // [tiles] K-stages completed per row tile
+  __nv_bfloat16* y;
+  int64_t ldy;
+  int M, N, K;
+  int kb4;
+  int tiles;
+  int num_kt;
+  uint64_t wait_limit_ns;
+  int* status;
+};
+
+__global__ void __launch_bounds__(GV_THREADS, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                const GemvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + GV_STAGES * GV_STAGE_BYTES);
+  uint64_t* empty = full + GV_STAGES;
+  uint64_t* acc_full = empty + GV_STAGES;
+  uint64_t* acc_empty = acc_full + GV_ACC_BUFS;
+  uint64_t* mma_done = acc_empty + GV_ACC_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GV_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < GV_ACC_BUFS; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], GV_EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t units = static_cast<int64_t>(p.tiles) * p.num_kt;
+  const int64_t u_begin = units * blockIdx.x / gridDim.x;
+  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+  const int ksteps_total = p.K / MMA_K;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      for (int64_t u = u_begin; u < u_end; ++u) {
+        const int tile = static_cast<int>(u / p.num_kt);
+        const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+        const int nk = min(4, ksteps_total - kt * 4);
+        uint8_t* sA = smem + stage * GV_STAGE_BYTES;
+        uint8_t* sB = sA + GV_A_BYTES;
+        uint8_t* sSFA = sB + GV_B_BYTES;
+        uint8_t* sSFB = sSFA + 4 * SF_ATOM;
+        mbar_arrive_expect_tx(&full[stage], GV_A_BYTES + GV_B_BYTES + 2 * nk * SF_ATOM);
+        tma_load_2d(sA, &tmW, &full[stage], kt * BK_BYTES, tile * BM);
+        tma_load_2d(sB, &tmX, &full[stage], kt * BK_BYTES, 0);
+        bulk_load(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[stage]);
+        bulk_load(sSFB, p.xsf + static_cast<int64_t>(kt) * 4 * SF_ATOM, nk * SF_ATOM, &full[stage]);
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == GV_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      for (int s = 0; s < GV_STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          (void)mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &no_abort, p.wait_limit_ns, p.status);
+        }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      const uint32_t idesc = idesc_mxf4nvf4(BM, GV_N);
+      int64_t u = u_begin;
+      bool ok = true;
+      while (u < u_end && ok) {
+        const int tile = static_cast<int>(u / p.num_kt);
+        const int64_t seg_end = min(u_end, static_cast<int64_t>(tile + 1) * p.num_kt);
+        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * GV_N;
+        bool first = true;
+        for (; u < seg_end; ++u) {
+          const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, ksteps_total - kt * 4);
+          const uint32_t sA = smem_u32(smem + stage * GV_STAGE_BYTES);
+          const uint32_t sB = sA + GV_A_BYTES;
+          const uint32_t sSFA = sB + GV_B_BYTES;
+          const uint32_t sSFB = sSFA + 4 * SF_ATOM;
+          const uint32_t tsfa = tmem_base + GV_SF_BASE + stage * GV_SF_COLS_PER_STAGE;
+          const uint32_t tsfb = tsfa + 16;
+          for (int j = 0; j < nk; ++j) {
+            tc_cp_32x128b_warpx4(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
+            tc_cp_32x128b_warpx4(tsfb + j * 4, sf_desc(sSFB + j * SF_ATOM));
+          }
+          for (int j = 0; j < nk; ++j) {
+            mma_mxf4nvf4(d_tmem, code_desc(sA + j * (MMA_K / 2)), code_desc(sB + j * (MMA_K / 2)), idesc,
+                         tsfa + j * 4, tsfb + j * 4, first ? 0u : 1u);
+            first = false;
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == GV_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == GV_ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      tc_commit(mma_done);
+      volatile int no_abort = 0;
+      (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
+    }
+  } else {
+    const int quad = warp & 3;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_w, *p.g_x));
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int64_t u = u_begin;
+    while (u < u_end) {
+      const int tile = static_cast<int>(u / p.num_kt);
+      const int64_t seg_end = min(u_end, static_cast<int64_t>(tile + 1) * p.num_kt);
+      const int seg_units = static_cast<int>(seg_end - u);
+      u = seg_end;
+      if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * GV_N, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == GV_ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+      // this warp owns weight rows (= output columns) n of one 32-row slice
+      const int n = tile * BM + quad * 32 + lane;
+      if (n < p.N) {
+#pragma unroll
+        for (int m = 0; m < GV_N; ++m)
+          if (m < p.M) atomicAdd(&p.y32[static_cast<int64_t>(m) * p.N + n], __uint_as_float(v[m]));
+      }
+      __threadfence();
+      __syncwarp();
+      int done = 0;
+      if (lane == 0) done = atomicAdd(&p.counters[tile * 4 + quad], seg_units) + seg_units;
+      done = __shfl_sync(0xFFFFFFFFu, done, 0);
+      if (done == p.num_kt) {
+        __threadfence();
+        if (n < p.N) {
+          for (int m = 0; m < p.M; ++m) {
+            const float sum = __ldcg(&p.y32[static_cast<int64_t>(m) * p.N + n]);
+            p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
+// clearing of the partial sums.  CTA 0 quantizes all M rows of x into 32
+// padded code rows and 128 padded scale rows; the other CTAs clear y32 and
+// the tile counters.
+constexpr int GP_THREADS = 1024;
+
+__global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                                   int64_t ldx, uint8_t* __restrict__ xq,
+                                                                   uint8_t* __restrict__ xsf, float* __restrict__ g_x,
+                                                                   float* __restrict__ y32, int64_t y32_words,
+                                                                   int* __restrict__ counters, int n_counters,
+                                                                   int* __restrict__ status) {
+  if (blockIdx.x > 0) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x - 1) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < y32_words; i += stride)
+      y32[i] = 0.0f;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n_counters; i += stride)
+      counters[i] = 0;
+    return;
+  }
+  const int chunks = K >> 3;                 // 16-B chunks per row
+  const int kb = K >> 4;
+  // pass 1: amax over the M real rows
+  uint32_t m = 0;
+  for (int64_t i = threadIdx.x; i < static_cast<int64_t>(M) * chunks; i += GP_THREADS) {
+    const int r = static_cast<int>(i / chunks);
+    const int c = static_cast<int>(i - static_cast<int64_t>(r) * chunks);
+    const uint4 v = *(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx) + c);
+    m = max(m, abs_max_bits8(v));
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t red[GP_THREADS / 32];
+  __shared__ float g_sh;
+  __shared__ int valid_sh;
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t t = red[threadIdx.x];
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (threadIdx.x == 0) {
+      bool valid;
+      const float g = global_scale_from_amax(__uint_as_float(t << 16), valid);
+      g_sh = valid ? g : 0.0f;
+      valid_sh = valid;
+      *g_x = g_sh;
+      if (!valid) record_status(status, kDevRange);
+    }
+  }
+  __syncthreads();
+  const float g = g_sh;
+  const bool valid = valid_sh != 0;
+  // pass 2: 32 code rows (rows >= M are zero) and 128 scale rows (rows >= M zero)
+  const int lane = threadIdx.x & 31;
+  const int64_t items = static_cast<int64_t>(128) * chunks;   // whole warps, chunks % 8 == 0
+  for (int64_t i = threadIdx.x; i < items; i += GP_THREADS) {
+    const int r = static_cast<int>(i / chunks);
+    const int c = static_cast<int>(i - static_cast<int64_t>(r) * chunks);
+    const bool real = r < M && valid;
+    const uint4 v = real ? *(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx) + c)
+                         : make_uint4(0, 0, 0, 0);
+    uint32_t s;
+    uint32_t q = quantize_half_block(v, real ? g : 0.0f, s);
+    if (!real) { q = 0; s = 0; }
+    if (r < GV_N) reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1))[c] = q;
+    const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
+    const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
+    const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
+    if ((lane & 7) == 0)
+      *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, c >> 1, kb)) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [rows, k] E2M1 codes (k/2 bytes per row) as a 2-D uint8 tensor, boxes of
+// 128 B x box_rows, 128-B swizzle (the tcgen05 K-major SW128 operand layout).
+bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                      const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                      nvfp4_out_dtype out, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  CUtensorMap tmA, tmB;
+  if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, BN)) return NVFP4_ERR_CUDA;
+  GemmParams p;
+  p.sfa = static_cast<const uint8_t*>(a_sf);
+  p.sfb = static_cast<const uint8_t*>(b_sf);
+  p.g_a = g_a;
+  p.g_b = g_b;
+  p.d = d;
+  p.ldd = ldd;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.kb4 = static_cast<int>(K / 64);
+  p.tiles_m = static_cast<int>((M + BM - 1) / BM);
+  p.tiles_n = static_cast<int>((N + BN - 1) / BN);
+  p.out_f32 = out == NVFP4_OUT_F32;
+  p.wait_limit_ns = wait_limit_ns();
+  p.status = device_status_ptr();
+  if (!p.status) return NVFP4_ERR_CUDA;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return launch_status(e);
+  gemm_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tmA, tmB, p);
+  return launch_status(cudaGetLastError());
+}
+
+}  // namespace
+
+nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                         const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
+                         int64_t ldd, nvfp4_out_dtype out, cudaStream_t s) {
+  if (N <= 128) return run_gemm<128>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  return run_gemm<256>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+}
+
+// Workspace of the GEMV: [32, K/2] activation codes | [128, K/16] activation
+// scales | g_x (16 B) | [M, N] fp32 partials | counters.
+struct GemvWs {
+  size_t xq, xsf, gx, y32, cnt, total;
+};
+
+static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
+  GemvWs w;
+  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
+  w.xq = 0;
+  w.xsf = al(w.xq + static_cast<size_t>(GV_N) * K / 2);
+  w.gx = al(w.xsf + static_cast<size_t>(128) * K / 16);
+  w.y32 = al(w.gx + 16);
+  w.cnt = al(w.y32 + static_cast<size_t>(M) * N * 4);
+  w.total = al(w.cnt + static_cast<size_t>((N + BM - 1) / BM) * 4 * 4);
+  return w;
+}
+
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) { return gemv_ws_layout(M, N, K).total; }
+
+nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
+                         const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s) {
+  const GemvWs L = gemv_ws_layout(M, N, K);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* xq = base + L.xq;
+  uint8_t* xsf = base + L.xsf;
+  float* gx = reinterpret_cast<float*>(base + L.gx);
+  float* y32 = reinterpret_cast<float*>(base + L.y32);
+  int* cnt = reinterpret_cast<int*>(base + L.cnt);
+  const int tiles = static_cast<int>((N + BM - 1) / BM);
+  const int sms = device_sm_count();
+
+  int* status = device_status_ptr();
+  if (!status) return NVFP4_ERR_CUDA;
+  gemv_prologue_kernel<<<sms, GP_THREADS, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(M),
+                                                  static_cast<int>(K), ldx, xq, xsf, gx, y32, M * N, cnt, tiles * 4,
+                                                  status);
+  nvfp4_status st = launch_status(cudaGetLastError());
+  if (st != NVFP4_OK) return st;
+
+  CUtensorMap tmW, tmX;
+  if (!make_code_map(&tmW, w_codes, N, K, BM) || !make_code_map(&tmX, xq, GV_N, K, GV_N)) return NVFP4_ERR_CUDA;
+  GemvParams p;
+  p.wsf = static_cast<const uint8_t*>(w_sf);
+  p.xsf = xsf;
+  p.g_w = g_w;
+  p.g_x = gx;
+  p.y32 = y32;
+  p.counters = cnt;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ldy = ldy;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.kb4 = static_cast<int>(K / 64);
+  p.tiles = tiles;
+  p.num_kt = static_cast<int>((K + BK - 1) / BK);
+  p.wait_limit_ns = wait_limit_ns();
+  p.status = device_status_ptr();
+  if (!p.status) return NVFP4_ERR_CUDA;
+  const int64_t units = static_cast<int64_t>(tiles) * p.num_kt;
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  cudaError_t e = cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_BYTES);
+  if (e != cudaSuccess) return launch_status(e);
+  gemv_kernel<<<grid, GV_THREADS, GV_SMEM_BYTES, s>>>(tmW, tmX, p);
+  return launch_status(cudaGetLastError());
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,43 @@
+// Host-side helpers shared by the library's translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "nvfp4.h"
+
+namespace nvfp4 {
+
+// Current device must be sm_100 (B200 / GB200).
+nvfp4_status check_arch();
+// Maximum dynamic shared memory per block and SM count of the current device.
+int device_sm_count();
+uint64_t wait_limit_ns();
+// Device address of the current device's status word (nullptr on failure).
+int* device_status_ptr();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline nvfp4_status launch_status(cudaError_t e) {
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// Launchers implemented in the .cu files (arguments already validated).
+nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s);
+nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                             nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, cudaStream_t s);
+nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst, cudaStream_t s);
+nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                         const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
+                         int64_t ldd, nvfp4_out_dtype out, cudaStream_t s);
+nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
+                         const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s);
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+}  // namespace nvfp4

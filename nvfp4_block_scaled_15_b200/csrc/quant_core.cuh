@@ -1,0 +1,79 @@
+// NVFP4 block quantization on a pair of lanes ("low-precision-floats",
+// section FP4 / MXFP4 / NVFP4: s_block = (block_amax / 6) / s_global and
+// x_hat = s_global * s_block * Q_E2M1(x / (s_global * s_block)), with the
+// encode scale g = 1 / s_global = 2688 / amax).
+//
+// Two adjacent lanes (2i, 2i+1) hold the two halves (8 bf16 each) of one
+// 16-element block; a single shuffle gives both the block amax.
+#pragma once
+#include <cstdint>
+#include <cuda_fp8.h>
+
+namespace nvfp4 {
+
+// fp32 global encode scale from the tensor amax; valid == false when it is
+// not a finite number (non-finite input, or amax too small).
+__device__ __forceinline__ float global_scale_from_amax(float amax, bool& valid) {
+  if (amax == 0.0f) {
+    valid = true;
+    return 1.0f;
+  }
+  const float g = __fdiv_rn(2688.0f, amax);
+  valid = isfinite(amax) && isfinite(g);
+  return g;
+}
+
+// |x| maximum of 8 bf16 values as 16-bit bit patterns (the order of |bf16|
+// equals the unsigned order of its low 15 bits).
+__device__ __forceinline__ uint32_t abs_max_bits8(const uint4 v) {
+  uint32_t m = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two fp32 values -> one byte of two E2M1 codes (RNE, saturating): lo goes to
+// bits 0..3, hi to bits 4..7.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(out)
+      : "f"(hi), "f"(lo));
+  return out;
+}
+
+// One half block: 8 bf16 in v.  Returns the 4 code bytes (element 0 in the
+// low nibble of byte 0) and, through sf, the block's E4M3 scale byte.  Every
+// lane of the warp must call this (it shuffles with lane ^ 1).
+__device__ __forceinline__ uint32_t quantize_half_block(const uint4 v, const float g, uint32_t& sf) {
+  uint32_t amax_bits = abs_max_bits8(v);
+  amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, 1));
+  const float ab = __uint_as_float(amax_bits << 16);
+  const float s_raw = __fdiv_rn(__fmul_rn(ab, g), 6.0f);
+  const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(s_raw, __NV_SATFINITE, __NV_E4M3);
+  sf = static_cast<uint32_t>(s8);
+  const __half_raw hs = __nv_cvt_fp8_to_halfraw(s8, __NV_E4M3);
+  const float sd = __half2float(__half(hs));
+  if (sd == 0.0f) return 0u;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float u0 = __fdiv_rn(__fmul_rn(bf16_lo(w[i]), g), sd);
+    const float u1 = __fdiv_rn(__fmul_rn(bf16_hi(w[i]), g), sd);
+    out |= e2m1x2(u0, u1) << (8 * i);
+  }
+  return out;
+}
+
+// Byte offset of (row r, block b) in the tensor-core scale layout whose
+// padded block count is kb_pad (a multiple of 4).
+__host__ __device__ __forceinline__ int64_t sf_tc_offset(int64_t r, int64_t b, int64_t kb_pad) {
+  return ((r >> 7) * (kb_pad >> 2) + (b >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
+}
+
+}  // namespace nvfp4

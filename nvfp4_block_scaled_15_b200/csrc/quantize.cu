@@ -1,0 +1,182 @@
+// NVFP4 quantization kernels: tensor amax, two-level block quantization and
+// the re-layout of block scales into the tensor-core scale format.
+//
+// Both passes stream HBM with 128-bit loads; each thread owns half of a
+// 16-element block and its neighbour lane the other half ("NVIDIA NVFP4 与
+// Micro-Scaling" section 三: global scale from |X|_max, then per-block
+// micro-scales; "low-precision-floats" section FP4 / MXFP4 / NVFP4 formulas).
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "quant_core.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;                          // 16-B chunks per thread per segment
+constexpr int kSegChunks = kThreads * kUnroll;      // chunks (of 8 bf16) per CTA row segment
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Pass 1: max |x|.  grid.x strides over rows, grid.y over row segments.
+__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int rows, int k,
+                                                        int64_t ldx, unsigned* __restrict__ amax_bits) {
+  const int chunks = k >> 3;
+  const int c0 = blockIdx.y * kSegChunks + threadIdx.x;
+  uint32_t m = 0;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int c = c0 + u * kThreads;
+      v[u] = (c < chunks) ? ld_stream(row + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) m = max(m, abs_max_bits8(v[u]));
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t red[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t t = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (threadIdx.x == 0 && t != 0) atomicMax(amax_bits, t << 16);
+  }
+}
+
+// Pass 2: block scales and codes.  blockIdx.x = row (rows_alloc >= rows; the
+// extra rows only exist in the tensor-core layout and get zero scales),
+// blockIdx.y = row segment of kSegChunks chunks.
+template <bool kTcLayout>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __restrict__ x, int rows, int k,
+                                                            int64_t ldx, uint8_t* __restrict__ codes,
+                                                            uint8_t* __restrict__ sf, float* __restrict__ g_out,
+                                                            const float* __restrict__ amax_in,
+                                                            int* __restrict__ status) {
+  const int r = blockIdx.x;
+  const int chunks = k >> 3;
+  const int kb = k >> 4;                      // blocks per row
+  const int lane = threadIdx.x & 31;
+  const int c0 = blockIdx.y * kSegChunks + threadIdx.x;
+
+  bool valid;
+  const float g = global_scale_from_amax(*amax_in, valid);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    *g_out = valid ? g : 0.0f;
+    if (!valid) record_status(status, kDevRange);
+  }
+  const bool real_row = r < rows;
+
+  uint4 v[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const int c = c0 + u * kThreads;
+    v[u] = (real_row && valid && c < chunks)
+               ? ld_stream(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx) + c)
+               : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const int c = c0 + u * kThreads;          // chunk index, 2 chunks per block
+    uint32_t s;
+    uint32_t q = quantize_half_block(v[u], valid ? g : 0.0f, s);
+    if (!valid) { q = 0; s = 0; }
+    if (!real_row) s = 0;
+    const bool in_row = c < chunks;
+    if (real_row && in_row) reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(r) * (k >> 1))[c] = q;
+    const int b = c >> 1;                     // block index in the row
+    if (!kTcLayout) {
+      if (real_row && in_row && (lane & 1) == 0) sf[static_cast<int64_t>(r) * kb + b] = static_cast<uint8_t>(s);
+    } else {
+      // lanes 0,2,4,6 (mod 8) hold blocks 4j..4j+3: gather them into one word
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
+      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
+      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
+      if (in_row && (lane & 7) == 0) {
+        const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        *reinterpret_cast<uint32_t*>(sf + sf_tc_offset(r, b, kb)) = word;
+      }
+    }
+  }
+}
+
+// Row-major [rows, kb] scales -> tensor-core atoms; one thread per output
+// 32-bit word (one row's 4 blocks of one atom).
+__global__ void swizzle_kernel(const uint8_t* __restrict__ src, int rows, int kb, int64_t words,
+                               uint32_t* __restrict__ dst) {
+  const int64_t kb4 = kb >> 2;
+  for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < words;
+       w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t atom = w >> 7;
+    const int idx = static_cast<int>(w & 127);
+    const int64_t i = atom / kb4;
+    const int64_t j = atom - i * kb4;
+    const int64_t r = i * 128 + (idx & 3) * 32 + (idx >> 2);
+    uint32_t val = 0;
+    if (r < rows) val = *reinterpret_cast<const uint32_t*>(src + r * kb + j * 4);
+    dst[w] = val;
+  }
+}
+
+}  // namespace
+
+nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(amax_dev, 0, sizeof(float), s);
+  if (e != cudaSuccess) return launch_status(e);
+  if (rows == 0 || k == 0) return NVFP4_OK;
+  const int segs = static_cast<int>((k / 8 + kSegChunks - 1) / kSegChunks);
+  const int64_t want = static_cast<int64_t>(device_sm_count()) * 8 / segs;
+  const int gx = static_cast<int>(rows < want ? rows : (want > 0 ? want : 1));
+  amax_kernel<<<dim3(gx, segs), kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
+                                                  static_cast<int>(k), ldx, reinterpret_cast<unsigned*>(amax_dev));
+  return launch_status(cudaGetLastError());
+}
+
+nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                             nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, cudaStream_t s) {
+  int* status = device_status_ptr();
+  if (!status) return NVFP4_ERR_CUDA;
+  const int segs = static_cast<int>((k / 8 + kSegChunks - 1) / kSegChunks);
+  const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
+  if (grid_rows == 0 || segs == 0) {
+    // nothing to quantize: still publish g (from the given amax)
+    quantize_kernel<false><<<dim3(1, 1), kThreads, 0, s>>>(static_cast<const uint16_t*>(x), 0, 0, ldx,
+                                                           static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf),
+                                                           g_dev, amax_dev, status);
+    return launch_status(cudaGetLastError());
+  }
+  dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  if (layout == NVFP4_SF_TCGEN05)
+    quantize_kernel<true><<<grid, kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
+                                                    static_cast<int>(k), ldx, static_cast<uint8_t*>(codes),
+                                                    static_cast<uint8_t*>(sf), g_dev, amax_dev, status);
+  else
+    quantize_kernel<false><<<grid, kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
+                                                     static_cast<int>(k), ldx, static_cast<uint8_t*>(codes),
+                                                     static_cast<uint8_t*>(sf), g_dev, amax_dev, status);
+  return launch_status(cudaGetLastError());
+}
+
+nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst, cudaStream_t s) {
+  const int64_t kb = k / 16;
+  const int64_t words = round_up(rows, 128) * kb / 4;
+  if (words == 0) return NVFP4_OK;
+  const int64_t blocks = (words + 255) / 256;
+  const int grid = static_cast<int>(blocks < 148 * 16 ? blocks : 148 * 16);
+  swizzle_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(src), static_cast<int>(rows),
+                                      static_cast<int>(kb), words, static_cast<uint32_t*>(dst));
+  return launch_status(cudaGetLastError());
+}
+
+}  // namespace nvfp4

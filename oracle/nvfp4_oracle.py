@@ -132,8 +132,12 @@ def amax(x_bits) -> np.float32:
 
 def global_scale(a) -> np.float32:
     """g = 2688 / amax in fp32 (encode direction: g = 1/s_global, s_global =
-    amax/(6*448) [P4 NVFP4]).  amax == 0 gives g = 1 (pages silent)."""
+    amax/(6*448) [P4 NVFP4]).  amax == 0 gives g = 1 (pages silent).  A
+    non-finite amax or g is an error (pages silent: the tensor has no
+    finite two-level encoding)."""
     a = np.float32(a)
+    if not np.isfinite(a):
+        raise RangeError(f"amax is not finite ({float(a)!r})")
     if a == 0:
         return np.float32(1.0)
     with np.errstate(over="ignore", divide="ignore", invalid="ignore"):

@@ -1,0 +1,58 @@
+"""Helpers shared by the GPU parity tests: device transfer of seeded inputs
+and the acceptance rules.
+
+Acceptance (written here once, used by every GEMM/GEMV test):
+  * codes, block scales, g and amax: bit-exact;
+  * fp32 output: |D - D_ref| <= 2^-20 * alpha * S per element, S = sum_k |a_k b_k|;
+  * bf16 output: within 1 bf16 ulp of bf16_rne(D_ref), or, where the pre-cast
+    bound itself spans more than that (heavy cancellation, |D_ref| << alpha*S),
+    |D - D_ref| <= 2^-20 * alpha * S + ulp_bf16(D)/2 (the pre-cast bound
+    carried through one rounding to bf16).
+"""
+import numpy as np
+import torch
+
+from oracle import nvfp4_oracle as O
+
+BOUND = 2.0 ** -20
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    """uint16 bf16 bit patterns (numpy) -> torch bf16 tensor on cuda:0."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.bfloat16).cuda()
+
+
+def host_u8(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy().astype(np.uint8)
+
+
+def host_bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def f32_scalar(t: torch.Tensor) -> np.float32:
+    return np.float32(t.detach().cpu().numpy().reshape(-1)[0])
+
+
+def check_f32(d_gpu: np.ndarray, d_ref: np.ndarray, s_ref: np.ndarray, alpha) -> None:
+    lim = BOUND * np.float64(alpha) * s_ref
+    err = np.abs(d_gpu.astype(np.float64) - d_ref)
+    bad = np.nonzero(err > lim)
+    assert bad[0].size == 0, (
+        f"{bad[0].size} fp32 outputs outside 2^-20*alpha*S; worst ratio {np.max(err / np.maximum(lim, 1e-300)):.3g}")
+
+
+def check_bf16(y_bits: np.ndarray, d_ref: np.ndarray, s_ref: np.ndarray, alpha) -> int:
+    """Returns how many elements needed the carried pre-cast bound."""
+    ref_bits = O.f64_to_bf16_rne(d_ref)
+    ulps = np.abs(O.bf16_ordinal(y_bits) - O.bf16_ordinal(ref_bits))
+    y = O.bf16_to_f32(y_bits).astype(np.float64)
+    _, e = np.frexp(np.where(y == 0, 1.0, y))
+    half_ulp = np.ldexp(1.0, np.maximum(e, -125) - 9)          # bf16 has 8 significant bits
+    carried = np.abs(y - d_ref) <= BOUND * np.float64(alpha) * s_ref + half_ulp
+    ok = (ulps <= 1) | carried
+    bad = np.nonzero(~ok)
+    assert bad[0].size == 0, (
+        f"{bad[0].size} bf16 outputs off; e.g. got {y[bad][:4]} want {d_ref[bad][:4]} ulps {ulps[bad][:4]}")
+    return int(np.count_nonzero((ulps > 1) & carried))

@@ -1,0 +1,166 @@
+"""Block-scaled GEMM parity: the tcgen05 GEMM against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4_oracle as O
+from nvfp4_block_scaled_15_b200 import inputs
+from parity import check_bf16, check_f32, dev_bf16, f32_scalar, host_bf16_bits, host_u8
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(lib, a_bits, b_bits, out_dtype):
+    qa = lib.quantize(dev_bf16(a_bits), lib.SF_TCGEN05)
+    qb = lib.quantize(dev_bf16(b_bits), lib.SF_TCGEN05)
+    d = lib.gemm(qa, qb, out_dtype=out_dtype)
+    assert lib.nvfp4_check_device_status() == lib.OK
+    return qa, qb, d
+
+
+def _oracle(a_bits, b_bits):
+    pa, sa, ga, _ = O.quantize(a_bits)
+    pb, sb, gb, _ = O.quantize(b_bits)
+    return O.gemm_ref(pa, sa, ga, pb, sb, gb)
+
+
+def test_tiny_end_to_end_config(lib):
+    """A [128,256] and W [256,256] N(0,1): quantize both, GEMM, fp32 and bf16 out."""
+    a, w = inputs.tiny_end_to_end()
+    d_ref, s_ref, alpha = _oracle(a, w)
+    _, _, d32 = _run(lib, a, w, torch.float32)
+    check_f32(d32.cpu().numpy(), d_ref, s_ref, alpha)
+    _, _, d16 = _run(lib, a, w, torch.bfloat16)
+    check_bf16(host_bf16_bits(d16), d_ref, s_ref, alpha)
+
+
+RAGGED = [
+    (1, 1, 64),          # one element, one MMA
+    (200, 136, 320),     # M and N tails, a 1-MMA last K stage
+    (129, 257, 512),     # tails past one tile in both directions
+    (300, 100, 1024),    # N <= 128 path
+    (128, 384, 2048),    # N tile at 256 + a 128-wide tail tile
+    (64, 512, 8192),     # long K
+    (2048, 2560, 256),   # more tiles than SMs (persistent loop)
+]
+
+
+@pytest.mark.parametrize("m,n,k", RAGGED, ids=lambda v: str(v))
+def test_gemm_shapes(lib, m, n, k):
+    a = inputs.activations_with_outliers(m, k, seed=m + k, fraction=0.01, factor=30.0)
+    b = inputs.gaussian_bf16((n, k), seed=n + 2 * k, std=0.02)
+    d_ref, s_ref, alpha = _oracle(a, b)
+    _, _, d32 = _run(lib, a, b, torch.float32)
+    check_f32(d32.cpu().numpy(), d_ref, s_ref, alpha)
+    _, _, d16 = _run(lib, a, b, torch.bfloat16)
+    check_bf16(host_bf16_bits(d16), d_ref, s_ref, alpha)
+
+
+def test_gemm_output_pitch(lib):
+    a = inputs.gaussian_bf16((130, 256), seed=91)
+    b = inputs.gaussian_bf16((140, 256), seed=92)
+    d_ref, s_ref, alpha = _oracle(a, b)
+    qa = lib.quantize(dev_bf16(a), lib.SF_TCGEN05)
+    qb = lib.quantize(dev_bf16(b), lib.SF_TCGEN05)
+    big = torch.full((130, 160), -7.0, dtype=torch.bfloat16, device="cuda")
+    lib.nvfp4_gemm(qa.codes, qa.sf, qa.g, qb.codes, qb.sf, qb.g, 130, 140, 256, big, 160, lib.OUT_BF16)
+    torch.cuda.synchronize()
+    check_bf16(host_bf16_bits(big[:, :140]), d_ref, s_ref, alpha)
+    assert torch.all(big[:, 140:] == -7.0)
+
+
+def _probe(lib, m, n, k, a_sf_rowmajor, b_sf_rowmajor):
+    """GEMM of all-ones codes (E2M1 1.0 = code 2) with given row-major scales, g = 1."""
+    codes_a = torch.full((m, k // 2), 0x22, dtype=torch.uint8, device="cuda")
+    codes_b = torch.full((n, k // 2), 0x22, dtype=torch.uint8, device="cuda")
+    sfa = torch.empty(lib.nvfp4_sf_bytes(m, k, lib.SF_TCGEN05), dtype=torch.uint8, device="cuda")
+    sfb = torch.empty(lib.nvfp4_sf_bytes(n, k, lib.SF_TCGEN05), dtype=torch.uint8, device="cuda")
+    lib.nvfp4_swizzle_sf(torch.from_numpy(a_sf_rowmajor).cuda(), m, k, sfa)
+    lib.nvfp4_swizzle_sf(torch.from_numpy(b_sf_rowmajor).cuda(), n, k, sfb)
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    d = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    lib.nvfp4_gemm(codes_a, sfa, one, codes_b, sfb, one, m, n, k, d, n, lib.OUT_F32)
+    torch.cuda.synchronize()
+    return d.cpu().numpy()
+
+
+@pytest.mark.parametrize("side", ["a", "b"])
+def test_scale_layout_probes(lib, side):
+    """Exactly one (row, block) scale is 2.0, all others 1.0: only the D entries
+    of that row (A side) or column (B side) grow, by exactly 16 (one block of
+    16 products 1 x 1).  Pins the tensor-core scale layout end to end."""
+    m, n, k = 256, 256, 512
+    kb = k // 16
+    for row, blk in [(0, 0), (37, 5), (77, 18), (100, 31), (161, 9), (255, 30)]:
+        sa = np.full((m, kb), 0x38, np.uint8)
+        sb = np.full((n, kb), 0x38, np.uint8)
+        (sa if side == "a" else sb)[row, blk] = 0x40
+        d = _probe(lib, m, n, k, sa, sb)
+        want = np.full((m, n), float(k))
+        if side == "a":
+            want[row, :] += 16.0
+        else:
+            want[:, row] += 16.0
+        assert np.array_equal(d, want), (side, row, blk, np.argwhere(d != want)[:4].tolist())
+
+
+def test_gemm_prefill_full_size_sampled(lib):
+    """Prefill workload 8192^3 (activations with 0.5% outlier channels x30,
+    weights N(0, 0.02)): 512 sampled outputs against the oracle, the codes of
+    the sampled rows bit-exact, and no non-finite output anywhere."""
+    a, w = inputs.prefill_gemm()
+    qa = lib.quantize(dev_bf16(a), lib.SF_TCGEN05)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    d = lib.gemm(qa, qw, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    assert torch.isfinite(d).all()
+    ga = O.global_scale(O.amax(a))
+    gw = O.global_scale(O.amax(w))
+    assert f32_scalar(qa.g) == ga and f32_scalar(qw.g) == gw
+    rng = np.random.default_rng(23)
+    rows = rng.choice(8192, 512)
+    cols = rng.choice(8192, 512)
+    ur, uc = np.unique(rows), np.unique(cols)
+    ca, sa = O.quantize_with_scale(a[ur], ga)
+    cw, sw = O.quantize_with_scale(w[uc], gw)
+    assert np.array_equal(host_u8(qa.codes)[ur], O.pack_codes(ca))
+    assert np.array_equal(host_u8(qw.codes)[uc], O.pack_codes(cw))
+    ri = np.searchsorted(ur, rows)
+    ci = np.searchsorted(uc, cols)
+    d_ref, s_ref, alpha = O.gemm_ref_entries(O.pack_codes(ca), sa, ga, O.pack_codes(cw), sw, gw, ri, ci)
+    got = host_bf16_bits(d)[rows, cols]
+    check_bf16(got, d_ref, s_ref, alpha)
+
+
+def test_gemm_quant_a_small(lib):
+    m, n, k = 200, 136, 640
+    a = inputs.silu_gated_bf16(m, k, seed_a=81, seed_b=82)
+    w = inputs.gaussian_bf16((n, k), seed=83, std=0.02)
+    d_ref, s_ref, alpha = _oracle(a, w)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    d = lib.gemm_quant_a(dev_bf16(a), qw, out_dtype=torch.float32)
+    assert lib.nvfp4_check_device_status() == lib.OK
+    check_f32(d.cpu().numpy(), d_ref, s_ref, alpha)
+
+
+def test_gemm_quant_a_long_k_full_size_sampled(lib):
+    """Long-K workload: A [4096, 28672] = a*silu(b) quantized inside the call,
+    W [8192, 28672] N(0, 0.02) pre-quantized; 256 sampled outputs."""
+    a, w = inputs.long_k()
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    d = lib.gemm_quant_a(dev_bf16(a), qw, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    assert torch.isfinite(d).all()
+    ga = O.global_scale(O.amax(a))
+    gw = O.global_scale(O.amax(w))
+    rng = np.random.default_rng(29)
+    rows = rng.choice(a.shape[0], 256)
+    cols = rng.choice(w.shape[0], 256)
+    ur, uc = np.unique(rows), np.unique(cols)
+    ca, sa = O.quantize_with_scale(a[ur], ga)
+    cw, sw = O.quantize_with_scale(w[uc], gw)
+    d_ref, s_ref, alpha = O.gemm_ref_entries(O.pack_codes(ca), sa, ga, O.pack_codes(cw), sw, gw,
+                                             np.searchsorted(ur, rows), np.searchsorted(uc, cols))
+    check_bf16(host_bf16_bits(d)[rows, cols], d_ref, s_ref, alpha)

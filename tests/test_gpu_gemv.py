@@ -1,0 +1,59 @@
+"""Decode batched GEMV parity (activations quantized inside the call)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4_oracle as O
+from nvfp4_block_scaled_15_b200 import inputs
+from parity import check_bf16, dev_bf16, host_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("m", [1, 3, 8, 16, 32])
+@pytest.mark.parametrize("n,k", [(1000, 1024), (128, 64), (384, 4096)], ids=lambda v: str(v))
+def test_gemv_matches_oracle(lib, m, n, k):
+    x = inputs.gaussian_bf16((m, k), seed=300 + m)
+    w = inputs.gaussian_bf16((n, k), seed=400 + n, std=0.02)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    y = lib.gemv_batched(dev_bf16(x), qw)
+    assert lib.nvfp4_check_device_status() == lib.OK
+    px, sx, gx, _ = O.quantize(x)
+    pw, sw, gw, _ = O.quantize(w)
+    d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, pw, sw, gw)
+    check_bf16(host_bf16_bits(y), d_ref, s_ref, alpha)
+
+
+def test_gemv_repeated_calls_reuse_workspace(lib):
+    """The workspace is re-initialised by every call: two calls, same answer."""
+    m, n, k = 8, 640, 512
+    x = inputs.gaussian_bf16((m, k), seed=501)
+    w = inputs.gaussian_bf16((n, k), seed=502, std=0.02)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    ws = torch.empty(lib.nvfp4_workspace_bytes(lib.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device="cuda")
+    xd = dev_bf16(x)
+    y1 = lib.gemv_batched(xd, qw, workspace=ws).clone()
+    y2 = lib.gemv_batched(xd, qw, workspace=ws)
+    px, sx, gx, _ = O.quantize(x)
+    pw, sw, gw, _ = O.quantize(w)
+    d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, pw, sw, gw)
+    check_bf16(host_bf16_bits(y1), d_ref, s_ref, alpha)
+    check_bf16(host_bf16_bits(y2), d_ref, s_ref, alpha)
+
+
+@pytest.mark.parametrize("m", [1, 8, 16])
+def test_gemv_decode_full_size_sampled(lib, m):
+    """Decode workload: W [28672, 8192] N(0,0.02) pre-quantized, x [M, 8192]
+    N(0,1); 512 sampled output columns per row against the oracle."""
+    x, w = inputs.decode_gemv(m)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    y = lib.gemv_batched(dev_bf16(x), qw)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    assert torch.isfinite(y).all()
+    gw = O.global_scale(O.amax(w))
+    px, sx, gx, _ = O.quantize(x)
+    cols = np.sort(np.random.default_rng(37).choice(w.shape[0], 512, replace=False))
+    cw, sw = O.quantize_with_scale(w[cols], gw)
+    d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, O.pack_codes(cw), sw, gw)
+    check_bf16(host_bf16_bits(y)[:, cols], d_ref, s_ref, alpha)
