@@ -1,0 +1,464 @@
+#!/usr/bin/env python3
+"""Benchmark of the NVFP4 hot path on B200.
+
+One step = the prefill linear-layer path on the 8192 x 8192 x 8192 workload
+(activations bf16 [8192, 8192] N(0,1) with 0.5% outlier channels x30,
+weights N(0, 0.02)): quantize the activations (amax pass + quantize pass,
+scales written in the tensor-core layout) and run the block-scaled GEMM
+against the pre-quantized weights, bf16 output.  value = 2*M*N*K per step
+over the device time of the step, summed over ranks (weak scaling: every
+rank runs its own replica; the path needs no exchange).
+
+Also reported on rank 0: the GEMM kernel's roofline (live CUDA events),
+end-to-end throughput through host buffers, the quantize-bandwidth,
+decode-GEMV and long-K workloads, SM clocks during the timed region, and
+the CPU oracle timed on a bounded sample of the same workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_block_scaled_15_b200 import inputs  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS & fraction of FP4 peak; quantize/GEMV GB/s vs HBM"
+M = N = K = 8192
+FLOPS_STEP = 2.0 * M * N * K
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0            # nominal dense ratio (9 PFLOP/s FP4 : 2.25 PFLOP/s BF16)
+GEMM_SOURCES = ["gemm.cu", "ptx.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_15_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(summary_name, src_files):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        info = json.load(f)
+    if info.get("source_hash") != kernel_source_hash(src_files):
+        return None
+    return info.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []          # (t, sm_mhz, reasons_bitmask)
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _reasons(self):
+        nv = self._nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return getattr(nv, fn)(self._h)
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM)
+                self.samples.append((time.perf_counter(), mhz, int(self._reasons())))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join(timeout=2)
+
+    def summary(self, t0, t1):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        timed = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = timed if len(timed) >= 3 else self.samples
+        bits = 0
+        for s in use:
+            bits |= s[2]
+        return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(v for k, v in _REASONS.items() if bits & k),
+                "samples": len(use), "window": "timed" if use is timed else "warmup+timed"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """The prefill step restated by the oracle on a slice: tensor amax of the
+    full activations, quantization of ``rows`` activation rows, and the fp64
+    block-scaled GEMM of those rows against ``cols`` pre-quantized weight rows."""
+
+    def __init__(self, a_bits, w_bits, rows, cols):
+        from oracle import nvfp4_oracle as O
+        self.O = O
+        self.a = a_bits
+        self.rows, self.cols = rows, cols
+        gw = O.global_scale(O.amax(w_bits))
+        cw, sw = O.quantize_with_scale(w_bits[:cols], gw)
+        self.w = (O.pack_codes(cw), sw, gw)
+
+    def step(self):
+        O = self.O
+        ga = O.global_scale(O.amax(self.a))
+        ca, sa = O.quantize_with_scale(self.a[:self.rows], ga)
+        d, s, alpha = O.gemm_ref(O.pack_codes(ca), sa, ga, *self.w)
+        return d
+
+    def flops(self):
+        return 2.0 * self.rows * self.cols * K
+
+
+def time_oracle(sample: OracleSample, reps: int = 1):
+    t = time.perf_counter()
+    for _ in range(reps):
+        sample.step()
+    return (time.perf_counter() - t) / reps
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    a, w = inputs.prefill_gemm()
+    sample = OracleSample(a, w, rows=256, cols=512)
+    for _ in range(args.warmup):
+        sample.step()
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        sample.step()
+        times.append(time.perf_counter() - t)
+    sec = statistics.mean(times)
+    value = sample.flops() / sec / 1e12
+    desc = (f"oracle prefill step on a slice: amax of A [8192,8192], quantize {sample.rows} rows of A, "
+            f"fp64 GEMM against {sample.cols} pre-quantized weight rows (K=8192)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(n_gpus):
+    return {"workload": "prefill GEMM 8192x8192x8192: activation quantize (amax + quantize, tcgen05 scale "
+                        "layout) + block-scaled NVFP4 GEMM, weights pre-quantized, bf16 out",
+            "M": M, "N": N, "K": K, "activations": "bf16 N(0,1), 0.5% outlier channels x30, seed 4",
+            "weights": "bf16 N(0,0.02), seed 5", "l2": "flushed before every step (256 MiB write)",
+            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    # host inputs first (the generator's process pool starts before CUDA)
+    a_bits, w_bits = inputs.prefill_gemm()
+    parts_inputs = None
+    if rank == 0 and not args.no_parts:
+        parts_inputs = {"quant": inputs.quantize_bandwidth(),
+                        "gemv": inputs.decode_gemv(16),
+                        "longk": inputs.long_k()}
+
+    import torch
+    import torch.distributed as dist
+    from nvfp4_block_scaled_15_b200 import nvfp4 as nv
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    peaks, peaks_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    hbm_peak = peaks["hbm_gbs"]
+
+    a = to_dev(a_bits)
+    w = to_dev(w_bits)
+    qw = nv.quantize(w, nv.SF_TCGEN05)
+    qa = nv.empty_quantized(M, K, nv.SF_TCGEN05, dev)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nv.quantize(a, nv.SF_TCGEN05, out=qa)
+        nv.gemm(qa, qw, out=d)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    assert nv.nvfp4_check_device_status() == nv.OK
+
+    sampler = ClockSampler(local).start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for e0, e1, e2 in ev:
+        flush.zero_()
+        e0.record(stream)
+        nv.quantize(a, nv.SF_TCGEN05, out=qa)
+        e1.record(stream)
+        nv.gemm(qa, qw, out=d)
+        e2.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t1 = time.perf_counter()
+    sampler.stop()
+    status = nv.nvfp4_check_device_status()
+    step_ms = [e0.elapsed_time(e2) for e0, e1, e2 in ev]
+    quant_ms = [e0.elapsed_time(e1) for e0, e1, e2 in ev]
+    gemm_ms = [e1.elapsed_time(e2) for e0, e1, e2 in ev]
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * FLOPS_STEP / (ms * 1e-3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if rank == 0:
+        e2e = bench_e2e(nv, torch, dev, a_bits, qw, qa, min(args.steps, 30))
+
+    result = None
+    if rank == 0:
+        gemm_avg = statistics.mean(gemm_ms)
+        achieved = FLOPS_STEP / (gemm_avg * 1e-3) / 1e12
+        traffic = profile_traffic("gemm_prefill_8192.json", GEMM_SOURCES)
+        result = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic", "config": config_block(world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp4_peak, "traffic": traffic,
+                         "kernel": "gemm_kernel<256> (tcgen05.mma kind::mxf4nvf4, 8192^3)",
+                         "peak_source": f"{peaks_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} "
+                                        "(nominal FP4:BF16 dense ratio)",
+                         "algorithmic": "2*M*N*K = 1.0995e12 FLOP per launch"},
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": sampler.summary(t0, t1),
+            "wall_ms_per_step": (t1 - t0) * 1e3 / args.steps,
+            "step_breakdown_ms": {"quantize_activations": statistics.mean(quant_ms), "gemm": gemm_avg},
+            "device_status": nv.nvfp4_status_string(status),
+        }
+    if rank == 0 and parts_inputs is not None:
+        result["parts"] = bench_parts(nv, torch, dev, flush, parts_inputs, hbm_peak, fp4_peak, peaks_src)
+        result["parts"]["gemm_only"] = {"tflops": result["roofline"]["achieved"],
+                                        "frac_fp4_peak": result["roofline"]["frac"]}
+    if rank == 0 and world == 1 and not args.no_cpu:
+        sample = OracleSample(a_bits, w_bits, rows=1024, cols=1024)
+        sec = time_oracle(sample)
+        result["cpu_baseline"] = {
+            "value": sample.flops() / sec / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"oracle prefill step on a slice: amax of A [8192,8192], quantize {sample.rows} rows, "
+                      f"fp64 GEMM against {sample.cols} pre-quantized weight rows, K=8192 "
+                      f"({sec:.1f} s on the host)"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def bench_e2e(nv, torch, dev, a_bits, qw, qa, steps):
+    a_host = torch.from_numpy(np.ascontiguousarray(a_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    d_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    a_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    d_dev = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        a_dev.copy_(a_host, non_blocking=True)
+        nv.quantize(a_dev, nv.SF_TCGEN05, out=qa)
+        nv.gemm(qa, qw, out=d_dev)
+        d_host.copy_(d_dev, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": FLOPS_STEP / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2}
+
+
+def _timed(torch, dev, flush, fn, reps):
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        flush.zero_()
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    return statistics.median(e0.elapsed_time(e1) for e0, e1 in ts)
+
+
+def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
+    out = {"peaks": f"{peaks_src}: HBM {hbm_peak} GB/s, FP4 {fp4_peak:.1f} TFLOP/s (bf16 x4)"}
+    reps = 20
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # quantize bandwidth [16384, 8192]
+    x = to_dev(pin["quant"])
+    rows, k = x.shape
+    q = nv.empty_quantized(rows, k, nv.SF_TCGEN05, dev)
+    ms_all = _timed(torch, dev, flush, lambda: nv.quantize(x, nv.SF_TCGEN05, out=q), reps)
+    ms_amax = _timed(torch, dev, flush, lambda: nv.nvfp4_amax(x, rows, k, k, q.amax), reps)
+    ms_q1 = _timed(torch, dev, flush, lambda: nv.nvfp4_quantize(x, rows, k, k, q.codes, q.sf, nv.SF_TCGEN05, q.g,
+                                                                q.amax, 1), reps)
+    two_pass = rows * k * 2 * 2 + rows * k // 2 + rows * k // 16
+    one_pass = rows * k * 2 + rows * k // 2 + rows * k // 16
+    out["quantize_16384x8192"] = {
+        "ms": ms_all, "gbs_two_pass": two_pass / ms_all / 1e6, "frac_hbm": two_pass / ms_all / 1e6 / hbm_peak,
+        "gbs_strict_one_read": one_pass / ms_all / 1e6,
+        "amax_ms": ms_amax, "amax_gbs": rows * k * 2 / ms_amax / 1e6,
+        "quantize_pass_ms": ms_q1, "quantize_pass_gbs": one_pass / ms_q1 / 1e6,
+        "quantize_pass_frac_hbm": one_pass / ms_q1 / 1e6 / hbm_peak}
+    del x, q
+
+    # decode GEMV: W [28672, 8192] pre-quantized, x [M, 8192] quantized in the call
+    xg, wg = pin["gemv"]
+    wq = nv.quantize(to_dev(wg), nv.SF_TCGEN05)
+    n, k = wg.shape
+    res = {}
+    for m in (1, 8, 16):
+        xm = to_dev(xg[:m])
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device=dev)
+        ms = _timed(torch, dev, flush, lambda: nv.gemv_batched(xm, wq, out=y, workspace=ws), reps)
+        algo = n * k // 2 + n * k // 16 + m * k * 2 + m * n * 2
+        res[f"M={m}"] = {"ms": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak,
+                         "algorithmic_bytes": algo}
+    out["gemv_28672x8192"] = res
+    del wq
+
+    # long-K: A [4096, 28672] bf16 quantized in the call, W [8192, 28672] pre-quantized
+    al, wl = pin["longk"]
+    am, k = al.shape
+    nn = wl.shape[0]
+    wq = nv.quantize(to_dev(wl), nv.SF_TCGEN05)
+    ad = to_dev(al)
+    dd = torch.empty((am, nn), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, am, nn, k), dtype=torch.uint8, device=dev)
+    ms = _timed(torch, dev, flush, lambda: nv.gemm_quant_a(ad, wq, out=dd, workspace=ws), 10)
+    fl = 2.0 * am * nn * k
+    out["long_k_4096x8192x28672"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_fp4_peak": fl / ms / 1e9 / fp4_peak}
+    assert nv.nvfp4_check_device_status() == nv.OK
+    return out
+
+
+if __name__ == "__main__":
+    main()

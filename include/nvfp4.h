@@ -38,8 +38,9 @@
  *     read and cleared by nvfp4_check_device_status().
  *   - Codes are dense: row r of a [rows, K] code matrix starts at byte
  *     r * K / 2.  bf16 inputs have a row pitch ld (in elements).
- *   - Pointers must be 16-byte aligned and ld must keep every row 16-byte
- *     aligned (ld % 8 == 0).
+ *   - Input and code/scale pointers must be 16-byte aligned and the bf16
+ *     input pitch must keep every row 16-byte aligned (ld % 8 == 0).  Output
+ *     pointers need only element alignment.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
@@ -144,8 +145,9 @@ NVFP4_API nvfp4_status nvfp4_swizzle_sf(const void* sf_rowmajor, int64_t rows, i
  * alpha = 1 / (g_a * g_b) computed in fp32 from *g_a_dev and *g_b_dev.
  *   a_codes [M, K/2], a_sf_tc TCGEN05 scales of A, g_a_dev one fp32 (encode scale of A)
  *   b_codes [N, K/2], b_sf_tc TCGEN05 scales of B, g_b_dev one fp32
- *   d: out, [M, N] with row pitch ldd elements, bf16 (round to nearest even)
- *      or fp32 per out_dtype.
+ *   d: out, [M, N] with row pitch ldd >= N elements, bf16 (round to nearest
+ *      even) or fp32 per out_dtype; element-aligned (16-byte aligned rows get
+ *      vector stores, other pitches element stores).
  * K % 64 == 0, K > 0, M, N >= 1 (any value; tails are masked).
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_sf_tc, const float* g_a_dev, const void* b_codes,

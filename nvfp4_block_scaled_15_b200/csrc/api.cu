@@ -187,7 +187,7 @@ static nvfp4_status check_gemm_operands(const void* a_codes, const void* a_sf, c
   if (!a_codes || !a_sf || !g_a || !b_codes || !b_sf || !g_b || !d) return NVFP4_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1) return NVFP4_ERR_INVALID_ARG;
   if ((K % 64) != 0 || M > 0x7FFFFF80 || N > 0x7FFFFF80 || K > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_sf) || !aligned16(b_sf) || !aligned16(d))
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_sf) || !aligned16(b_sf))
     return NVFP4_ERR_MISALIGNED;
   return NVFP4_OK;
 }
@@ -199,8 +199,7 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_sf_tc, const float* g
   if (st != NVFP4_OK) return st;
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
   if (ldd < N) return NVFP4_ERR_INVALID_ARG;
-  if ((out_dtype == NVFP4_OUT_BF16 && (ldd % 8) != 0) || (out_dtype == NVFP4_OUT_F32 && (ldd % 4) != 0))
-    return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(d) & (out_dtype == NVFP4_OUT_F32 ? 3u : 1u)) != 0) return NVFP4_ERR_MISALIGNED;
   if ((st = check_arch()) != NVFP4_OK) return st;
   return launch_gemm(a_codes, a_sf_tc, g_a_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype,
                      reinterpret_cast<cudaStream_t>(stream));
@@ -257,8 +256,7 @@ nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_c
   if (st != NVFP4_OK) return st;
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
   if (ldd < N) return NVFP4_ERR_INVALID_ARG;
-  if ((out_dtype == NVFP4_OUT_BF16 && (ldd % 8) != 0) || (out_dtype == NVFP4_OUT_F32 && (ldd % 4) != 0))
-    return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(d) & (out_dtype == NVFP4_OUT_F32 ? 3u : 1u)) != 0) return NVFP4_ERR_MISALIGNED;
   if ((st = check_arch()) != NVFP4_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = launch_amax(a_bf16, M, K, lda, amax_a, s)) != NVFP4_OK) return st;

@@ -72,6 +72,7 @@ struct GemmParams {
   int kb4;          // scale atoms along K per 128-row group (= K / 64)
   int tiles_m, tiles_n;
   int out_f32;
+  int vec_store;    // rows of D are 16-byte aligned: vector stores allowed
   uint64_t wait_limit_ns;
   int* status;
 };
@@ -98,7 +99,7 @@ __device__ __forceinline__ void store_row(const GemmParams& p, int row, int col0
   if (row >= p.M) return;
   if (p.out_f32) {
     float* out = static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + col0;
-    if (col0 + NV <= p.N) {
+    if (p.vec_store && col0 + NV <= p.N) {
 #pragma unroll
       for (int i = 0; i < NV; i += 4) {
         float4 f = make_float4(__uint_as_float(v[i]) * alpha, __uint_as_float(v[i + 1]) * alpha,
@@ -112,7 +113,7 @@ __device__ __forceinline__ void store_row(const GemmParams& p, int row, int col0
     }
   } else {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + col0;
-    if (col0 + NV <= p.N) {
+    if (p.vec_store && col0 + NV <= p.N) {
 #pragma unroll
       for (int i = 0; i < NV; i += 8) {
         uint4 w;
@@ -667,6 +668,8 @@ nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, c
   p.tiles_m = static_cast<int>((M + BM - 1) / BM);
   p.tiles_n = static_cast<int>((N + BN - 1) / BN);
   p.out_f32 = out == NVFP4_OUT_F32;
+  const int64_t row_bytes = ldd * (p.out_f32 ? 4 : 2);
+  p.vec_store = aligned16(d) && (row_bytes % 16) == 0;
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;

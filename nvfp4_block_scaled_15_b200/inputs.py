@@ -53,19 +53,40 @@ def normal(seed: int, start: int, count: int, stream: int = 0) -> np.ndarray:
     return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
 
 
-def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
-    """Round fp64 to bf16 (round-to-nearest-even, one rounding), as uint16 bits."""
-    v = np.asarray(v, dtype=np.float64)
-    out = np.empty(v.shape, dtype=np.uint16)
-    flat_v = v.reshape(-1)
-    flat_o = out.reshape(-1)
-    for s in range(0, flat_v.size, _CHUNK):
-        x = flat_v[s:s + _CHUNK]
-        mant, exp = np.frexp(x)                     # x = mant * 2**exp, 0.5 <= |mant| < 1
-        exp = np.maximum(exp, -125)                 # bf16 subnormal quantum is 2**-133
-        q = np.rint(np.ldexp(x, 8 - exp))           # 8 significant bits, ties to even
+def _f64_to_bf16_slow(x: np.ndarray) -> np.ndarray:
+    mant, exp = np.frexp(x)                     # x = mant * 2**exp, 0.5 <= |mant| < 1
+    exp = np.maximum(exp, -125)                 # bf16 subnormal quantum is 2**-133
+    q = np.rint(np.ldexp(x, 8 - exp))           # 8 significant bits, ties to even
+    with np.errstate(over="ignore"):
         y = np.ldexp(q, exp - 8).astype(np.float32)  # exact: y has <= 8 significant bits
-        flat_o[s:s + _CHUNK] = (y.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    return (y.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round fp64 to bf16 (round-to-nearest-even, one rounding), as uint16 bits.
+
+    Works on the fp64 bit pattern: keep 7 of the 52 fraction bits, round the
+    other 45 to nearest-even, re-bias the exponent.  Values outside the bf16
+    normal range (zero, subnormal, overflow) take a frexp-based path.
+    """
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    bits = v.view(np.uint64)
+    sign = (bits >> np.uint64(63)).astype(np.uint16)
+    exp = ((bits >> np.uint64(52)) & np.uint64(0x7FF)).astype(np.int64)
+    frac = bits & np.uint64((1 << 52) - 1)
+    keep = (frac >> np.uint64(45)).astype(np.int64)
+    rest = frac & np.uint64((1 << 45) - 1)
+    half = np.uint64(1 << 44)
+    up = (rest > half) | ((rest == half) & ((keep & 1) == 1))
+    keep = keep + up
+    exp = exp + (keep >> 7)
+    keep = keep & 127
+    bexp = exp - 1023 + 127
+    out = ((sign << np.uint16(15)) | (np.clip(bexp, 0, 255).astype(np.uint16) << np.uint16(7))
+           | keep.astype(np.uint16))
+    odd = (bexp <= 0) | (bexp >= 255)
+    if np.any(odd):
+        out[odd] = _f64_to_bf16_slow(v[odd])
     return out
 
 
@@ -74,14 +95,74 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+# ---------------------------------------------------------------------------
+# Chunked generation.  Every element depends only on (seed, stream, index),
+# so chunks can be produced in any order, serially or by a process pool.
+# ---------------------------------------------------------------------------
+_PARALLEL_MIN = 1 << 24        # elements; smaller tensors are generated serially
+
+
+def _chunk_values(kind: str, params: tuple, start: int, count: int) -> np.ndarray:
+    if kind == "gauss":
+        seed, std, stream = params
+        return f64_to_bf16_bits(std * normal(seed, start, count, stream))
+    if kind == "outlier":
+        seed, k, cols, factor = params
+        z = normal(seed, start, count)
+        is_out = np.zeros(k, dtype=bool)
+        is_out[cols] = True
+        col = np.arange(start, start + count, dtype=np.int64) % k
+        z = np.where(is_out[col], z * factor, z)
+        return f64_to_bf16_bits(z)
+    if kind == "silu":
+        seed_a, seed_b = params
+        a = normal(seed_a, start, count).astype(np.float32)
+        b = normal(seed_b, start, count).astype(np.float32)
+        silu = b / (np.float32(1.0) + np.exp(-b))
+        return f64_to_bf16_bits((a * silu).astype(np.float64))
+    raise ValueError(kind)
+
+
+def _worker_fill(shm_name: str, n: int, kind: str, params: tuple, start: int, count: int) -> None:
+    from multiprocessing import shared_memory
+    shm = shared_memory.SharedMemory(name=shm_name)
+    try:
+        out = np.ndarray((n,), dtype=np.uint16, buffer=shm.buf)
+        out[start:start + count] = _chunk_values(kind, params, start, count)
+        del out
+    finally:
+        shm.close()
+
+
+def _generate(kind: str, params: tuple, n: int) -> np.ndarray:
+    import os
+    workers = int(os.environ.get("NVFP4_GEN_WORKERS", "0")) or min(32, os.cpu_count() or 1)
+    if n < _PARALLEL_MIN or workers <= 1:
+        out = np.empty(n, dtype=np.uint16)
+        for s in range(0, n, _CHUNK):
+            c = min(_CHUNK, n - s)
+            out[s:s + c] = _chunk_values(kind, params, s, c)
+        return out
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    from multiprocessing import shared_memory
+    shm = shared_memory.SharedMemory(create=True, size=max(2, 2 * n))
+    try:
+        with ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn")) as ex:
+            futs = [ex.submit(_worker_fill, shm.name, n, kind, params, s, min(_CHUNK, n - s))
+                    for s in range(0, n, _CHUNK)]
+            for f in futs:
+                f.result()
+        return np.ndarray((n,), dtype=np.uint16, buffer=shm.buf).copy()
+    finally:
+        shm.close()
+        shm.unlink()
+
+
 def gaussian_bf16(shape, seed: int, std: float = 1.0, stream: int = 0) -> np.ndarray:
     """bf16 bits of ``std * N(0, 1)`` in row-major ``shape``."""
     n = int(np.prod(shape))
-    out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, _CHUNK):
-        c = min(_CHUNK, n - s)
-        out[s:s + c] = f64_to_bf16_bits(std * normal(seed, s, c, stream))
-    return out.reshape(shape)
+    return _generate("gauss", (seed, float(std), stream), n).reshape(shape)
 
 
 def outlier_columns(k: int, fraction: float, seed: int) -> np.ndarray:
@@ -102,28 +183,12 @@ def activations_with_outliers(rows: int, k: int, seed: int, fraction: float,
     The outlier columns are multiplied in fp64 before the single bf16 rounding.
     """
     cols = outlier_columns(k, fraction, seed)
-    scale = np.ones(k, dtype=np.float64)
-    scale[cols] = factor
-    out = np.empty((rows, k), dtype=np.uint16)
-    rows_per_chunk = max(1, _CHUNK // k)
-    for r in range(0, rows, rows_per_chunk):
-        rr = min(rows_per_chunk, rows - r)
-        z = normal(seed, r * k, rr * k).reshape(rr, k)
-        out[r:r + rr] = f64_to_bf16_bits(z * scale)
-    return out
+    return _generate("outlier", (seed, k, cols, float(factor)), rows * k).reshape(rows, k)
 
 
 def silu_gated_bf16(rows: int, k: int, seed_a: int, seed_b: int) -> np.ndarray:
     """bf16 bits of ``a * silu(b)`` with a, b ~ N(0,1); silu evaluated in fp32."""
-    out = np.empty((rows, k), dtype=np.uint16)
-    rows_per_chunk = max(1, _CHUNK // k)
-    for r in range(0, rows, rows_per_chunk):
-        rr = min(rows_per_chunk, rows - r)
-        a = normal(seed_a, r * k, rr * k).astype(np.float32)
-        b = normal(seed_b, r * k, rr * k).astype(np.float32)
-        silu = b / (np.float32(1.0) + np.exp(-b))
-        out[r:r + rr] = f64_to_bf16_bits((a * silu).astype(np.float64)).reshape(rr, k)
-    return out
+    return _generate("silu", (seed_a, seed_b), rows * k).reshape(rows, k)
 
 
 # --------------------------------------------------------------------------

@@ -77,7 +77,7 @@ def test_argument_errors_return_before_any_device_work(nv):
     assert raw("nvfp4_gemm", fake, fake, fake, fake, fake, fake, 8, 8, 96, fake, 8, 0, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert raw("nvfp4_gemm", fake, fake, fake, fake, fake, fake, 0, 8, 64, fake, 8, 0, None) == nv.ERR_INVALID_ARG
     assert raw("nvfp4_gemm", fake, fake, fake, fake, fake, fake, 8, 8, 64, fake, 4, 0, None) == nv.ERR_INVALID_ARG
-    assert raw("nvfp4_gemm", fake, fake, fake, fake, fake, fake, 8, 8, 64, fake, 12, 0, None) == nv.ERR_MISALIGNED
+    assert raw("nvfp4_gemm", fake, fake, fake, fake, fake, fake, 8, 8, 64, fake + 1, 12, 0, None) == nv.ERR_MISALIGNED
     assert raw("nvfp4_gemm", fake, fake, fake, fake + 4, fake, fake, 8, 8, 64, fake, 8, 0, None) == nv.ERR_MISALIGNED
     assert raw("nvfp4_gemv_batched", fake, 33, 64, fake, fake, fake, 128, 64, fake, 128, fake, 1 << 30, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert raw("nvfp4_gemv_batched", fake, 4, 64, fake, fake, fake, 128, 64, fake, 128, fake, 16, None) == nv.ERR_WORKSPACE
