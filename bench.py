@@ -72,15 +72,23 @@ def kernel_source_hash(files):
 
 
 def profile_traffic(summary_name, src_files):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    """DRAM bytes per launch from a committed ncu summary (``source_hash:`` and
+    ``dram_bytes_per_launch:`` lines), if it matches the current kernel source."""
     path = os.path.join(ROOT, "profiles", summary_name)
     if not os.path.exists(path):
         return None
+    info = {}
     with open(path) as f:
-        info = json.load(f)
+        for line in f:
+            if ":" in line and not line.startswith(("|", "#", " ")):
+                key, _, val = line.partition(":")
+                info[key.strip()] = val.strip()
     if info.get("source_hash") != kernel_source_hash(src_files):
         return None
-    return info.get("dram_bytes_per_launch")
+    try:
+        return int(info["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # ---------------------------------------------------------------------------
@@ -322,7 +330,7 @@ def main():
     if rank == 0:
         gemm_avg = statistics.mean(gemm_ms)
         achieved = FLOPS_STEP / (gemm_avg * 1e-3) / 1e12
-        traffic = profile_traffic("gemm_prefill_8192.json", GEMM_SOURCES)
+        traffic = profile_traffic("gemm_prefill_8192.md", GEMM_SOURCES)
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -345,7 +353,7 @@ def main():
         result["parts"]["gemm_only"] = {"tflops": result["roofline"]["achieved"],
                                         "frac_fp4_peak": result["roofline"]["frac"]}
     if rank == 0 and world == 1 and not args.no_cpu:
-        sample = OracleSample(a_bits, w_bits, rows=1024, cols=1024)
+        sample = OracleSample(a_bits, w_bits, rows=8192, cols=2048)
         sec = time_oracle(sample)
         result["cpu_baseline"] = {
             "value": sample.flops() / sec / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
