@@ -175,6 +175,31 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t
                                 int64_t ldy, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gemv_batched without a workspace argument, for callers that cannot
+ * allocate device memory: code that must not call the allocator (inside a
+ * CUDA graph capture, on a real-time path after start-up), or a plug-in whose
+ * host framework hands it only input and output buffers.  The pages have no
+ * counterpart of this entry point; it computes exactly what
+ * nvfp4_gemv_batched computes.
+ *   Scratch: a fixed 4 MiB array inside the library, present on every GPU
+ *     that loads it until the process exits.  Shapes whose workspace
+ *     (nvfp4_workspace_bytes(NVFP4_OP_GEMV_BATCHED, M, N, K)) exceeds 4 MiB
+ *     are rejected with NVFP4_ERR_WORKSPACE, before anything is enqueued;
+ *     M <= 16 with N <= 32768 and K <= 16384 always fits.
+ *   Set-up: the first call on a device (made with that device current) looks
+ *     up the scratch's device address; make that first call before any stream
+ *     capture.  Nothing is allocated or freed, then or later.
+ *   Sharing: every call on a device uses the same scratch and overwrites what
+ *     the previous call left there (each call clears what must start at
+ *     zero).  Calls that overlap on the device race: serialise them, e.g. on
+ *     one stream.
+ * Other arguments, constraints and errors as nvfp4_gemv_batched.
+ */
+NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M, int64_t ldx, const void* w_codes,
+                                const void* w_sf_tc, const float* g_w_dev, int64_t N, int64_t K,
+                                void* y_bf16, int64_t ldy, nvfp4_stream_t stream);
+
+/*
  * Long-K GEMM whose A operand arrives in bf16: A [M, K] (pitch lda) is
  * quantized to NVFP4 with the nvfp4_quantize rule (tensor amax first), then
  * multiplied by pre-quantized B as in nvfp4_gemm.

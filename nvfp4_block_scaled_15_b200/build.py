@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnvfp4.so")
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "gemv_noalloc.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "quant_core.cuh"]
 
 NVCC_FLAGS = [

@@ -50,6 +50,7 @@ _SIGS = {
     "nvfp4_workspace_bytes": ([_i32, _i64, _i64, _i64], _sz),
     "nvfp4_gemv_batched": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _sz, _vp], _i32),
     "nvfp4_gemm_quant_a": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp], _i32),
+    "nvfp4_gemv_batched_noalloc": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp], _i32),
     "nvfp4_check_device_status": ([_vp], _i32),
     "nvfp4_set_wait_limit_ns": ([_u64], None),
     "nvfp4_selftest_wait_timeout": ([_u64, _vp], _i32),
@@ -130,6 +131,12 @@ def nvfp4_gemm(a_codes, a_sf, g_a, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtyp
 def nvfp4_gemv_batched(x, m, ldx, w_codes, w_sf, g_w, n, k, y, ldy, workspace, ws_bytes, stream=None) -> None:
     _check(_lib.nvfp4_gemv_batched(_p(x), m, ldx, _p(w_codes), _p(w_sf), _p(g_w), n, k, _p(y), ldy,
                                    _p(workspace), ws_bytes, _s(stream)), "nvfp4_gemv_batched")
+
+
+def nvfp4_gemv_batched_noalloc(x, m, ldx, w_codes, w_sf, g_w, n, k, y, ldy, stream=None) -> None:
+    """nvfp4_gemv_batched on the library's fixed scratch (no workspace argument)."""
+    _check(_lib.nvfp4_gemv_batched_noalloc(_p(x), m, ldx, _p(w_codes), _p(w_sf), _p(g_w), n, k, _p(y), ldy,
+                                           _s(stream)), "nvfp4_gemv_batched_noalloc")
 
 
 def nvfp4_gemm_quant_a(a, lda, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, workspace, ws_bytes,
