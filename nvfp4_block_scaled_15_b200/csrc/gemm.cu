@@ -406,7 +406,37 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
-      for (int64_t u = u_begin; u < u_end; ++u) {
+      // weights do not depend on the prologue: fill the ring with them first
+      const int64_t pre_end = min(u_end, u_begin + GV_STAGES);
+      for (int64_t u = u_begin; u < pre_end; ++u) {
+        const int tile = static_cast<int>(u / p.num_kt);
+        const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+        const int nk = min(4, ksteps_total - kt * 4);
+        const int s = static_cast<int>(u - u_begin);
+        uint8_t* sA = smem + s * GV_STAGE_BYTES;
+        uint8_t* sSFA = sA + GV_A_BYTES + GV_B_BYTES;
+        mbar_arrive_expect_tx(&full[s], GV_A_BYTES + GV_B_BYTES + 2 * nk * SF_ATOM);
+        tma_load_2d(sA, &tmW, &full[s], kt * BK_BYTES, tile * BM);
+        bulk_load(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[s]);
+      }
+      // activations, their scales: only once the prologue grid has finished
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int64_t u = u_begin; u < pre_end; ++u) {
+        const int tile = static_cast<int>(u / p.num_kt);
+        const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+        const int nk = min(4, ksteps_total - kt * 4);
+        const int s = static_cast<int>(u - u_begin);
+        uint8_t* sB = smem + s * GV_STAGE_BYTES + GV_A_BYTES;
+        uint8_t* sSFB = sB + GV_B_BYTES + 4 * SF_ATOM;
+        tma_load_2d(sB, &tmX, &full[s], kt * BK_BYTES, 0);
+        bulk_load(sSFB, p.xsf + static_cast<int64_t>(kt) * 4 * SF_ATOM, nk * SF_ATOM, &full[s]);
+        issued_mask |= 1u << s;
+        if (++stage == GV_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      for (int64_t u = pre_end; u < u_end; ++u) {
         const int tile = static_cast<int>(u / p.num_kt);
         const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
@@ -491,6 +521,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     }
   } else {
     const int quad = warp & 3;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_w, *p.g_x));
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -546,10 +577,16 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 }
 
 // Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
-// clearing of the partial sums.  CTA 0 quantizes all M rows of x into 32
-// padded code rows and 128 padded scale rows; the other CTAs clear y32 and
-// the tile counters.
-constexpr int GP_THREADS = 1024;
+// clearing of the partial sums.  Grid = 128 + GP_ZERO_CTAS CTAs:
+//   CTA r < M        computes the amax of all M rows (x is small; each row CTA
+//                    reads it from L2) and quantizes row r;
+//   CTA M <= r < 128 writes zero codes (r < 32) and zero scales for padding row r;
+//   CTA >= 128       clears the fp32 partial sums and the tile counters.
+// It lets the dependent GEMV grid launch at once (programmatic dependent
+// launch): the GEMV streams weights while this runs and waits for it only
+// before it touches the activations, g_x or the partial sums.
+constexpr int GP_THREADS = 256;
+constexpr int GP_ZERO_CTAS = 16;
 
 __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                    int64_t ldx, uint8_t* __restrict__ xq,
@@ -557,58 +594,69 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
                                                                    float* __restrict__ y32, int64_t y32_words,
                                                                    int* __restrict__ counters, int n_counters,
                                                                    int* __restrict__ status) {
-  if (blockIdx.x > 0) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x - 1) * blockDim.x;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < y32_words; i += stride)
-      y32[i] = 0.0f;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n_counters; i += stride)
-      counters[i] = 0;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int chunks = K >> 3;                 // 16-B chunks per row (a multiple of 8)
+  const int kb = K >> 4;
+  if (b >= 128) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x - 128) * GP_THREADS;
+    for (int64_t i = static_cast<int64_t>(b - 128) * GP_THREADS + tid; i < y32_words; i += stride) y32[i] = 0.0f;
+    for (int64_t i = static_cast<int64_t>(b - 128) * GP_THREADS + tid; i < n_counters; i += stride) counters[i] = 0;
     return;
   }
-  const int chunks = K >> 3;                 // 16-B chunks per row
-  const int kb = K >> 4;
-  // pass 1: amax over the M real rows
-  uint32_t m = 0;
-  for (int64_t i = threadIdx.x; i < static_cast<int64_t>(M) * chunks; i += GP_THREADS) {
-    const int r = static_cast<int>(i / chunks);
-    const int c = static_cast<int>(i - static_cast<int64_t>(r) * chunks);
-    const uint4 v = *(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx) + c);
-    m = max(m, abs_max_bits8(v));
-  }
-  m = __reduce_max_sync(0xFFFFFFFFu, m);
-  __shared__ uint32_t red[GP_THREADS / 32];
-  __shared__ float g_sh;
-  __shared__ int valid_sh;
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    uint32_t t = red[threadIdx.x];
-    t = __reduce_max_sync(0xFFFFFFFFu, t);
-    if (threadIdx.x == 0) {
-      bool valid;
-      const float g = global_scale_from_amax(__uint_as_float(t << 16), valid);
-      g_sh = valid ? g : 0.0f;
-      valid_sh = valid;
-      *g_x = g_sh;
-      if (!valid) record_status(status, kDevRange);
+  const int r = b;
+  if (r >= M) {
+    if (r < GV_N) {
+      uint4* row = reinterpret_cast<uint4*>(xq + static_cast<int64_t>(r) * (K >> 1));
+      for (int c = tid; c < (K >> 5); c += GP_THREADS) row[c] = make_uint4(0, 0, 0, 0);
     }
+    for (int j = tid; j < (kb >> 2); j += GP_THREADS)
+      *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, 4 * j, kb)) = 0u;
+    return;
   }
+  // amax over the M real rows, 8 loads in flight per thread
+  constexpr int U = 8;
+  const int total = M * chunks;
+  uint32_t mx = 0;
+  for (int base = 0; base < total; base += U * GP_THREADS) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * GP_THREADS + tid;
+      if (i < total) {
+        const int rr = i / chunks;
+        const int c = i - rr * chunks;
+        v[u] = *(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(rr) * ldx) + c);
+      } else {
+        v[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) mx = max(mx, abs_max_bits8(v[u]));
+  }
+  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+  __shared__ uint32_t red[GP_THREADS / 32];
+  if (lane == 0) red[tid >> 5] = mx;
   __syncthreads();
-  const float g = g_sh;
-  const bool valid = valid_sh != 0;
-  // pass 2: 32 code rows (rows >= M are zero) and 128 scale rows (rows >= M zero)
-  const int lane = threadIdx.x & 31;
-  const int64_t items = static_cast<int64_t>(128) * chunks;   // whole warps, chunks % 8 == 0
-  for (int64_t i = threadIdx.x; i < items; i += GP_THREADS) {
-    const int r = static_cast<int>(i / chunks);
-    const int c = static_cast<int>(i - static_cast<int64_t>(r) * chunks);
-    const bool real = r < M && valid;
-    const uint4 v = real ? *(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx) + c)
-                         : make_uint4(0, 0, 0, 0);
+  uint32_t t = lane < GP_THREADS / 32 ? red[lane] : 0u;
+  t = __reduce_max_sync(0xFFFFFFFFu, t);
+  bool valid;
+  const float g = global_scale_from_amax(__uint_as_float(t << 16), valid);
+  if (r == 0 && tid == 0) {
+    *g_x = valid ? g : 0.0f;
+    if (!valid) record_status(status, kDevRange);
+  }
+  // quantize row r: every warp covers 32 consecutive chunks (16 blocks)
+  const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
+  uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1));
+  for (int c = tid; c < chunks; c += GP_THREADS) {
+    const uint4 v = valid ? row[c] : make_uint4(0, 0, 0, 0);
     uint32_t s;
-    uint32_t q = quantize_half_block(v, real ? g : 0.0f, s);
-    if (!real) { q = 0; s = 0; }
-    if (r < GV_N) reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1))[c] = q;
+    uint32_t q = quantize_half_block(v, valid ? g : 0.0f, s);
+    if (!valid) { q = 0; s = 0; }
+    qrow[c] = q;
     const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
     const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
     const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
@@ -724,9 +772,9 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
 
   int* status = device_status_ptr();
   if (!status) return NVFP4_ERR_CUDA;
-  gemv_prologue_kernel<<<sms, GP_THREADS, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(M),
-                                                  static_cast<int>(K), ldx, xq, xsf, gx, y32, M * N, cnt, tiles * 4,
-                                                  status);
+  gemv_prologue_kernel<<<128 + GP_ZERO_CTAS, GP_THREADS, 0, s>>>(
+      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), ldx, xq, xsf, gx, y32, M * N, cnt,
+      tiles * 4, status);
   nvfp4_status st = launch_status(cudaGetLastError());
   if (st != NVFP4_OK) return st;
 
@@ -754,8 +802,18 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
   const int grid = static_cast<int>(units < sms ? units : sms);
   cudaError_t e = cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_BYTES);
   if (e != cudaSuccess) return launch_status(e);
-  gemv_kernel<<<grid, GV_THREADS, GV_SMEM_BYTES, s>>>(tmW, tmX, p);
-  return launch_status(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(GV_THREADS);
+  cfg.dynamicSmemBytes = GV_SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemv_kernel, tmW, tmX, p);
+  return launch_status(e);
 }
 
 }  // namespace nvfp4

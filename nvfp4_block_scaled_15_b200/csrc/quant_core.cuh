@@ -46,6 +46,17 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   return out;
 }
 
+// RN(t / d) given y = RN(1 / d): q = RN(t * y); r = t - q * d is exact with
+// one FMA; RN(q + r * y) equals RN(t / d) (Markstein's theorem on FMA-based
+// division, P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  A zero quotient
+// takes the sign of t, as t / d would.
+__device__ __forceinline__ float div_rn_by_recip(float t, float d, float y) {
+  const float q = __fmul_rn(t, y);
+  const float r = __fmaf_rn(-q, d, t);
+  return copysignf(__fmaf_rn(r, y, q), t);
+}
+
 // One half block: 8 bf16 in v.  Returns the 4 code bytes (element 0 in the
 // low nibble of byte 0) and, through sf, the block's E4M3 scale byte.  Every
 // lane of the warp must call this (it shuffles with lane ^ 1).
@@ -59,12 +70,13 @@ __device__ __forceinline__ uint32_t quantize_half_block(const uint4 v, const flo
   const __half_raw hs = __nv_cvt_fp8_to_halfraw(s8, __NV_E4M3);
   const float sd = __half2float(__half(hs));
   if (sd == 0.0f) return 0u;
+  const float y = __frcp_rn(sd);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float u0 = __fdiv_rn(__fmul_rn(bf16_lo(w[i]), g), sd);
-    const float u1 = __fdiv_rn(__fmul_rn(bf16_hi(w[i]), g), sd);
+    const float u0 = div_rn_by_recip(__fmul_rn(bf16_lo(w[i]), g), sd, y);
+    const float u1 = div_rn_by_recip(__fmul_rn(bf16_hi(w[i]), g), sd, y);
     out |= e2m1x2(u0, u1) << (8 * i);
   }
   return out;
