@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--part", choices=["quantize", "gemv", "longk", "gemm"], default=None,
+                    help="run one workload alone, --steps times (for profiling); prints its timing")
     return ap.parse_args()
 
 
@@ -248,6 +250,9 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
+    if args.part:
+        run_part(args)
+        return
 
     # host inputs first (the generator's process pool starts before CUDA)
     a_bits, w_bits = inputs.prefill_gemm()
@@ -337,7 +342,7 @@ def main():
             "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic", "config": config_block(world),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp4_peak, "traffic": traffic,
-                         "kernel": "gemm_kernel<256> (tcgen05.mma kind::mxf4nvf4, 8192^3)",
+                         "kernel": "gemm_pair_kernel (tcgen05.mma.cta_group::2 kind::mxf4nvf4, 256x256 tiles, 8192^3)",
                          "peak_source": f"{peaks_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} "
                                         "(nominal FP4:BF16 dense ratio)",
                          "algorithmic": "2*M*N*K = 1.0995e12 FLOP per launch"},
@@ -466,6 +471,55 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
     out["long_k_4096x8192x28672"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_fp4_peak": fl / ms / 1e9 / fp4_peak}
     assert nv.nvfp4_check_device_status() == nv.OK
     return out
+
+
+def run_part(args):
+    """One workload alone: generate its inputs, run it ``--steps`` times with the
+    L2 flushed in between, print the median time."""
+    if args.part == "quantize":
+        x_bits = inputs.quantize_bandwidth()
+    elif args.part == "gemv":
+        xg, wg = inputs.decode_gemv(16)
+    elif args.part == "longk":
+        al, wl = inputs.long_k()
+    else:
+        a_bits, w_bits = inputs.prefill_gemm()
+    import torch
+    from nvfp4_block_scaled_15_b200 import nvfp4 as nv
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    out = {"part": args.part}
+    if args.part == "quantize":
+        x = to_dev(x_bits)
+        q = nv.empty_quantized(*x.shape, nv.SF_TCGEN05, dev)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.quantize(x, nv.SF_TCGEN05, out=q), args.steps)
+    elif args.part == "gemv":
+        wq = nv.quantize(to_dev(wg), nv.SF_TCGEN05)
+        n, k = wg.shape
+        for m in (1, 16):
+            xm = to_dev(xg[:m])
+            y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device=dev)
+            out[f"ms_M{m}"] = _timed(torch, dev, flush, lambda: nv.gemv_batched(xm, wq, out=y, workspace=ws),
+                                     args.steps)
+    elif args.part == "longk":
+        wq = nv.quantize(to_dev(wl), nv.SF_TCGEN05)
+        ad = to_dev(al)
+        dd = torch.empty((al.shape[0], wl.shape[0]), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, al.shape[0], wl.shape[0], al.shape[1]),
+                         dtype=torch.uint8, device=dev)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.gemm_quant_a(ad, wq, out=dd, workspace=ws), args.steps)
+    else:
+        qa = nv.quantize(to_dev(a_bits), nv.SF_TCGEN05)
+        qw = nv.quantize(to_dev(w_bits), nv.SF_TCGEN05)
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.gemm(qa, qw, out=d), args.steps)
+    out["device_status"] = nv.nvfp4_status_string(nv.nvfp4_check_device_status())
+    print(json.dumps(out), flush=True)
 
 
 if __name__ == "__main__":

@@ -320,6 +320,212 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Paired-CTA GEMM: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages 128 rows of A, its
+// half (128 rows) of B, its rows' A scales and the scales of all 256 B rows;
+// the tensor core reads the B halves from both CTAs, so each SM stages and
+// reads half the B bytes of the one-CTA kernel.  The leader (rank 0) issues
+// the scale copies and MMAs for both; both CTAs' loads complete on the
+// leader's "full" barriers, and its commits arrive on both CTAs' barriers.
+// ---------------------------------------------------------------------------
+struct PairCfg {
+  static constexpr int BN = 256;                       // N per tile (both CTAs)
+  static constexpr int STAGES = 5;
+  static constexpr int A_BYTES = BM * BK_BYTES;        // this CTA's 128 rows of A
+  static constexpr int B_BYTES = 128 * BK_BYTES;       // this CTA's half of B
+  static constexpr int SFA_BYTES = 4 * SF_ATOM;
+  static constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;    // scales of all 256 B rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int SF_COLS_PER_STAGE = 4 * 4 + 4 * 8;
+  static constexpr int TMEM_SF_BASE = BN;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = (2 + EPI_WARPS) * 32;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-B aligned");
+  static_assert(TMEM_SF_BASE + STAGES * SF_COLS_PER_STAGE <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                     const GemmParams p) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* mma_done = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * C::EPI_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSFA);
+    prefetch_tmap(&tmSFB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();                         // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int tiles_m = (p.M + 255) / 256;
+  const int tiles_n = (p.N + C::BN - 1) / C::BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int num_kt = (p.K + BK - 1) / BK;
+  const int ksteps_total = p.K / MMA_K;
+
+  if (warp == 0) {
+    // ------------------------- producer (both CTAs) -------------------------
+    if (elect_one()) {
+      const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+        const int tm = t % tiles_m;
+        const int tn = t / tiles_m;
+        const int m_cta = tm * 256 + static_cast<int>(rank) * 128;
+        const int n0 = tn * C::BN;
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          uint8_t* sSFA = sB + C::B_BYTES;
+          uint8_t* sSFB = sSFA + C::SFA_BYTES;
+          const uint32_t bar = full_leader + stage * 8;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(sA, &tmA, bar, kt * BK_BYTES, m_cta);
+          tma_load_2d_pair(sB, &tmB, bar, kt * BK_BYTES, n0 + static_cast<int>(rank) * 128);
+          tma_load_3d_pair(sSFA, &tmSFA, bar, 0, kt * 4, m_cta / 128);
+          tma_load_3d_pair(sSFB, &tmSFB, bar, 0, kt * 4, n0 / 128);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // the leader's full barriers count both CTAs' bytes: drain them there
+      if (leader)
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued_mask & (1u << s)) {
+            volatile int no_abort = 0;
+            (void)mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &no_abort, p.wait_limit_ns, p.status);
+          }
+    }
+  } else if (warp == 1) {
+    // ------------------------- MMA issuer (leader) -------------------------
+    if (leader && elect_one()) {
+      const uint32_t idesc = idesc_mxf4nvf4(256, C::BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+        if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, ksteps_total - kt * 4);
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sSFA = sB + C::B_BYTES;
+          const uint32_t sSFB = sSFA + C::SFA_BYTES;
+          const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE + stage * C::SF_COLS_PER_STAGE;
+          const uint32_t tsfb = tsfa + 16;
+          for (int j = 0; j < nk; ++j) {
+            tc_cp_32x128b_warpx4_pair(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
+            tc_cp_32x128b_warpx4_pair(tsfb + j * 8, sf_desc(sSFB + j * SF_ATOM));
+            tc_cp_32x128b_warpx4_pair(tsfb + j * 8 + 4, sf_desc(sSFB + 4 * SF_ATOM + j * SF_ATOM));
+          }
+          for (int j = 0; j < nk; ++j)
+            mma_mxf4nvf4_pair(tmem_base, code_desc(sA + j * (MMA_K / 2)), code_desc(sB + j * (MMA_K / 2)), idesc,
+                              tsfa + j * 4, tsfb + j * 8, (kt | j) != 0);
+          tc_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(acc_full, 0x3);
+        acc_phase ^= 1;
+      }
+      tc_commit_pair_mc(mma_done, 0x1);
+      volatile int no_abort = 0;
+      (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
+    }
+  } else {
+    // ------------------------- epilogue (both CTAs) -------------------------
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    const int half = ew >> 2;
+    constexpr int HALF = C::BN / 2;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles; t += npairs) {
+      const int tm = t % tiles_m;
+      const int tn = t / tiles_m;
+      if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
+      tc_fence_after();
+      uint32_t v[HALF];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * HALF;
+#pragma unroll
+      for (int c = 0; c < HALF / 32; ++c) tmem_ld_32x32b_x32(taddr + c * 32, v + c * 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      acc_phase ^= 1;
+      const int row = tm * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
+      const int col0 = tn * C::BN + half * HALF;
+      if (col0 < p.N) store_row<HALF>(p, row, col0, v, alpha);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();                         // no CTA leaves while its pair still uses its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Decode GEMV: swap-AB (weights are the 128-row MMA operand, the <= 32
 // activation rows the N = 32 operand) with stream-K over (row tile, K stage)
 // units so all SMs stream weights evenly.  Partial sums meet in an fp32
@@ -354,6 +560,18 @@ struct GemvParams {
   uint64_t wait_limit_ns;
   int* status;
 };
+
+// K stage of unit u (of weight tile `tile`).  Each tile walks its K stages
+// from a tile-dependent start, so the CTAs streaming different tiles at the
+// same moment read different column offsets of the 4-KiB-strided weight rows
+// instead of all hitting the same DRAM channels.  A bijection on a tile's
+// stages: stream-K ranges still partition each tile's K.
+__device__ __forceinline__ int gv_stage_k(int64_t u, int tile, int num_kt) {
+  const int raw = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
+  const int off = static_cast<int>((static_cast<int64_t>(tile) * 7) % num_kt);
+  const int k = raw + off;
+  return k >= num_kt ? k - num_kt : k;
+}
 
 __global__ void __launch_bounds__(GV_THREADS, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -410,7 +628,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       const int64_t pre_end = min(u_end, u_begin + GV_STAGES);
       for (int64_t u = u_begin; u < pre_end; ++u) {
         const int tile = static_cast<int>(u / p.num_kt);
-        const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+        const int kt = gv_stage_k(u, tile, p.num_kt);
         const int nk = min(4, ksteps_total - kt * 4);
         const int s = static_cast<int>(u - u_begin);
         uint8_t* sA = smem + s * GV_STAGE_BYTES;
@@ -423,7 +641,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int64_t u = u_begin; u < pre_end; ++u) {
         const int tile = static_cast<int>(u / p.num_kt);
-        const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+        const int kt = gv_stage_k(u, tile, p.num_kt);
         const int nk = min(4, ksteps_total - kt * 4);
         const int s = static_cast<int>(u - u_begin);
         uint8_t* sB = smem + s * GV_STAGE_BYTES + GV_A_BYTES;
@@ -438,7 +656,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       }
       for (int64_t u = pre_end; u < u_end; ++u) {
         const int tile = static_cast<int>(u / p.num_kt);
-        const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+        const int kt = gv_stage_k(u, tile, p.num_kt);
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
         const int nk = min(4, ksteps_total - kt * 4);
         uint8_t* sA = smem + stage * GV_STAGE_BYTES;
@@ -480,7 +698,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         const uint32_t d_tmem = tmem_base + acc * GV_N;
         bool first = true;
         for (; u < seg_end; ++u) {
-          const int kt = static_cast<int>(u - static_cast<int64_t>(tile) * p.num_kt);
+          const int kt = gv_stage_k(u, tile, p.num_kt);
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
             ok = false;
             break;
@@ -577,16 +795,19 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 }
 
 // Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
-// clearing of the partial sums.  Grid = 128 + GP_ZERO_CTAS CTAs:
-//   CTA r < M        computes the amax of all M rows (x is small; each row CTA
-//                    reads it from L2) and quantizes row r;
-//   CTA M <= r < 128 writes zero codes (r < 32) and zero scales for padding row r;
-//   CTA >= 128       clears the fp32 partial sums and the tile counters.
+// clearing of the partial sums.  Launched in clusters of GP_CLUSTER CTAs:
+//   cluster 0: CTA c owns activation rows c, c+8, c+16, c+24.  Each CTA
+//     reduces the amax of its real rows, the cluster exchanges the partial
+//     maxima through distributed shared memory, then every CTA quantizes its
+//     rows (zero codes/scales for rows >= M) and clears its share of the
+//     padding scale rows 32..127;
+//   other clusters: clear the fp32 partial sums and the tile counters.
 // It lets the dependent GEMV grid launch at once (programmatic dependent
 // launch): the GEMV streams weights while this runs and waits for it only
 // before it touches the activations, g_x or the partial sums.
 constexpr int GP_THREADS = 256;
-constexpr int GP_ZERO_CTAS = 16;
+constexpr int GP_CLUSTER = 8;
+constexpr int GP_ZERO_CLUSTERS = 2;
 
 __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                    int64_t ldx, uint8_t* __restrict__ xq,
@@ -595,74 +816,90 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
                                                                    int* __restrict__ counters, int n_counters,
                                                                    int* __restrict__ status) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int b = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  if (blockIdx.x >= GP_CLUSTER) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x - GP_CLUSTER) * GP_THREADS;
+    const int64_t first = static_cast<int64_t>(blockIdx.x - GP_CLUSTER) * GP_THREADS + tid;
+    for (int64_t i = first; i < y32_words; i += stride) y32[i] = 0.0f;
+    for (int64_t i = first; i < n_counters; i += stride) counters[i] = 0;
+    return;
+  }
+  const int c = static_cast<int>(cluster_ctarank());
   const int chunks = K >> 3;                 // 16-B chunks per row (a multiple of 8)
   const int kb = K >> 4;
-  if (b >= 128) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x - 128) * GP_THREADS;
-    for (int64_t i = static_cast<int64_t>(b - 128) * GP_THREADS + tid; i < y32_words; i += stride) y32[i] = 0.0f;
-    for (int64_t i = static_cast<int64_t>(b - 128) * GP_THREADS + tid; i < n_counters; i += stride) counters[i] = 0;
-    return;
-  }
-  const int r = b;
-  if (r >= M) {
-    if (r < GV_N) {
-      uint4* row = reinterpret_cast<uint4*>(xq + static_cast<int64_t>(r) * (K >> 1));
-      for (int c = tid; c < (K >> 5); c += GP_THREADS) row[c] = make_uint4(0, 0, 0, 0);
-    }
-    for (int j = tid; j < (kb >> 2); j += GP_THREADS)
-      *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, 4 * j, kb)) = 0u;
-    return;
-  }
-  // amax over the M real rows, 8 loads in flight per thread
-  constexpr int U = 8;
-  const int total = M * chunks;
+  __shared__ uint32_t red[GP_THREADS / 32];
+  __shared__ uint32_t partial;
+  // amax of this CTA's real rows
   uint32_t mx = 0;
-  for (int base = 0; base < total; base += U * GP_THREADS) {
-    uint4 v[U];
+  for (int r = c; r < M; r += GP_CLUSTER) {
+    const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
+    for (int base = 0; base < chunks; base += 4 * GP_THREADS) {
+      uint4 v[4];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = base + u * GP_THREADS + tid;
-      if (i < total) {
-        const int rr = i / chunks;
-        const int c = i - rr * chunks;
-        v[u] = *(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(rr) * ldx) + c);
-      } else {
-        v[u] = make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * GP_THREADS + tid;
+        v[u] = i < chunks ? row[i] : make_uint4(0, 0, 0, 0);
       }
-    }
 #pragma unroll
-    for (int u = 0; u < U; ++u) mx = max(mx, abs_max_bits8(v[u]));
+      for (int u = 0; u < 4; ++u) mx = max(mx, abs_max_bits8(v[u]));
+    }
   }
   mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-  __shared__ uint32_t red[GP_THREADS / 32];
   if (lane == 0) red[tid >> 5] = mx;
   __syncthreads();
-  uint32_t t = lane < GP_THREADS / 32 ? red[lane] : 0u;
-  t = __reduce_max_sync(0xFFFFFFFFu, t);
+  if (tid < 32) {
+    uint32_t t = lane < GP_THREADS / 32 ? red[lane] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (tid == 0) partial = t;
+  }
+  __syncwarp();
+  cluster_sync_all();                        // every CTA's partial is visible cluster-wide
+  __shared__ uint32_t cluster_max;
+  if (tid < 32) {
+    uint32_t all = tid < GP_CLUSTER ? ld_shared_cluster_u32(mapa_shared(smem_u32(&partial), tid)) : 0u;
+    all = __reduce_max_sync(0xFFFFFFFFu, all);
+    if (tid == 0) cluster_max = all;
+  }
+  __syncthreads();
+  const uint32_t all = cluster_max;
   bool valid;
-  const float g = global_scale_from_amax(__uint_as_float(t << 16), valid);
-  if (r == 0 && tid == 0) {
+  const float g = global_scale_from_amax(__uint_as_float(all << 16), valid);
+  if (c == 0 && tid == 0) {
     *g_x = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
-  // quantize row r: every warp covers 32 consecutive chunks (16 blocks)
-  const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
-  uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1));
-  for (int c = tid; c < chunks; c += GP_THREADS) {
-    const uint4 v = valid ? row[c] : make_uint4(0, 0, 0, 0);
-    uint32_t s;
-    uint32_t q = quantize_half_block(v, valid ? g : 0.0f, s);
-    if (!valid) { q = 0; s = 0; }
-    qrow[c] = q;
-    const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
-    const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
-    const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
-    if ((lane & 7) == 0)
-      *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, c >> 1, kb)) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  // quantize this CTA's rows (rows >= M get zero codes and scales)
+  const float sixth = __frcp_rn(6.0f);
+  const float rtab = recip_table_lane();
+  for (int r = c; r < GV_N; r += GP_CLUSTER) {
+    const bool real = r < M && valid;
+    const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
+    uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1));
+    // every lane runs every iteration (the quantizer shuffles across the warp);
+    // only the loads and stores are predicated.  chunks % 8 == 0, so each
+    // group of 8 lanes that gathers 4 block scales is entirely in or out.
+    for (int base = 0; base < chunks; base += GP_THREADS) {
+      const int i = base + tid;
+      const bool in = i < chunks;
+      const uint4 v = (real && in) ? row[i] : make_uint4(0, 0, 0, 0);
+      uint32_t s;
+      uint32_t q = quantize_half_block(v, real ? g : 0.0f, s, sixth, rtab);
+      if (!real) { q = 0; s = 0; }
+      if (in) qrow[i] = q;
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
+      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
+      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
+      if (in && (lane & 7) == 0)
+        *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, i >> 1, kb)) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    }
   }
+  // padding scale rows 32..127
+  for (int r = GV_N + c; r < 128; r += GP_CLUSTER)
+    for (int j = tid; j < (kb >> 2); j += GP_THREADS)
+      *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, 4 * j, kb)) = 0u;
+  __syncwarp();
+  cluster_sync_all();                        // no CTA leaves while a peer may still read its partial
 }
 
 // ---------------------------------------------------------------------------
@@ -693,6 +930,82 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, in
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Tensor-core scale array of a [rows, k] operand as a 3-D uint32 tensor
+// (128 words per 512-B atom, k/64 atoms per 128-row group, row groups);
+// a box of 4 atoms x `groups` row groups = one K stage of 256.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int groups) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int64_t kb4 = k / 64;
+  const int64_t rg = (rows + 127) / 128;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(kb4), static_cast<cuuint64_t>(rg)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(SF_ATOM), static_cast<cuuint64_t>(kb4 * SF_ATOM)};
+  cuuint32_t box[3] = {128, 4, static_cast<cuuint32_t>(groups)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                           const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                           nvfp4_out_dtype out, cudaStream_t s) {
+  using C = PairCfg;
+  CUtensorMap tmA, tmB, tmSFA, tmSFB;
+  if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, 128) ||
+      !make_sf_map(&tmSFA, a_sf, M, K, 1) || !make_sf_map(&tmSFB, b_sf, N, K, 2))
+    return NVFP4_ERR_CUDA;
+  GemmParams p;
+  p.sfa = static_cast<const uint8_t*>(a_sf);
+  p.sfb = static_cast<const uint8_t*>(b_sf);
+  p.g_a = g_a;
+  p.g_b = g_b;
+  p.d = d;
+  p.ldd = ldd;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.kb4 = static_cast<int>(K / 64);
+  p.tiles_m = static_cast<int>((M + 255) / 256);
+  p.tiles_n = static_cast<int>((N + C::BN - 1) / C::BN);
+  p.out_f32 = out == NVFP4_OUT_F32;
+  const int64_t row_bytes = ldd * (p.out_f32 ? 4 : 2);
+  p.vec_store = aligned16(d) && (row_bytes % 16) == 0;
+  p.wait_limit_ns = wait_limit_ns();
+  p.status = device_status_ptr();
+  if (!p.status) return NVFP4_ERR_CUDA;
+  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return launch_status(e);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // as many resident pairs as the device holds at once, never more than tiles
+  static int max_pairs[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return launch_status(cudaGetLastError());
+  if (dev < 64 && max_pairs[dev] == 0) {
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel, &cfg);
+    if (e != cudaSuccess || clusters < 1) return launch_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+    max_pairs[dev] = clusters;
+  }
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int pairs = tiles < max_pairs[dev < 64 ? dev : 0] ? tiles : max_pairs[dev < 64 ? dev : 0];
+  cfg.gridDim = dim3(2 * pairs);
+  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tmA, tmB, tmSFA, tmSFB, p);
+  return launch_status(e);
 }
 
 template <int BN>
@@ -735,7 +1048,8 @@ nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a
                          const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                          int64_t ldd, nvfp4_out_dtype out, cudaStream_t s) {
   if (N <= 128) return run_gemm<128>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
-  return run_gemm<256>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  if (M <= 128) return run_gemm<256>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  return run_gemm_pair(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
 }
 
 // Workspace of the GEMV: [32, K/2] activation codes | [128, K/16] activation
@@ -772,11 +1086,23 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
 
   int* status = device_status_ptr();
   if (!status) return NVFP4_ERR_CUDA;
-  gemv_prologue_kernel<<<128 + GP_ZERO_CTAS, GP_THREADS, 0, s>>>(
-      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), ldx, xq, xsf, gx, y32, M * N, cnt,
-      tiles * 4, status);
-  nvfp4_status st = launch_status(cudaGetLastError());
-  if (st != NVFP4_OK) return st;
+  {
+    cudaLaunchConfig_t pcfg = {};
+    cudaLaunchAttribute pattr[1];
+    pattr[0].id = cudaLaunchAttributeClusterDimension;
+    pattr[0].val.clusterDim.x = GP_CLUSTER;
+    pattr[0].val.clusterDim.y = 1;
+    pattr[0].val.clusterDim.z = 1;
+    pcfg.gridDim = dim3(GP_CLUSTER * (1 + GP_ZERO_CLUSTERS));
+    pcfg.blockDim = dim3(GP_THREADS);
+    pcfg.stream = s;
+    pcfg.attrs = pattr;
+    pcfg.numAttrs = 1;
+    const cudaError_t pe = cudaLaunchKernelEx(&pcfg, gemv_prologue_kernel, static_cast<const uint16_t*>(x),
+                                              static_cast<int>(M), static_cast<int>(K), ldx, xq, xsf, gx, y32,
+                                              static_cast<int64_t>(M) * N, cnt, tiles * 4, status);
+    if (pe != cudaSuccess) return launch_status(pe);
+  }
 
   CUtensorMap tmW, tmX;
   if (!make_code_map(&tmW, w_codes, N, K, BM) || !make_code_map(&tmX, xq, GV_N, K, GV_N)) return NVFP4_ERR_CUDA;

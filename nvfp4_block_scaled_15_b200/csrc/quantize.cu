@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   const int lane = threadIdx.x & 31;
   const int c0 = blockIdx.y * kSegChunks + threadIdx.x;
 
+  const float sixth = __frcp_rn(6.0f);
+  const float rtab = recip_table_lane();
   bool valid;
   const float g = global_scale_from_amax(*amax_in, valid);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   for (int u = 0; u < kUnroll; ++u) {
     const int c = c0 + u * kThreads;          // chunk index, 2 chunks per block
     uint32_t s;
-    uint32_t q = quantize_half_block(v[u], valid ? g : 0.0f, s);
+    uint32_t q = quantize_half_block(v[u], valid ? g : 0.0f, s, sixth, rtab);
     if (!valid) { q = 0; s = 0; }
     if (!real_row) s = 0;
     const bool in_row = c < chunks;

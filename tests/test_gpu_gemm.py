@@ -42,6 +42,9 @@ RAGGED = [
     (128, 384, 2048),    # N tile at 256 + a 128-wide tail tile
     (64, 512, 8192),     # long K
     (2048, 2560, 256),   # more tiles than SMs (persistent loop)
+    (300, 520, 320),     # CTA-pair path: odd number of 128-row groups, N tail in the peer's half
+    (257, 129, 192),     # CTA-pair path: K stage with 3 of 4 scale atoms
+    (1000, 700, 1024),   # CTA-pair path: tails in M and N, several tiles
 ]
 
 
@@ -84,14 +87,17 @@ def _probe(lib, m, n, k, a_sf_rowmajor, b_sf_rowmajor):
     return d.cpu().numpy()
 
 
+@pytest.mark.parametrize("m,n", [(256, 256), (128, 256)], ids=["cta_pair", "one_cta"])
 @pytest.mark.parametrize("side", ["a", "b"])
-def test_scale_layout_probes(lib, side):
+def test_scale_layout_probes(lib, side, m, n):
     """Exactly one (row, block) scale is 2.0, all others 1.0: only the D entries
     of that row (A side) or column (B side) grow, by exactly 16 (one block of
-    16 products 1 x 1).  Pins the tensor-core scale layout end to end."""
-    m, n, k = 256, 256, 512
+    16 products 1 x 1).  Pins the tensor-core scale layout end to end, for the
+    CTA-pair kernel (256 x 256) and the one-CTA kernel (M <= 128)."""
+    k = 512
     kb = k // 16
-    for row, blk in [(0, 0), (37, 5), (77, 18), (100, 31), (161, 9), (255, 30)]:
+    limit = m if side == "a" else n
+    for row, blk in [(r, b) for r, b in [(0, 0), (37, 5), (77, 18), (100, 31), (161, 9), (255, 30)] if r < limit]:
         sa = np.full((m, kb), 0x38, np.uint8)
         sb = np.full((n, kb), 0x38, np.uint8)
         (sa if side == "a" else sb)[row, blk] = 0x40
