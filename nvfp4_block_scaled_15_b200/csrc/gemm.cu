@@ -549,8 +549,8 @@ struct GemvParams {
   const uint8_t* xsf;      // activation scales, tensor-core layout (128 padded rows)
   const float* g_w;
   const float* g_x;
-  float* y32;              // [M, N] fp32 partial sums (zeroed by the prologue)
-  int* counters;           // [tiles] K-stages completed per row tile
+  float* partials;         // [2 * grid][M][128] fp32: slot 2c = CTA c's first segment, 2c+1 its last
+  int* counters;           // [tiles * 4] arrivals per (weight tile, 32-row quarter); cleared by the prologue
   __nv_bfloat16* y;
   int64_t ldy;
   int M, N, K;
@@ -738,16 +738,25 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
     }
   } else {
+    // Stream-K fix-up.  Ranges hold at least num_kt units (grid <= tiles), so
+    // a weight tile has at most two contributors: the CTA holding its first
+    // stages and the next CTA holding the rest.  A CTA that covers a whole
+    // tile writes bf16 outputs directly; a split tile's two partial sums meet
+    // in the partial slots, and whichever contributor arrives second adds
+    // them (fp32 addition commutes: the result does not depend on who).
     const int quad = warp & 3;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_w, *p.g_x));
+    const int cta = blockIdx.x;
     int acc = 0;
     uint32_t acc_phase = 0;
     int64_t u = u_begin;
     while (u < u_end) {
       const int tile = static_cast<int>(u / p.num_kt);
-      const int64_t seg_end = min(u_end, static_cast<int64_t>(tile + 1) * p.num_kt);
-      const int seg_units = static_cast<int>(seg_end - u);
+      const int64_t tile_begin = static_cast<int64_t>(tile) * p.num_kt;
+      const int64_t seg_end = min(u_end, tile_begin + p.num_kt);
+      const bool has_head = u == tile_begin;                    // this segment holds the tile's first stage
+      const bool has_tail = seg_end == tile_begin + p.num_kt;   // ... and its last stage
       u = seg_end;
       if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
       tc_fence_after();
@@ -761,25 +770,37 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         acc = 0;
         acc_phase ^= 1;
       }
-      // this warp owns weight rows (= output columns) n of one 32-row slice
-      const int n = tile * BM + quad * 32 + lane;
-      if (n < p.N) {
+      const int col = quad * 32 + lane;                         // row of the weight tile
+      const int n = tile * BM + col;                            // output column
+      if (has_head && has_tail) {
+        if (n < p.N) {
 #pragma unroll
-        for (int m = 0; m < GV_N; ++m)
-          if (m < p.M) atomicAdd(&p.y32[static_cast<int64_t>(m) * p.N + n], __uint_as_float(v[m]));
+          for (int m = 0; m < GV_N; ++m)
+            if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(__uint_as_float(v[m]) * alpha);
+        }
+        continue;
       }
+      // my slot: 2*cta for the tail of a tile I start in the middle of, 2*cta+1
+      // for the head of a tile I leave unfinished
+      float* mine = p.partials + (static_cast<int64_t>(2 * cta + (has_head ? 1 : 0)) * p.M) * BM;
+      const float* other = p.partials + (static_cast<int64_t>(has_head ? 2 * (cta + 1) : 2 * (cta - 1) + 1) * p.M) * BM;
+#pragma unroll
+      for (int m = 0; m < GV_N; ++m)
+        if (m < p.M) mine[m * BM + col] = __uint_as_float(v[m]);
       __threadfence();
       __syncwarp();
-      int done = 0;
-      if (lane == 0) done = atomicAdd(&p.counters[tile * 4 + quad], seg_units) + seg_units;
-      done = __shfl_sync(0xFFFFFFFFu, done, 0);
-      if (done == p.num_kt) {
+      int arrived = 0;
+      if (lane == 0) arrived = atomicAdd(&p.counters[tile * 4 + quad], 1);
+      arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
+      if (arrived == 1) {                                       // second of the two: finish
         __threadfence();
         if (n < p.N) {
-          for (int m = 0; m < p.M; ++m) {
-            const float sum = __ldcg(&p.y32[static_cast<int64_t>(m) * p.N + n]);
-            p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
-          }
+#pragma unroll
+          for (int m = 0; m < GV_N; ++m)
+            if (m < p.M) {
+              const float sum = __uint_as_float(v[m]) + __ldcg(other + m * BM + col);
+              p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
+            }
         }
       }
     }
@@ -795,24 +816,22 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 }
 
 // Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
-// clearing of the partial sums.  Launched in clusters of GP_CLUSTER CTAs:
+// clearing of the fix-up counters.  Launched in clusters of GP_CLUSTER CTAs:
 //   cluster 0: CTA c owns activation rows c, c+8, c+16, c+24.  Each CTA
 //     reduces the amax of its real rows, the cluster exchanges the partial
 //     maxima through distributed shared memory, then every CTA quantizes its
-//     rows (zero codes/scales for rows >= M) and clears its share of the
-//     padding scale rows 32..127;
-//   other clusters: clear the fp32 partial sums and the tile counters.
+//     real rows and zeroes its padding rows (codes and scales);
+//   other clusters: clear the tile counters.
 // It lets the dependent GEMV grid launch at once (programmatic dependent
 // launch): the GEMV streams weights while this runs and waits for it only
 // before it touches the activations, g_x or the partial sums.
 constexpr int GP_THREADS = 256;
 constexpr int GP_CLUSTER = 8;
-constexpr int GP_ZERO_CLUSTERS = 2;
+constexpr int GP_ZERO_CLUSTERS = 1;
 
 __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                    int64_t ldx, uint8_t* __restrict__ xq,
                                                                    uint8_t* __restrict__ xsf, float* __restrict__ g_x,
-                                                                   float* __restrict__ y32, int64_t y32_words,
                                                                    int* __restrict__ counters, int n_counters,
                                                                    int* __restrict__ status) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -821,7 +840,6 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
   if (blockIdx.x >= GP_CLUSTER) {
     const int64_t stride = static_cast<int64_t>(gridDim.x - GP_CLUSTER) * GP_THREADS;
     const int64_t first = static_cast<int64_t>(blockIdx.x - GP_CLUSTER) * GP_THREADS + tid;
-    for (int64_t i = first; i < y32_words; i += stride) y32[i] = 0.0f;
     for (int64_t i = first; i < n_counters; i += stride) counters[i] = 0;
     return;
   }
@@ -869,11 +887,20 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
     *g_x = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
-  // quantize this CTA's rows (rows >= M get zero codes and scales)
+  // quantize this CTA's real rows; padding rows (M <= r < 32) get zero codes
+  // and scales.  Rows 32..127 of the scale layout are padding too: each 16-B
+  // chunk (r % 32) of an atom holds rows r, r+32, r+64, r+96, so writing the
+  // chunk of row r < 32 whole (its 4 scales, then 12 zero bytes) also clears them.
   const float sixth = __frcp_rn(6.0f);
   const float rtab = recip_table_lane();
   for (int r = c; r < GV_N; r += GP_CLUSTER) {
-    const bool real = r < M && valid;
+    uint4* chunk_row = reinterpret_cast<uint4*>(xsf) + r;       // + 32 * atom
+    if (r >= M || !valid) {
+      uint4* qrow = reinterpret_cast<uint4*>(xq + static_cast<int64_t>(r) * (K >> 1));
+      for (int i = tid; i < (K >> 5); i += GP_THREADS) qrow[i] = make_uint4(0, 0, 0, 0);
+      for (int j = tid; j < (kb >> 2); j += GP_THREADS) chunk_row[32 * j] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
     const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
     uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1));
     // every lane runs every iteration (the quantizer shuffles across the warp);
@@ -882,22 +909,17 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
     for (int base = 0; base < chunks; base += GP_THREADS) {
       const int i = base + tid;
       const bool in = i < chunks;
-      const uint4 v = (real && in) ? row[i] : make_uint4(0, 0, 0, 0);
+      const uint4 v = in ? row[i] : make_uint4(0, 0, 0, 0);
       uint32_t s;
-      uint32_t q = quantize_half_block(v, real ? g : 0.0f, s, sixth, rtab);
-      if (!real) { q = 0; s = 0; }
+      const uint32_t q = quantize_half_block(v, g, s, sixth, rtab);
       if (in) qrow[i] = q;
       const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
       const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
       const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
-      if (in && (lane & 7) == 0)
-        *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, i >> 1, kb)) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      if (in && (lane & 7) == 0)                                // atom i / 8 of row r
+        chunk_row[32 * (i >> 3)] = make_uint4(s | (s1 << 8) | (s2 << 16) | (s3 << 24), 0u, 0u, 0u);
     }
   }
-  // padding scale rows 32..127
-  for (int r = GV_N + c; r < 128; r += GP_CLUSTER)
-    for (int j = tid; j < (kb >> 2); j += GP_THREADS)
-      *reinterpret_cast<uint32_t*>(xsf + sf_tc_offset(r, 4 * j, kb)) = 0u;
   __syncwarp();
   cluster_sync_all();                        // no CTA leaves while a peer may still read its partial
 }
@@ -1053,9 +1075,12 @@ nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a
 }
 
 // Workspace of the GEMV: [32, K/2] activation codes | [128, K/16] activation
-// scales | g_x (16 B) | [M, N] fp32 partials | counters.
+// scales | g_x (16 B) | fp32 partial slots [2 * GV_MAX_CTAS][M][128] |
+// counters [tiles * 4].
+constexpr int GV_MAX_CTAS = 160;
+
 struct GemvWs {
-  size_t xq, xsf, gx, y32, cnt, total;
+  size_t xq, xsf, gx, part, cnt, total;
 };
 
 static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
@@ -1064,8 +1089,8 @@ static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
   w.xq = 0;
   w.xsf = al(w.xq + static_cast<size_t>(GV_N) * K / 2);
   w.gx = al(w.xsf + static_cast<size_t>(128) * K / 16);
-  w.y32 = al(w.gx + 16);
-  w.cnt = al(w.y32 + static_cast<size_t>(M) * N * 4);
+  w.part = al(w.gx + 16);
+  w.cnt = al(w.part + static_cast<size_t>(2 * GV_MAX_CTAS) * M * BM * 4);
   w.total = al(w.cnt + static_cast<size_t>((N + BM - 1) / BM) * 4 * 4);
   return w;
 }
@@ -1079,7 +1104,7 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
   uint8_t* xq = base + L.xq;
   uint8_t* xsf = base + L.xsf;
   float* gx = reinterpret_cast<float*>(base + L.gx);
-  float* y32 = reinterpret_cast<float*>(base + L.y32);
+  float* partials = reinterpret_cast<float*>(base + L.part);
   int* cnt = reinterpret_cast<int*>(base + L.cnt);
   const int tiles = static_cast<int>((N + BM - 1) / BM);
   const int sms = device_sm_count();
@@ -1099,8 +1124,8 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
     pcfg.attrs = pattr;
     pcfg.numAttrs = 1;
     const cudaError_t pe = cudaLaunchKernelEx(&pcfg, gemv_prologue_kernel, static_cast<const uint16_t*>(x),
-                                              static_cast<int>(M), static_cast<int>(K), ldx, xq, xsf, gx, y32,
-                                              static_cast<int64_t>(M) * N, cnt, tiles * 4, status);
+                                              static_cast<int>(M), static_cast<int>(K), ldx, xq, xsf, gx, cnt,
+                                              tiles * 4, status);
     if (pe != cudaSuccess) return launch_status(pe);
   }
 
@@ -1111,7 +1136,7 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
   p.xsf = xsf;
   p.g_w = g_w;
   p.g_x = gx;
-  p.y32 = y32;
+  p.partials = partials;
   p.counters = cnt;
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ldy = ldy;
@@ -1124,8 +1149,10 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;
-  const int64_t units = static_cast<int64_t>(tiles) * p.num_kt;
-  const int grid = static_cast<int>(units < sms ? units : sms);
+  // grid <= tiles: every CTA's stream-K range spans at least one tile's worth
+  // of stages, so each tile has at most two contributors
+  int grid = tiles < sms ? tiles : sms;
+  if (grid > GV_MAX_CTAS) grid = GV_MAX_CTAS;
   cudaError_t e = cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_BYTES);
   if (e != cudaSuccess) return launch_status(e);
   cudaLaunchConfig_t cfg = {};

@@ -24,6 +24,23 @@ def test_gemv_matches_oracle(lib, m, n, k):
     check_bf16(host_bf16_bits(y), d_ref, s_ref, alpha)
 
 
+@pytest.mark.parametrize("m", [1, 7, 16])
+def test_gemv_tiles_split_between_ctas(lib, m):
+    """160 weight tiles on at most 148 CTAs: stream-K ranges split tiles
+    between neighbouring CTAs, whose partial sums meet in the workspace.
+    Every output is checked against the oracle."""
+    n, k = 160 * 128, 1024
+    x = inputs.gaussian_bf16((m, k), seed=900 + m)
+    w = inputs.gaussian_bf16((n, k), seed=901, std=0.02)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    y = lib.gemv_batched(dev_bf16(x), qw)
+    assert lib.nvfp4_check_device_status() == lib.OK
+    px, sx, gx, _ = O.quantize(x)
+    pw, sw, gw, _ = O.quantize(w)
+    d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, pw, sw, gw)
+    check_bf16(host_bf16_bits(y), d_ref, s_ref, alpha)
+
+
 def test_gemv_repeated_calls_reuse_workspace(lib):
     """The workspace is re-initialised by every call: two calls, same answer."""
     m, n, k = 8, 640, 512
