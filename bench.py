@@ -434,7 +434,17 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
                                                                 q.amax, 1), reps)
     two_pass = rows * k * 2 * 2 + rows * k // 2 + rows * k // 16
     one_pass = rows * k * 2 + rows * k // 2 + rows * k // 16
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(10):
+        nv.quantize(x, nv.SF_TCGEN05, out=q)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_b2b = e0.elapsed_time(e1) / 10
     out["quantize_16384x8192"] = {
+        "back_to_back_ms": ms_b2b, "back_to_back_gbs_two_pass": two_pass / ms_b2b / 1e6,
+        "back_to_back_frac_hbm": two_pass / ms_b2b / 1e6 / hbm_peak,
         "ms": ms_all, "gbs_two_pass": two_pass / ms_all / 1e6, "frac_hbm": two_pass / ms_all / 1e6 / hbm_peak,
         "gbs_strict_one_read": one_pass / ms_all / 1e6,
         "amax_ms": ms_amax, "amax_gbs": rows * k * 2 / ms_amax / 1e6,
@@ -456,7 +466,29 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
         res[f"M={m}"] = {"ms": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak,
                          "algorithmic_bytes": algo}
     out["gemv_28672x8192"] = res
-    del wq
+    # decode throughput: calls back to back (as layers follow one another),
+    # three weight copies in rotation so no call finds its weights in L2
+    wqs = [wq] + [nv.quantize(to_dev(wg), nv.SF_TCGEN05) for _ in range(2)]
+    thr = {}
+    for m in (1, 8, 16):
+        xm = to_dev(xg[:m])
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device=dev)
+        calls = 30
+        for i in range(6):
+            nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+        stream = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(calls):
+            nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / calls
+        algo = n * k // 2 + n * k // 16 + m * k * 2 + m * n * 2
+        thr[f"M={m}"] = {"ms_per_call": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak}
+    out["gemv_28672x8192_back_to_back"] = thr
+    del wq, wqs
 
     # long-K: A [4096, 28672] bf16 quantized in the call, W [8192, 28672] pre-quantized
     al, wl = pin["longk"]

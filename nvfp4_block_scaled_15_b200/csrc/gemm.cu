@@ -336,13 +336,21 @@ struct PairCfg {
   static constexpr int SFA_BYTES = 4 * SF_ATOM;
   static constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;    // scales of all 256 B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int SF_COLS_PER_STAGE = 4 * 4 + 4 * 8;
-  static constexpr int TMEM_SF_BASE = BN;
+  // Two accumulators that share OVL columns: acc0 = [0, 256), acc1 =
+  // [256 - OVL, 512 - OVL).  The epilogue drains the shared columns first and
+  // releases them, so the next tile's MMAs start while the rest of the
+  // previous accumulator is still being drained.  The last OVL columns hold
+  // the scale factors of the current K stage (one region, refreshed per stage:
+  // tcgen05.cp and tcgen05.mma issued by one thread execute in order).
+  static constexpr int OVL = 64;
+  static constexpr int ACC1_COL = BN - OVL;
+  static constexpr int TMEM_SF_BASE = 2 * BN - OVL;
+  static constexpr int SF_COLS = 4 * 4 + 4 * 8;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-B aligned");
-  static_assert(TMEM_SF_BASE + STAGES * SF_COLS_PER_STAGE <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(TMEM_SF_BASE + SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -355,9 +363,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* mma_done = acc_empty + 1;
+  uint64_t* acc_full = empty + C::STAGES;      // MMA -> epilogue, one phase per tile
+  uint64_t* acc_empty = acc_full + 1;          // [2] accumulator b fully drained
+  uint64_t* ovl_free = acc_empty + 2;          // shared columns drained, one phase per tile
+  uint64_t* mma_done = ovl_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -374,7 +383,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * C::EPI_WARPS);
+    mbar_init(&acc_empty[0], 2 * C::EPI_WARPS);
+    mbar_init(&acc_empty[1], 2 * C::EPI_WARPS);
+    mbar_init(ovl_free, 2 * 4);                // the 4 warps per CTA that hold the shared columns
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -445,34 +456,62 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     // ------------------------- MMA issuer (leader) -------------------------
     if (leader && elect_one()) {
       const uint32_t idesc = idesc_mxf4nvf4(256, C::BN);
+      const uint32_t smem_base = smem_u32(smem);
+      const bool full_last_stage = (ksteps_total & 3) == 0;   // every K stage holds 4 MMA-K steps
+      const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE;
+      const uint32_t tsfb = tsfa + 16;
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t acc_phase = 0;
-      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
-        if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+      uint32_t empty_phase = 0;                 // bit b: phase parity of acc_empty[b]
+      int j = 0;                                // tiles issued by this pair
+      bool ok = true;
+      for (int t = pair; t < num_tiles && !*abort_flag && ok; t += npairs, ++j) {
+        const int b = j & 1;
+        // accumulator b was drained by the epilogue of tile j-2, and the columns
+        // it shares with accumulator b^1 by the epilogue of tile j-1
+        if (!mbar_wait_bounded(&acc_empty[b], ((empty_phase >> b) & 1u) ^ 1u, abort_flag, p.wait_limit_ns, p.status))
+          break;
+        empty_phase ^= 1u << b;
+        if (!mbar_wait_bounded(ovl_free, static_cast<uint32_t>(j & 1) ^ 1, abort_flag, p.wait_limit_ns, p.status))
+          break;
         tc_fence_after();
-        bool ok = true;
+        const uint32_t d_tmem = tmem_base + (b ? C::ACC1_COL : 0);
         for (int kt = 0; kt < num_kt; ++kt) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = min(4, ksteps_total - kt * 4);
-          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
-          const uint32_t sSFA = sB + C::B_BYTES;
-          const uint32_t sSFB = sSFA + C::SFA_BYTES;
-          const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE + stage * C::SF_COLS_PER_STAGE;
-          const uint32_t tsfb = tsfa + 16;
-          for (int j = 0; j < nk; ++j) {
-            tc_cp_32x128b_warpx4_pair(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
-            tc_cp_32x128b_warpx4_pair(tsfb + j * 8, sf_desc(sSFB + j * SF_ATOM));
-            tc_cp_32x128b_warpx4_pair(tsfb + j * 8 + 4, sf_desc(sSFB + 4 * SF_ATOM + j * SF_ATOM));
+          // Stage base descriptors, advanced by constants: the start-address
+          // field is address >> 4, so +2 per 32-B MMA-K step of codes and +32
+          // per 512-B scale atom.
+          const uint32_t sA = smem_base + stage * C::STAGE_BYTES;
+          const uint64_t ad = code_desc(sA);
+          const uint64_t bd = code_desc(sA + C::A_BYTES);
+          const uint64_t fa = sf_desc(sA + C::A_BYTES + C::B_BYTES);
+          const uint64_t fb = sf_desc(sA + C::A_BYTES + C::B_BYTES + C::SFA_BYTES);
+          if (kt + 1 < num_kt || full_last_stage) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              tc_cp_32x128b_warpx4_pair(tsfa + jj * 4, fa + 32 * jj);
+              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8, fb + 32 * jj);
+              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8 + 4, fb + 128 + 32 * jj);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              mma_mxf4nvf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, idesc, tsfa + jj * 4, tsfb + jj * 8,
+                                (kt | jj) != 0);
+          } else {
+            const int nk = ksteps_total - kt * 4;
+            for (int jj = 0; jj < nk; ++jj) {
+              tc_cp_32x128b_warpx4_pair(tsfa + jj * 4, fa + 32 * jj);
+              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8, fb + 32 * jj);
+              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8 + 4, fb + 128 + 32 * jj);
+            }
+            for (int jj = 0; jj < nk; ++jj)
+              mma_mxf4nvf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, idesc, tsfa + jj * 4, tsfb + jj * 8,
+                                (kt | jj) != 0);
           }
-          for (int j = 0; j < nk; ++j)
-            mma_mxf4nvf4_pair(tmem_base, code_desc(sA + j * (MMA_K / 2)), code_desc(sB + j * (MMA_K / 2)), idesc,
-                              tsfa + j * 4, tsfb + j * 8, (kt | j) != 0);
           tc_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == C::STAGES) {
             stage = 0;
@@ -481,7 +520,6 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         }
         if (!ok) break;
         tc_commit_pair_mc(acc_full, 0x3);
-        acc_phase ^= 1;
       }
       tc_commit_pair_mc(mma_done, 0x1);
       volatile int no_abort = 0;
@@ -495,21 +533,45 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     constexpr int HALF = C::BN / 2;
     const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-    uint32_t acc_phase = 0;
-    for (int t = pair; t < num_tiles; t += npairs) {
+    const uint32_t ovl_free_leader = mapa_shared(smem_u32(ovl_free), 0);
+    int j = 0;
+    for (int t = pair; t < num_tiles; t += npairs, ++j) {
+      const int b = j & 1;
       const int tm = t % tiles_m;
       const int tn = t / tiles_m;
-      if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
+      if (!mbar_wait_bounded(acc_full, static_cast<uint32_t>(j & 1), abort_flag, p.wait_limit_ns, p.status)) break;
       tc_fence_after();
       uint32_t v[HALF];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * HALF;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (b ? C::ACC1_COL : 0) + half * HALF;
+      // The shared columns [256-OVL, 256) are the last OVL of accumulator 0
+      // (held by half 1) and the first OVL of accumulator 1 (held by half 0).
+      if (b == 0 && half == 1) {
+        tmem_ld_32x32b_x32(taddr + 64, v + 64);
+        tmem_ld_32x32b_x32(taddr + 96, v + 96);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
+        tmem_ld_32x32b_x32(taddr + 0, v + 0);
+        tmem_ld_32x32b_x32(taddr + 32, v + 32);
+      } else if (b == 1 && half == 0) {
+        tmem_ld_32x32b_x32(taddr + 0, v + 0);
+        tmem_ld_32x32b_x32(taddr + 32, v + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
+        tmem_ld_32x32b_x32(taddr + 64, v + 64);
+        tmem_ld_32x32b_x32(taddr + 96, v + 96);
+      } else {
 #pragma unroll
-      for (int c = 0; c < HALF / 32; ++c) tmem_ld_32x32b_x32(taddr + c * 32, v + c * 32);
+        for (int c = 0; c < HALF / 32; ++c) tmem_ld_32x32b_x32(taddr + c * 32, v + c * 32);
+      }
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-      acc_phase ^= 1;
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8u * b);
       const int row = tm * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
       const int col0 = tn * C::BN + half * HALF;
       if (col0 < p.N) store_row<HALF>(p, row, col0, v, alpha);

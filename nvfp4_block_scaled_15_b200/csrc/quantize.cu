@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
     if (!valid) record_status(status, kDevRange);
   }
   const bool real_row = r < rows;
+  // tensor-core layout: byte of (row r, block b) = row_base + (b / 4) * 512 + b % 4
+  const int64_t row_base = (static_cast<int64_t>(r >> 7) * (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
 
   uint4 v[kUnroll];
 #pragma unroll
@@ -101,14 +103,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
     if (!kTcLayout) {
       if (real_row && in_row && (lane & 1) == 0) sf[static_cast<int64_t>(r) * kb + b] = static_cast<uint8_t>(s);
     } else {
-      // lanes 0,2,4,6 (mod 8) hold blocks 4j..4j+3: gather them into one word
-      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
-      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
-      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
-      if (in_row && (lane & 7) == 0) {
-        const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
-        *reinterpret_cast<uint32_t*>(sf + sf_tc_offset(r, b, kb)) = word;
-      }
+      if (in_row && (lane & 1) == 0) sf[row_base + ((b >> 2) << 9) + (b & 3)] = static_cast<uint8_t>(s);
     }
   }
 }
