@@ -328,6 +328,9 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // the scale copies and MMAs for both; both CTAs' loads complete on the
 // leader's "full" barriers, and its commits arrive on both CTAs' barriers.
 // ---------------------------------------------------------------------------
+#ifndef NVFP4_PAIR_SF_BUFS
+#define NVFP4_PAIR_SF_BUFS 1
+#endif
 struct PairCfg {
   static constexpr int BN = 256;                       // N per tile (both CTAs)
   static constexpr int STAGES = 5;
@@ -342,15 +345,16 @@ struct PairCfg {
   // previous accumulator is still being drained.  The last OVL columns hold
   // the scale factors of the current K stage (one region, refreshed per stage:
   // tcgen05.cp and tcgen05.mma issued by one thread execute in order).
-  static constexpr int OVL = 64;
+  static constexpr int SF_BUFS = NVFP4_PAIR_SF_BUFS;
+  static constexpr int SF_COLS = 4 * 4 + 4 * 8;        // one K stage: SFA 16 + SFB 32 columns
+  static constexpr int OVL = SF_BUFS == 1 ? 64 : 128;
   static constexpr int ACC1_COL = BN - OVL;
   static constexpr int TMEM_SF_BASE = 2 * BN - OVL;
-  static constexpr int SF_COLS = 4 * 4 + 4 * 8;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-B aligned");
-  static_assert(TMEM_SF_BASE + SF_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(TMEM_SF_BASE + SF_BUFS * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -458,8 +462,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       const uint32_t idesc = idesc_mxf4nvf4(256, C::BN);
       const uint32_t smem_base = smem_u32(smem);
       const bool full_last_stage = (ksteps_total & 3) == 0;   // every K stage holds 4 MMA-K steps
-      const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE;
-      const uint32_t tsfb = tsfa + 16;
+      uint32_t tsfa = tmem_base + C::TMEM_SF_BASE;
+      uint32_t tsfb = tsfa + 16;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_phase = 0;                 // bit b: phase parity of acc_empty[b]
@@ -513,6 +517,11 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                                 (kt | jj) != 0);
           }
           tc_commit_pair_mc(&empty[stage], 0x3);
+          if (C::SF_BUFS == 2) {
+            const uint32_t flip = static_cast<uint32_t>(C::SF_COLS);
+            tsfa = (tsfa == tmem_base + C::TMEM_SF_BASE) ? tsfa + flip : tsfa - flip;
+            tsfb = tsfa + 16;
+          }
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
@@ -546,13 +555,20 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (b ? C::ACC1_COL : 0) + half * HALF;
       // The shared columns [256-OVL, 256) are the last OVL of accumulator 0
       // (held by half 1) and the first OVL of accumulator 1 (held by half 0).
-      if (b == 0 && half == 1) {
+      if (C::OVL > 64 && ((b == 0 && half == 1) || (b == 1 && half == 0))) {
+#pragma unroll
+        for (int c = 0; c < HALF / 32; ++c) tmem_ld_32x32b_x32(taddr + c * 32, v + c * 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(ovl_free_leader);
+      } else if (b == 0 && half == 1) {
         tmem_ld_32x32b_x32(taddr + 64, v + 64);
         tmem_ld_32x32b_x32(taddr + 96, v + 96);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
+        if (lane == 0) mbar_arrive_cluster_relaxed(ovl_free_leader);
         tmem_ld_32x32b_x32(taddr + 0, v + 0);
         tmem_ld_32x32b_x32(taddr + 32, v + 32);
       } else if (b == 1 && half == 0) {
@@ -561,7 +577,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ovl_free_leader);
+        if (lane == 0) mbar_arrive_cluster_relaxed(ovl_free_leader);
         tmem_ld_32x32b_x32(taddr + 64, v + 64);
         tmem_ld_32x32b_x32(taddr + 96, v + 96);
       } else {
@@ -571,7 +587,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8u * b);
+      if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader + 8u * b);
       const int row = tm * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
       const int col0 = tn * C::BN + half * HALF;
       if (col0 < p.N) store_row<HALF>(p, row, col0, v, alpha);

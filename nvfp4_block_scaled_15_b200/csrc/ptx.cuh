@@ -232,6 +232,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Arrive without release semantics.  For signalling that tensor-memory reads
+// are complete (tcgen05.wait::ld has returned): a release arrive at cluster
+// scope would also wait for every earlier global store of the thread to be
+// performed, which puts the previous tile's output stores on the path of the
+// accumulator handoff.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Tiled loads into this CTA's shared memory whose completion bytes are
 // counted on the barrier at `mbar_cluster` (the pair leader's).  No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t mbar_cluster, int32_t x,
