@@ -73,6 +73,7 @@ struct GemmParams {
   int tiles_m, tiles_n;
   int out_f32;
   int vec_store;    // rows of D are 16-byte aligned: vector stores allowed
+  int tma_store;    // bf16 D written by TMA stores through shared memory (CTA-pair kernel)
   uint64_t wait_limit_ns;
   int* status;
 };
@@ -328,9 +329,6 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // the scale copies and MMAs for both; both CTAs' loads complete on the
 // leader's "full" barriers, and its commits arrive on both CTAs' barriers.
 // ---------------------------------------------------------------------------
-#ifndef NVFP4_PAIR_SF_BUFS
-#define NVFP4_PAIR_SF_BUFS 1
-#endif
 struct PairCfg {
   static constexpr int BN = 256;                       // N per tile (both CTAs)
   static constexpr int STAGES = 5;
@@ -345,27 +343,32 @@ struct PairCfg {
   // previous accumulator is still being drained.  The last OVL columns hold
   // the scale factors of the current K stage (one region, refreshed per stage:
   // tcgen05.cp and tcgen05.mma issued by one thread execute in order).
-  static constexpr int SF_BUFS = NVFP4_PAIR_SF_BUFS;
   static constexpr int SF_COLS = 4 * 4 + 4 * 8;        // one K stage: SFA 16 + SFB 32 columns
-  static constexpr int OVL = SF_BUFS == 1 ? 64 : 128;
+  static constexpr int OVL = 64;
   static constexpr int ACC1_COL = BN - OVL;
   static constexpr int TMEM_SF_BASE = 2 * BN - OVL;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  // Output staging for bf16 D: per epilogue warp two 32 x 32 bf16 boxes
+  // (64-B rows, 64-B swizzle) written to global memory by TMA stores.
+  static constexpr int EPI_BOX_COLS = 32;
+  static constexpr int EPI_BOX_BYTES = 32 * EPI_BOX_COLS * 2;
+  static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BOX_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 256 + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-B aligned");
-  static_assert(TMEM_SF_BASE + SF_BUFS * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(TMEM_SF_BASE + SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                     const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   using C = PairCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* epi_smem = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;      // MMA -> epilogue, one phase per tile
   uint64_t* acc_empty = acc_full + 1;          // [2] accumulator b fully drained
@@ -399,6 +402,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmSFA);
     prefetch_tmap(&tmSFB);
+    if (p.tma_store) prefetch_tmap(&tmD);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -462,8 +466,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       const uint32_t idesc = idesc_mxf4nvf4(256, C::BN);
       const uint32_t smem_base = smem_u32(smem);
       const bool full_last_stage = (ksteps_total & 3) == 0;   // every K stage holds 4 MMA-K steps
-      uint32_t tsfa = tmem_base + C::TMEM_SF_BASE;
-      uint32_t tsfb = tsfa + 16;
+      const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE;
+      const uint32_t tsfb = tsfa + 16;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_phase = 0;                 // bit b: phase parity of acc_empty[b]
@@ -517,11 +521,6 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                                 (kt | jj) != 0);
           }
           tc_commit_pair_mc(&empty[stage], 0x3);
-          if (C::SF_BUFS == 2) {
-            const uint32_t flip = static_cast<uint32_t>(C::SF_COLS);
-            tsfa = (tsfa == tmem_base + C::TMEM_SF_BASE) ? tsfa + flip : tsfa - flip;
-            tsfb = tsfa + 16;
-          }
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
@@ -555,14 +554,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (b ? C::ACC1_COL : 0) + half * HALF;
       // The shared columns [256-OVL, 256) are the last OVL of accumulator 0
       // (held by half 1) and the first OVL of accumulator 1 (held by half 0).
-      if (C::OVL > 64 && ((b == 0 && half == 1) || (b == 1 && half == 0))) {
-#pragma unroll
-        for (int c = 0; c < HALF / 32; ++c) tmem_ld_32x32b_x32(taddr + c * 32, v + c * 32);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster_relaxed(ovl_free_leader);
-      } else if (b == 0 && half == 1) {
+      if (b == 0 && half == 1) {
         tmem_ld_32x32b_x32(taddr + 64, v + 64);
         tmem_ld_32x32b_x32(taddr + 96, v + 96);
         tmem_ld_wait();
@@ -588,10 +580,43 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader + 8u * b);
-      const int row = tm * 256 + static_cast<int>(rank) * 128 + quad * 32 + lane;
+      const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const int col0 = tn * C::BN + half * HALF;
-      if (col0 < p.N) store_row<HALF>(p, row, col0, v, alpha);
+      if (p.tma_store) {
+        // Coalesced output: each 32 x 32 box goes through one of this warp's
+        // two staging buffers and leaves by a TMA store; rows and columns past
+        // the end of D are clipped by the store.
+        if (row0 < p.M) {
+#pragma unroll
+          for (int c = 0; c < HALF / C::EPI_BOX_COLS; ++c) {
+            if (col0 + c * C::EPI_BOX_COLS >= p.N) break;
+            uint8_t* box = epi_smem + (ew * 2 + (c & 1)) * C::EPI_BOX_BYTES;
+            if (lane == 0) bulk_wait_group_read<1>();   // the store that last read this buffer is done
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t* f = v + c * C::EPI_BOX_COLS + q * 8;
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(f[0]) * alpha, __uint_as_float(f[1]) * alpha);
+              w.y = pack_bf16x2(__uint_as_float(f[2]) * alpha, __uint_as_float(f[3]) * alpha);
+              w.z = pack_bf16x2(__uint_as_float(f[4]) * alpha, __uint_as_float(f[5]) * alpha);
+              w.w = pack_bf16x2(__uint_as_float(f[6]) * alpha, __uint_as_float(f[7]) * alpha);
+              // 64-B swizzle: 16-B chunk q of row r sits at chunk q ^ ((r >> 1) & 3)
+              *reinterpret_cast<uint4*>(box + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = w;
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmD, box, col0 + c * C::EPI_BOX_COLS, row0);
+              bulk_commit_group();
+            }
+          }
+        }
+      } else if (col0 < p.N) {
+        store_row<HALF>(p, row0 + lane, col0, v, alpha);
+      }
     }
+    if (p.tma_store && lane == 0) bulk_wait_group<0>();
   }
 
   __syncwarp();
@@ -1050,15 +1075,37 @@ bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int 
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map of a bf16 D [rows, cols] with row pitch ld elements: 32 x 32
+// boxes, 64-B swizzle (matching the epilogue's staging layout).
+bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(PairCfg::EPI_BOX_COLS), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                            const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
                            nvfp4_out_dtype out, cudaStream_t s) {
   using C = PairCfg;
-  CUtensorMap tmA, tmB, tmSFA, tmSFB;
+  CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
   if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, 128) ||
       !make_sf_map(&tmSFA, a_sf, M, K, 1) || !make_sf_map(&tmSFB, b_sf, N, K, 2))
     return NVFP4_ERR_CUDA;
-  GemmParams p;
+  // bf16 D whose base, row pitch and row end (N) fall on 16-B boundaries leaves
+  // through TMA stores.  The store clips boxes at the tensor's edge in whole
+  // 16-B chunks, so a row end inside a chunk would be overrun: such D takes
+  // the direct-store path.
+  const bool tma_store = out == NVFP4_OUT_BF16 && aligned16(d) && (ldd * 2) % 16 == 0 && N % 8 == 0;
+  memset(&tmD, 0, sizeof(tmD));
+  if (tma_store && !make_out_map(&tmD, d, M, N, ldd)) return NVFP4_ERR_CUDA;
+  GemmParams p{};
   p.sfa = static_cast<const uint8_t*>(a_sf);
   p.sfb = static_cast<const uint8_t*>(b_sf);
   p.g_a = g_a;
@@ -1074,6 +1121,7 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   p.out_f32 = out == NVFP4_OUT_F32;
   const int64_t row_bytes = ldd * (p.out_f32 ? 4 : 2);
   p.vec_store = aligned16(d) && (row_bytes % 16) == 0;
+  p.tma_store = tma_store;
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;
@@ -1104,7 +1152,7 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   const int tiles = p.tiles_m * p.tiles_n;
   const int pairs = tiles < max_pairs[dev < 64 ? dev : 0] ? tiles : max_pairs[dev < 64 ? dev : 0];
   cfg.gridDim = dim3(2 * pairs);
-  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tmA, tmB, tmSFA, tmSFB, p);
+  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tmA, tmB, tmSFA, tmSFB, tmD, p);
   return launch_status(e);
 }
 
@@ -1115,7 +1163,7 @@ nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, c
   using C = GemmCfg<BN>;
   CUtensorMap tmA, tmB;
   if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, BN)) return NVFP4_ERR_CUDA;
-  GemmParams p;
+  GemmParams p{};
   p.sfa = static_cast<const uint8_t*>(a_sf);
   p.sfb = static_cast<const uint8_t*>(b_sf);
   p.g_a = g_a;

@@ -59,17 +59,24 @@ def test_gemm_shapes(lib, m, n, k):
     check_bf16(host_bf16_bits(d16), d_ref, s_ref, alpha)
 
 
-def test_gemm_output_pitch(lib):
-    a = inputs.gaussian_bf16((130, 256), seed=91)
-    b = inputs.gaussian_bf16((140, 256), seed=92)
+@pytest.mark.parametrize("n", [140, 136, 264], ids=lambda v: f"n{v}")
+def test_gemm_output_pitch(lib, n):
+    """D written into a wider, taller buffer (row pitch 288): nothing outside
+    the M x N window changes.  N = 140 ends inside a 16-B chunk (direct
+    stores); N = 136 and 264 end on a chunk boundary inside a 32-column box
+    (TMA stores clipped at the tensor edge)."""
+    m = 130
+    a = inputs.gaussian_bf16((m, 256), seed=91)
+    b = inputs.gaussian_bf16((n, 256), seed=92)
     d_ref, s_ref, alpha = _oracle(a, b)
     qa = lib.quantize(dev_bf16(a), lib.SF_TCGEN05)
     qb = lib.quantize(dev_bf16(b), lib.SF_TCGEN05)
-    big = torch.full((130, 160), -7.0, dtype=torch.bfloat16, device="cuda")
-    lib.nvfp4_gemm(qa.codes, qa.sf, qa.g, qb.codes, qb.sf, qb.g, 130, 140, 256, big, 160, lib.OUT_BF16)
+    big = torch.full((m + 40, 288), -7.0, dtype=torch.bfloat16, device="cuda")
+    lib.nvfp4_gemm(qa.codes, qa.sf, qa.g, qb.codes, qb.sf, qb.g, m, n, 256, big, 288, lib.OUT_BF16)
     torch.cuda.synchronize()
-    check_bf16(host_bf16_bits(big[:, :140]), d_ref, s_ref, alpha)
-    assert torch.all(big[:, 140:] == -7.0)
+    check_bf16(host_bf16_bits(big[:m, :n]), d_ref, s_ref, alpha)
+    assert torch.all(big[:m, n:] == -7.0)
+    assert torch.all(big[m:, :] == -7.0)
 
 
 def _probe(lib, m, n, k, a_sf_rowmajor, b_sf_rowmajor):
