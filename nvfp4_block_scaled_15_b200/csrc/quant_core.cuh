@@ -124,6 +124,76 @@ __device__ __forceinline__ uint32_t quantize_half_block(const uint4 v, const flo
   return e2m1x8(u[0], u[1], u[2], u[3]);
 }
 
+// ---------------------------------------------------------------------------
+// Whole-block form: one lane owns a 16-element block (8 words of bf16x2), so
+// the block amax needs no shuffle and per-block work is shared by 16 values.
+// ---------------------------------------------------------------------------
+
+// Shared-memory table of the positive E4M3 scales: entry s (0 <= s < 128)
+// holds {sd, RN(1/sd)} for sd the E4M3 value of byte s (RN(1/0) stored as 0).
+// __frcp_rn is the correctly rounded reciprocal.
+__device__ __forceinline__ void fill_scale_table(float2* table) {
+  for (int s = static_cast<int>(threadIdx.x); s < 128; s += static_cast<int>(blockDim.x)) {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(s), __NV_E4M3);
+    const float sd = __half2float(__half(h));
+    table[s] = make_float2(sd, sd > 0.0f ? __frcp_rn(sd) : 0.0f);
+  }
+}
+
+// |x| maximum of 16 bf16 values as a bf16 bit pattern without sign.  The
+// bf16 max keeps the larger magnitude exactly; with .NaN a NaN input gives a
+// NaN pattern, as the integer maximum of the magnitude bits would.
+__device__ __forceinline__ uint32_t abs_max_bits16(const uint32_t (&w)[8]) {
+  uint32_t m;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(w[0]), "r"(w[1]));
+#pragma unroll
+  for (int i = 2; i < 8; ++i) asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[i]));
+  m &= 0x7FFF7FFFu;
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// 16 codes of one block (element 0 in the low nibble of c.x) for the scale
+// entry e = {sd, RN(1/sd)}: RN(RN(x * g) / sd) by the FMA correction, then
+// E2M1 RNE with saturation; sd == 0 gives all-zero codes.
+__device__ __forceinline__ uint2 block_codes(const uint32_t (&w)[8], float g, float2 e) {
+  const float2 g2 = make_float2(g, g);
+  const float2 y2 = make_float2(e.y, e.y);
+  const float2 nsd2 = make_float2(-e.x, -e.x);
+  float2 u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 t = __fmul2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), g2);   // x * g
+    const float2 q = __fmul2_rn(t, y2);                                         // RN(t * RN(1/sd))
+    const float2 r = __ffma2_rn(q, nsd2, t);                                    // t - q * sd, exact
+    const float2 d = __ffma2_rn(r, y2, q);                                      // RN(t / sd)
+    u[i] = make_float2(copysignf(d.x, t.x), copysignf(d.y, t.y));
+  }
+  uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
+  if (e.x == 0.0f) c = make_uint2(0u, 0u);
+  return c;
+}
+
+// Two blocks at once: their E4M3 scales (s = RN_e4m3(RN(RN(amax_b * g) / 6)),
+// satfinite) go through the packed units and one paired conversion.
+__device__ __forceinline__ void quantize_two_blocks(const uint32_t (&w0)[8], const uint32_t (&w1)[8], float g,
+                                                    const float2* table, uint2& c0, uint2& c1, uint32_t& s0,
+                                                    uint32_t& s1) {
+  const float sixth = __frcp_rn(6.0f);
+  const float2 ab = make_float2(__uint_as_float(abs_max_bits16(w0) << 16), __uint_as_float(abs_max_bits16(w1) << 16));
+  const float2 t = __fmul2_rn(ab, make_float2(g, g));
+  const float2 q = __fmul2_rn(t, make_float2(sixth, sixth));
+  const float2 r = __ffma2_rn(q, make_float2(-6.0f, -6.0f), t);
+  const float2 sr = __ffma2_rn(r, make_float2(sixth, sixth), q);               // RN(t / 6)
+  uint32_t s2;
+  asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n\tcvt.u32.u16 %0, h;\n\t}"
+      : "=r"(s2)
+      : "f"(sr.y), "f"(sr.x));
+  s0 = s2 & 0xFFu;
+  s1 = (s2 >> 8) & 0xFFu;
+  c0 = block_codes(w0, g, table[s0 & 0x7Fu]);
+  c1 = block_codes(w1, g, table[s1 & 0x7Fu]);
+}
+
 // Byte offset of (row r, block b) in the tensor-core scale layout whose
 // padded block count is kb_pad (a multiple of 4).
 __host__ __device__ __forceinline__ int64_t sf_tc_offset(int64_t r, int64_t b, int64_t kb_pad) {

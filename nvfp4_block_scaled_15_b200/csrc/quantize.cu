@@ -1,8 +1,8 @@
 // NVFP4 quantization kernels: tensor amax, two-level block quantization and
 // the re-layout of block scales into the tensor-core scale format.
 //
-// Both passes stream HBM with 128-bit loads; each thread owns half of a
-// 16-element block and its neighbour lane the other half ("NVIDIA NVFP4 与
+// Both passes stream HBM with wide loads; in the quantize pass each thread
+// owns whole 16-element blocks ("NVIDIA NVFP4 与
 // Micro-Scaling" section 三: global scale from |X|_max, then per-block
 // micro-scales; "low-precision-floats" section FP4 / MXFP4 / NVFP4 formulas).
 #include <cuda_runtime.h>
@@ -55,56 +55,99 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
   }
 }
 
-// Pass 2: block scales and codes.  blockIdx.x = row (rows_alloc >= rows; the
-// extra rows only exist in the tensor-core layout and get zero scales),
-// blockIdx.y = row segment of kSegChunks chunks.
-template <bool kTcLayout>
+// Pass 2: block scales and codes.  Each thread owns two whole 16-element
+// blocks of one row (b0 = segment * kSegBlocks + thread, b1 = b0 + kThreads),
+// so a warp reads 1 KB of contiguous input per load.  One CTA per (row,
+// segment of kSegBlocks blocks); rows_alloc >= rows (the extra rows only exist
+// in the tensor-core layout and get zero scales).  Rows are taken last to
+// first: the amax pass read them first to last, so the rows it read last are
+// the ones most likely still in L2 when this pass starts.
+// kWide: x and its row pitch are 32-B aligned, each block is one 256-bit load.
+constexpr int kSegBlocks = 2 * kThreads;
+
+template <bool kWide>
+__device__ __forceinline__ void load_block(const uint16_t* p, uint32_t (&w)[8]) {
+  if (kWide) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+  } else {
+    const uint4 a = ld_stream(reinterpret_cast<const uint4*>(p));
+    const uint4 b = ld_stream(reinterpret_cast<const uint4*>(p) + 1);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+}
+
+template <bool kTcLayout, bool kWide>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                             int64_t ldx, uint8_t* __restrict__ codes,
                                                             uint8_t* __restrict__ sf, float* __restrict__ g_out,
                                                             const float* __restrict__ amax_in,
                                                             int* __restrict__ status) {
-  const int r = blockIdx.x;
-  const int chunks = k >> 3;
+  __shared__ float2 table[128];
+  const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
   const int kb = k >> 4;                      // blocks per row
-  const int lane = threadIdx.x & 31;
-  const int c0 = blockIdx.y * kSegChunks + threadIdx.x;
+  const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
+  const int b1 = b0 + kThreads;
 
-  const float sixth = __frcp_rn(6.0f);
-  const float rtab = recip_table_lane();
   bool valid;
-  const float g = global_scale_from_amax(*amax_in, valid);
+  float g = global_scale_from_amax(*amax_in, valid);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     *g_out = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
+  if (!valid) g = 0.0f;                        // all-zero codes and scales
   const bool real_row = r < rows;
-  // tensor-core layout: byte of (row r, block b) = row_base + (b / 4) * 512 + b % 4
-  const int64_t row_base = (static_cast<int64_t>(r >> 7) * (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
 
-  uint4 v[kUnroll];
+  uint32_t w0[8], w1[8];
+  const uint16_t* xr = x + static_cast<int64_t>(r) * ldx;
+  if (real_row && valid && b0 < kb) {
+    load_block<kWide>(xr + b0 * 16, w0);
+  } else {
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    const int c = c0 + u * kThreads;
-    v[u] = (real_row && valid && c < chunks)
-               ? ld_stream(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx) + c)
-               : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 8; ++i) w0[i] = 0u;
   }
+  if (real_row && valid && b1 < kb) {
+    load_block<kWide>(xr + b1 * 16, w1);
+  } else {
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    const int c = c0 + u * kThreads;          // chunk index, 2 chunks per block
-    uint32_t s;
-    uint32_t q = quantize_half_block(v[u], valid ? g : 0.0f, s, sixth, rtab);
-    if (!valid) { q = 0; s = 0; }
-    if (!real_row) s = 0;
-    const bool in_row = c < chunks;
-    if (real_row && in_row) reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(r) * (k >> 1))[c] = q;
-    const int b = c >> 1;                     // block index in the row
-    if (!kTcLayout) {
-      if (real_row && in_row && (lane & 1) == 0) sf[static_cast<int64_t>(r) * kb + b] = static_cast<uint8_t>(s);
+    for (int i = 0; i < 8; ++i) w1[i] = 0u;
+  }
+  fill_scale_table(table);                    // overlaps the loads in flight
+  __syncthreads();
+
+  uint2 c0, c1;
+  uint32_t s0, s1;
+  quantize_two_blocks(w0, w1, g, table, c0, c1, s0, s1);
+
+  if (real_row) {
+    uint8_t* cr = codes + static_cast<int64_t>(r) * (k >> 1);
+    if ((reinterpret_cast<uintptr_t>(codes) & 7u) == 0) {
+      if (b0 < kb) *reinterpret_cast<uint2*>(cr + b0 * 8) = c0;
+      if (b1 < kb) *reinterpret_cast<uint2*>(cr + b1 * 8) = c1;
     } else {
-      if (in_row && (lane & 1) == 0) sf[row_base + ((b >> 2) << 9) + (b & 3)] = static_cast<uint8_t>(s);
+      if (b0 < kb) {
+        reinterpret_cast<uint32_t*>(cr + b0 * 8)[0] = c0.x;
+        reinterpret_cast<uint32_t*>(cr + b0 * 8)[1] = c0.y;
+      }
+      if (b1 < kb) {
+        reinterpret_cast<uint32_t*>(cr + b1 * 8)[0] = c1.x;
+        reinterpret_cast<uint32_t*>(cr + b1 * 8)[1] = c1.y;
+      }
     }
+  }
+  if (!kTcLayout) {
+    if (real_row) {
+      uint8_t* sr = sf + static_cast<int64_t>(r) * kb;
+      if (b0 < kb) sr[b0] = static_cast<uint8_t>(s0);
+      if (b1 < kb) sr[b1] = static_cast<uint8_t>(s1);
+    }
+  } else {
+    // byte of (row r, block b) = row_base + (b / 4) * 512 + b % 4
+    const int64_t row_base = (static_cast<int64_t>(r >> 7) * (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+    if (b0 < kb) sf[row_base + ((b0 >> 2) << 9) + (b0 & 3)] = static_cast<uint8_t>(s0);
+    if (b1 < kb) sf[row_base + ((b1 >> 2) << 9) + (b1 & 3)] = static_cast<uint8_t>(s1);
   }
 }
 
@@ -144,24 +187,30 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx
                              nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, cudaStream_t s) {
   int* status = device_status_ptr();
   if (!status) return NVFP4_ERR_CUDA;
-  const int segs = static_cast<int>((k / 8 + kSegChunks - 1) / kSegChunks);
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  uint8_t* cs = static_cast<uint8_t*>(codes);
+  uint8_t* ss = static_cast<uint8_t*>(sf);
+  const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
   const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
   if (grid_rows == 0 || segs == 0) {
     // nothing to quantize: still publish g (from the given amax)
-    quantize_kernel<false><<<dim3(1, 1), kThreads, 0, s>>>(static_cast<const uint16_t*>(x), 0, 0, ldx,
-                                                           static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf),
-                                                           g_dev, amax_dev, status);
+    quantize_kernel<false, false><<<dim3(1, 1), kThreads, 0, s>>>(xs, 0, 0, ldx, cs, ss, g_dev, amax_dev, status);
     return launch_status(cudaGetLastError());
   }
-  dim3 grid(static_cast<unsigned>(grid_rows), segs);
-  if (layout == NVFP4_SF_TCGEN05)
-    quantize_kernel<true><<<grid, kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
-                                                    static_cast<int>(k), ldx, static_cast<uint8_t*>(codes),
-                                                    static_cast<uint8_t*>(sf), g_dev, amax_dev, status);
-  else
-    quantize_kernel<false><<<grid, kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
-                                                     static_cast<int>(k), ldx, static_cast<uint8_t*>(codes),
-                                                     static_cast<uint8_t*>(sf), g_dev, amax_dev, status);
+  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  const int ir = static_cast<int>(rows), ik = static_cast<int>(k);
+  if (layout == NVFP4_SF_TCGEN05) {
+    if (wide)
+      quantize_kernel<true, true><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
+    else
+      quantize_kernel<true, false><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
+  } else {
+    if (wide)
+      quantize_kernel<false, true><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
+    else
+      quantize_kernel<false, false><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
+  }
   return launch_status(cudaGetLastError());
 }
 
