@@ -669,9 +669,9 @@ struct GemvParams {
 // same moment read different column offsets of the 4-KiB-strided weight rows
 // instead of all hitting the same DRAM channels.  A bijection on a tile's
 // stages: stream-K ranges still partition each tile's K.
-__device__ __forceinline__ int gv_stage_k(int64_t u, int tile, int num_kt) {
-  const int raw = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
-  const int off = static_cast<int>((static_cast<int64_t>(tile) * 7) % num_kt);
+__device__ __forceinline__ int gv_stage_k(int u, int tile, int num_kt) {
+  const int raw = u - tile * num_kt;
+  const int off = (tile * 7) % num_kt;
   const int k = raw + off;
   return k >= num_kt ? k - num_kt : k;
 }
@@ -717,9 +717,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int64_t units = static_cast<int64_t>(p.tiles) * p.num_kt;
-  const int64_t u_begin = units * blockIdx.x / gridDim.x;
-  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+  // unit counts fit in int (checked at launch)
+  const int units = p.tiles * p.num_kt;
+  const int u_begin = static_cast<int>(static_cast<int64_t>(units) * blockIdx.x / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<int64_t>(units) * (blockIdx.x + 1) / gridDim.x);
   const int ksteps_total = p.K / MMA_K;
 
   if (warp == 0) {
@@ -727,26 +728,28 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
+      const uint64_t stream = l2_evict_first_policy();   // weights are read once
       // weights do not depend on the prologue: fill the ring with them first
-      const int64_t pre_end = min(u_end, u_begin + GV_STAGES);
-      for (int64_t u = u_begin; u < pre_end; ++u) {
-        const int tile = static_cast<int>(u / p.num_kt);
+      const int pre_end = min(u_end, u_begin + GV_STAGES);
+      for (int u = u_begin; u < pre_end; ++u) {
+        const int tile = u / p.num_kt;
         const int kt = gv_stage_k(u, tile, p.num_kt);
         const int nk = min(4, ksteps_total - kt * 4);
-        const int s = static_cast<int>(u - u_begin);
+        const int s = u - u_begin;
         uint8_t* sA = smem + s * GV_STAGE_BYTES;
         uint8_t* sSFA = sA + GV_A_BYTES + GV_B_BYTES;
         mbar_arrive_expect_tx(&full[s], GV_A_BYTES + GV_B_BYTES + 2 * nk * SF_ATOM);
-        tma_load_2d(sA, &tmW, &full[s], kt * BK_BYTES, tile * BM);
-        bulk_load(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[s]);
+        tma_load_2d_hint(sA, &tmW, &full[s], kt * BK_BYTES, tile * BM, stream);
+        bulk_load_hint(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[s],
+                       stream);
       }
       // activations, their scales: only once the prologue grid has finished
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int64_t u = u_begin; u < pre_end; ++u) {
-        const int tile = static_cast<int>(u / p.num_kt);
+      for (int u = u_begin; u < pre_end; ++u) {
+        const int tile = u / p.num_kt;
         const int kt = gv_stage_k(u, tile, p.num_kt);
         const int nk = min(4, ksteps_total - kt * 4);
-        const int s = static_cast<int>(u - u_begin);
+        const int s = u - u_begin;
         uint8_t* sB = smem + s * GV_STAGE_BYTES + GV_A_BYTES;
         uint8_t* sSFB = sB + GV_B_BYTES + 4 * SF_ATOM;
         tma_load_2d(sB, &tmX, &full[s], kt * BK_BYTES, 0);
@@ -757,8 +760,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
           phase ^= 1;
         }
       }
-      for (int64_t u = pre_end; u < u_end; ++u) {
-        const int tile = static_cast<int>(u / p.num_kt);
+      for (int u = pre_end; u < u_end; ++u) {
+        const int tile = u / p.num_kt;
         const int kt = gv_stage_k(u, tile, p.num_kt);
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
         const int nk = min(4, ksteps_total - kt * 4);
@@ -767,9 +770,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         uint8_t* sSFA = sB + GV_B_BYTES;
         uint8_t* sSFB = sSFA + 4 * SF_ATOM;
         mbar_arrive_expect_tx(&full[stage], GV_A_BYTES + GV_B_BYTES + 2 * nk * SF_ATOM);
-        tma_load_2d(sA, &tmW, &full[stage], kt * BK_BYTES, tile * BM);
+        tma_load_2d_hint(sA, &tmW, &full[stage], kt * BK_BYTES, tile * BM, stream);
         tma_load_2d(sB, &tmX, &full[stage], kt * BK_BYTES, 0);
-        bulk_load(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[stage]);
+        bulk_load_hint(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM,
+                       &full[stage], stream);
         bulk_load(sSFB, p.xsf + static_cast<int64_t>(kt) * 4 * SF_ATOM, nk * SF_ATOM, &full[stage]);
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -791,11 +795,11 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       const uint32_t idesc = idesc_mxf4nvf4(BM, GV_N);
-      int64_t u = u_begin;
+      int u = u_begin;
       bool ok = true;
       while (u < u_end && ok) {
-        const int tile = static_cast<int>(u / p.num_kt);
-        const int64_t seg_end = min(u_end, static_cast<int64_t>(tile + 1) * p.num_kt);
+        const int tile = u / p.num_kt;
+        const int seg_end = min(u_end, (tile + 1) * p.num_kt);
         if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * GV_N;
@@ -853,11 +857,11 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     const int cta = blockIdx.x;
     int acc = 0;
     uint32_t acc_phase = 0;
-    int64_t u = u_begin;
+    int u = u_begin;
     while (u < u_end) {
-      const int tile = static_cast<int>(u / p.num_kt);
-      const int64_t tile_begin = static_cast<int64_t>(tile) * p.num_kt;
-      const int64_t seg_end = min(u_end, tile_begin + p.num_kt);
+      const int tile = u / p.num_kt;
+      const int tile_begin = tile * p.num_kt;
+      const int seg_end = min(u_end, tile_begin + p.num_kt);
       const bool has_head = u == tile_begin;                    // this segment holds the tile's first stage
       const bool has_tail = seg_end == tile_begin + p.num_kt;   // ... and its last stage
       u = seg_end;
@@ -919,18 +923,27 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 }
 
 // Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
-// clearing of the fix-up counters.  Launched in clusters of GP_CLUSTER CTAs:
-//   cluster 0: CTA c owns activation rows c, c+8, c+16, c+24.  Each CTA
-//     reduces the amax of its real rows, the cluster exchanges the partial
-//     maxima through distributed shared memory, then every CTA quantizes its
-//     real rows and zeroes its padding rows (codes and scales);
-//   other clusters: clear the tile counters.
+// clearing of the fix-up counters, in one cluster of GP_CLUSTER CTAs.  CTA c
+// owns activation rows c, c+8, c+16, c+24 (those below M): it reduces the
+// amax of its rows, the cluster exchanges the partial maxima through
+// distributed shared memory, then each CTA quantizes its rows (two whole
+// 16-element blocks per thread at a time).  Only real rows are written: a
+// padding row r (M <= r < 32) of the activation operand only feeds output
+// column r of the MMA, which is never stored, so its contents do not matter.
 // It lets the dependent GEMV grid launch at once (programmatic dependent
 // launch): the GEMV streams weights while this runs and waits for it only
 // before it touches the activations, g_x or the partial sums.
 constexpr int GP_THREADS = 256;
 constexpr int GP_CLUSTER = 8;
-constexpr int GP_ZERO_CLUSTERS = 1;
+constexpr int GP_ROWS = GV_N / GP_CLUSTER;    // activation rows per CTA
+static_assert(GP_ROWS == 4, "row selection below assumes four rows per CTA");
+
+__device__ __forceinline__ void gp_load_block(const uint16_t* p, uint32_t (&w)[8]) {
+  const uint4 a = reinterpret_cast<const uint4*>(p)[0];
+  const uint4 b = reinterpret_cast<const uint4*>(p)[1];
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+}
 
 __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                    int64_t ldx, uint8_t* __restrict__ xq,
@@ -938,36 +951,52 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
                                                                    int* __restrict__ counters, int n_counters,
                                                                    int* __restrict__ status) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  if (blockIdx.x >= GP_CLUSTER) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x - GP_CLUSTER) * GP_THREADS;
-    const int64_t first = static_cast<int64_t>(blockIdx.x - GP_CLUSTER) * GP_THREADS + tid;
-    for (int64_t i = first; i < n_counters; i += stride) counters[i] = 0;
-    return;
-  }
-  const int c = static_cast<int>(cluster_ctarank());
-  const int chunks = K >> 3;                 // 16-B chunks per row (a multiple of 8)
-  const int kb = K >> 4;
+  __shared__ float2 table[128];
   __shared__ uint32_t red[GP_THREADS / 32];
   __shared__ uint32_t partial;
-  // amax of this CTA's real rows
+  __shared__ uint32_t cluster_max;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int c = static_cast<int>(cluster_ctarank());
+  const int kb = K >> 4;                     // 16-element blocks per row
+
+  // amax of this CTA's rows.  Rows of up to 2 * GP_THREADS blocks stay in
+  // registers (two blocks per thread) for the quantization below; longer
+  // rows are read again from L2.
+  const bool resident = kb <= 2 * GP_THREADS;
+  uint32_t wr[GP_ROWS][2][8];
   uint32_t mx = 0;
-  for (int r = c; r < M; r += GP_CLUSTER) {
-    const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
-    for (int base = 0; base < chunks; base += 4 * GP_THREADS) {
-      uint4 v[4];
+  if (resident) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + u * GP_THREADS + tid;
-        v[u] = i < chunks ? row[i] : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < GP_ROWS; ++i) {
+      const int r = c + i * GP_CLUSTER;
+      const uint16_t* row = x + static_cast<int64_t>(r) * ldx;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int b = tid + h * GP_THREADS;
+        if (r < M && b < kb) {
+          gp_load_block(row + b * 16, wr[i][h]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) wr[i][h][q] = 0u;
+        }
       }
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) mx = max(mx, abs_max_bits8(v[u]));
+    for (int i = 0; i < GP_ROWS; ++i) mx = max(mx, max(abs_max_bits16(wr[i][0]), abs_max_bits16(wr[i][1])));
+  } else {
+    for (int r = c; r < M; r += GP_CLUSTER) {
+      const uint16_t* row = x + static_cast<int64_t>(r) * ldx;
+      for (int b = tid; b < kb; b += GP_THREADS) {
+        uint32_t w[8];
+        gp_load_block(row + b * 16, w);
+        mx = max(mx, abs_max_bits16(w));
+      }
     }
   }
   mx = __reduce_max_sync(0xFFFFFFFFu, mx);
   if (lane == 0) red[tid >> 5] = mx;
+  fill_scale_table(table);
   __syncthreads();
   if (tid < 32) {
     uint32_t t = lane < GP_THREADS / 32 ? red[lane] : 0u;
@@ -975,56 +1004,82 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
     if (tid == 0) partial = t;
   }
   __syncwarp();
-  cluster_sync_all();                        // every CTA's partial is visible cluster-wide
-  __shared__ uint32_t cluster_max;
+  // No global store precedes this barrier, so its release arrive does not wait
+  // on memory traffic: it only publishes `partial` to the cluster.
+  cluster_sync_all();
   if (tid < 32) {
     uint32_t all = tid < GP_CLUSTER ? ld_shared_cluster_u32(mapa_shared(smem_u32(&partial), tid)) : 0u;
     all = __reduce_max_sync(0xFFFFFFFFu, all);
     if (tid == 0) cluster_max = all;
   }
-  __syncthreads();
-  const uint32_t all = cluster_max;
+  __syncthreads();                           // cluster_max visible to the CTA
+  cluster_sync_relaxed();                    // peers' partials read: CTAs may leave from here on
+  for (int i = c * GP_THREADS + tid; i < n_counters; i += GP_CLUSTER * GP_THREADS) counters[i] = 0;
   bool valid;
-  const float g = global_scale_from_amax(__uint_as_float(all << 16), valid);
+  float g = global_scale_from_amax(__uint_as_float(cluster_max << 16), valid);
   if (c == 0 && tid == 0) {
     *g_x = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
-  // quantize this CTA's real rows; padding rows (M <= r < 32) get zero codes
-  // and scales.  Rows 32..127 of the scale layout are padding too: each 16-B
-  // chunk (r % 32) of an atom holds rows r, r+32, r+64, r+96, so writing the
-  // chunk of row r < 32 whole (its 4 scales, then 12 zero bytes) also clears them.
-  const float sixth = __frcp_rn(6.0f);
-  const float rtab = recip_table_lane();
-  for (int r = c; r < GV_N; r += GP_CLUSTER) {
-    uint4* chunk_row = reinterpret_cast<uint4*>(xsf) + r;       // + 32 * atom
-    if (r >= M || !valid) {
-      uint4* qrow = reinterpret_cast<uint4*>(xq + static_cast<int64_t>(r) * (K >> 1));
-      for (int i = tid; i < (K >> 5); i += GP_THREADS) qrow[i] = make_uint4(0, 0, 0, 0);
-      for (int j = tid; j < (kb >> 2); j += GP_THREADS) chunk_row[32 * j] = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-    const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
-    uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(r) * (K >> 1));
-    // every lane runs every iteration (the quantizer shuffles across the warp);
-    // only the loads and stores are predicated.  chunks % 8 == 0, so each
-    // group of 8 lanes that gathers 4 block scales is entirely in or out.
-    for (int base = 0; base < chunks; base += GP_THREADS) {
-      const int i = base + tid;
-      const bool in = i < chunks;
-      const uint4 v = in ? row[i] : make_uint4(0, 0, 0, 0);
-      uint32_t s;
-      const uint32_t q = quantize_half_block(v, g, s, sixth, rtab);
-      if (in) qrow[i] = q;
-      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
-      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 4);
-      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 6);
-      if (in && (lane & 7) == 0)                                // atom i / 8 of row r
-        chunk_row[32 * (i >> 3)] = make_uint4(s | (s1 << 8) | (s2 << 16) | (s3 << 24), 0u, 0u, 0u);
+  if (!valid) g = 0.0f;                      // all-zero codes and scales
+
+  // quantize this CTA's rows.  Scale of (row r < 32, block b) in the padded
+  // 128-row scale layout: byte (b / 4) * 512 + r * 16 + b % 4; the other 12
+  // bytes of that 16-B chunk belong to rows r + 32, r + 64, r + 96 (absent
+  // from the N = 32 operand) and are written as zeros.
+  for (int i = 0; i < GP_ROWS; ++i) {
+    const int r = c + i * GP_CLUSTER;
+    if (r >= M) break;
+    const uint16_t* row = x + static_cast<int64_t>(r) * ldx;
+    uint8_t* qrow = xq + static_cast<int64_t>(r) * (K >> 1);
+    for (int b0 = tid; b0 < kb; b0 += 2 * GP_THREADS) {
+      const int b1 = b0 + GP_THREADS;
+      uint32_t w0[8], w1[8];
+      if (resident) {
+        // wr[i] held by a run-time row index: select through a switch so the
+        // array stays in registers
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          w0[q] = i == 0 ? wr[0][0][q] : i == 1 ? wr[1][0][q] : i == 2 ? wr[2][0][q] : wr[3][0][q];
+          w1[q] = i == 0 ? wr[0][1][q] : i == 1 ? wr[1][1][q] : i == 2 ? wr[2][1][q] : wr[3][1][q];
+        }
+      } else {
+        gp_load_block(row + b0 * 16, w0);
+        if (b1 < kb) {
+          gp_load_block(row + b1 * 16, w1);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) w1[q] = 0u;
+        }
+      }
+      if (!valid) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          w0[q] = 0u;
+          w1[q] = 0u;
+        }
+      }
+      uint2 c0, c1;
+      uint32_t s0, s1;
+      quantize_two_blocks(w0, w1, g, table, c0, c1, s0, s1);
+      *reinterpret_cast<uint2*>(qrow + b0 * 8) = c0;
+      uint8_t* chunk0 = xsf + (b0 >> 2) * 512 + r * 16;
+      chunk0[b0 & 3] = static_cast<uint8_t>(s0);
+      if ((b0 & 3) == 0) {
+        uint32_t* z = reinterpret_cast<uint32_t*>(chunk0);
+        z[1] = 0u; z[2] = 0u; z[3] = 0u;
+      }
+      if (b1 < kb) {
+        *reinterpret_cast<uint2*>(qrow + b1 * 8) = c1;
+        uint8_t* chunk1 = xsf + (b1 >> 2) * 512 + r * 16;
+        chunk1[b1 & 3] = static_cast<uint8_t>(s1);
+        if ((b1 & 3) == 0) {
+          uint32_t* z = reinterpret_cast<uint32_t*>(chunk1);
+          z[1] = 0u; z[2] = 0u; z[3] = 0u;
+        }
+      }
     }
   }
-  __syncwarp();
-  cluster_sync_all();                        // no CTA leaves while a peer may still read its partial
 }
 
 // ---------------------------------------------------------------------------
@@ -1234,6 +1289,8 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
   int* cnt = reinterpret_cast<int*>(base + L.cnt);
   const int tiles = static_cast<int>((N + BM - 1) / BM);
   const int sms = device_sm_count();
+  const int64_t num_kt = (K + BK - 1) / BK;
+  if (static_cast<int64_t>(tiles) * num_kt > (int64_t{1} << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
 
   int* status = device_status_ptr();
   if (!status) return NVFP4_ERR_CUDA;
@@ -1244,7 +1301,7 @@ nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_co
     pattr[0].val.clusterDim.x = GP_CLUSTER;
     pattr[0].val.clusterDim.y = 1;
     pattr[0].val.clusterDim.z = 1;
-    pcfg.gridDim = dim3(GP_CLUSTER * (1 + GP_ZERO_CLUSTERS));
+    pcfg.gridDim = dim3(GP_CLUSTER);
     pcfg.blockDim = dim3(GP_THREADS);
     pcfg.stream = s;
     pcfg.attrs = pattr;
