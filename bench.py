@@ -41,7 +41,7 @@ FLOPS_STEP = 2.0 * M * N * K
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0            # nominal dense ratio (9 PFLOP/s FP4 : 2.25 PFLOP/s BF16)
-GEMM_SOURCES = ["gemm.cu", "ptx.cuh"]
+GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "tc_common.cuh"]
 
 
 def parse_args():

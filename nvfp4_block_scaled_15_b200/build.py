@@ -13,8 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnvfp4.so")
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "gemv_noalloc.cu"]
-HEADERS = ["internal.h", "ptx.cuh", "quant_core.cuh"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "gemv.cu", "gemv_noalloc.cu"]
+HEADERS = ["internal.h", "ptx.cuh", "quant_core.cuh", "tc_common.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

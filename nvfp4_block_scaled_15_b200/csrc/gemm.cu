@@ -24,18 +24,37 @@
 
 #include "internal.h"
 #include "ptx.cuh"
-#include "quant_core.cuh"
+#include "tc_common.cuh"
 
 namespace nvfp4 {
 
-namespace {
+// Tensor-map encoders declared in tc_common.cuh (the GEMV uses them too).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
 
-constexpr int BM = 128;          // rows of A per tile (MMA M)
-constexpr int BK = 256;          // K elements per pipeline stage (128 B of codes per row)
-constexpr int BK_BYTES = BK / 2;
-constexpr int MMA_K = 64;        // K per tcgen05.mma for kind::mxf4nvf4
-constexpr int SF_ATOM = 512;     // bytes of one 128-row x 4-block scale atom
-constexpr uint32_t TMEM_COLS = 512;
+bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
 
 // ---------------------------------------------------------------------------
 // GEMM configuration
@@ -80,19 +99,6 @@ struct GemmParams {
 
 __host__ __device__ __forceinline__ int round_up_int(int a, int b) { return (a + b - 1) / b * b; }
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// smem descriptor of a 128-B swizzled, K-major code tile (8-row groups 1024 B apart)
-__device__ __forceinline__ uint64_t code_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
-// smem descriptor of one 512-B scale atom read as 32 rows x 16 B (no swizzle)
-__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
 
 template <int NV>
 __device__ __forceinline__ void store_row(const GemmParams& p, int row, int col0, const uint32_t (&v)[NV],
@@ -629,489 +635,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Decode GEMV: swap-AB (weights are the 128-row MMA operand, the <= 32
-// activation rows the N = 32 operand) with stream-K over (row tile, K stage)
-// units so all SMs stream weights evenly.  Partial sums meet in an fp32
-// workspace; the CTA that completes a row tile writes its bf16 outputs.
-// ---------------------------------------------------------------------------
-constexpr int GV_N = 32;                      // MMA N (activation rows, zero-padded)
-constexpr int GV_STAGES = 8;
-constexpr int GV_A_BYTES = BM * BK_BYTES;     // weights
-constexpr int GV_B_BYTES = GV_N * BK_BYTES;   // activations
-constexpr int GV_STAGE_BYTES = GV_A_BYTES + GV_B_BYTES + 2 * 4 * SF_ATOM;
-constexpr int GV_ACC_BUFS = 2;
-constexpr int GV_SF_BASE = GV_ACC_BUFS * GV_N;
-constexpr int GV_SF_COLS_PER_STAGE = 32;      // 16 for A, 16 for B (one 4-column atom per MMA-K)
-constexpr int GV_EPI_WARPS = 4;
-constexpr int GV_THREADS = (2 + GV_EPI_WARPS) * 32;
-constexpr int GV_SMEM_BYTES = GV_STAGES * GV_STAGE_BYTES + 256 + 1024;
-static_assert(GV_SF_BASE + GV_STAGES * GV_SF_COLS_PER_STAGE <= (int)TMEM_COLS, "TMEM budget");
-
-struct GemvParams {
-  const uint8_t* wsf;      // weight scales, tensor-core layout
-  const uint8_t* xsf;      // activation scales, tensor-core layout (128 padded rows)
-  const float* g_w;
-  const float* g_x;
-  float* partials;         // [2 * grid][M][128] fp32: slot 2c = CTA c's first segment, 2c+1 its last
-  int* counters;           // [tiles * 4] arrivals per (weight tile, 32-row quarter); cleared by the prologue
-  __nv_bfloat16* y;
-  int64_t ldy;
-  int M, N, K;
-  int kb4;
-  int tiles;
-  int num_kt;
-  uint64_t wait_limit_ns;
-  int* status;
-};
-
-// K stage of unit u (of weight tile `tile`).  Each tile walks its K stages
-// from a tile-dependent start, so the CTAs streaming different tiles at the
-// same moment read different column offsets of the 4-KiB-strided weight rows
-// instead of all hitting the same DRAM channels.  A bijection on a tile's
-// stages: stream-K ranges still partition each tile's K.
-__device__ __forceinline__ int gv_stage_k(int u, int tile, int num_kt) {
-  const int raw = u - tile * num_kt;
-  const int off = (tile * 7) % num_kt;
-  const int k = raw + off;
-  return k >= num_kt ? k - num_kt : k;
-}
-
-__global__ void __launch_bounds__(GV_THREADS, 1)
-    gemv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                const GemvParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + GV_STAGES * GV_STAGE_BYTES);
-  uint64_t* empty = full + GV_STAGES;
-  uint64_t* acc_full = empty + GV_STAGES;
-  uint64_t* acc_empty = acc_full + GV_ACC_BUFS;
-  uint64_t* mma_done = acc_empty + GV_ACC_BUFS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < GV_STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < GV_ACC_BUFS; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], GV_EPI_WARPS);
-    }
-    mbar_init(mma_done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmW);
-    prefetch_tmap(&tmX);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  // unit counts fit in int (checked at launch)
-  const int units = p.tiles * p.num_kt;
-  const int u_begin = static_cast<int>(static_cast<int64_t>(units) * blockIdx.x / gridDim.x);
-  const int u_end = static_cast<int>(static_cast<int64_t>(units) * (blockIdx.x + 1) / gridDim.x);
-  const int ksteps_total = p.K / MMA_K;
-
-  if (warp == 0) {
-    if (elect_one()) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_parity = 0;
-      const uint64_t stream = l2_evict_first_policy();   // weights are read once
-      // weights do not depend on the prologue: fill the ring with them first
-      const int pre_end = min(u_end, u_begin + GV_STAGES);
-      for (int u = u_begin; u < pre_end; ++u) {
-        const int tile = u / p.num_kt;
-        const int kt = gv_stage_k(u, tile, p.num_kt);
-        const int nk = min(4, ksteps_total - kt * 4);
-        const int s = u - u_begin;
-        uint8_t* sA = smem + s * GV_STAGE_BYTES;
-        uint8_t* sSFA = sA + GV_A_BYTES + GV_B_BYTES;
-        mbar_arrive_expect_tx(&full[s], GV_A_BYTES + GV_B_BYTES + 2 * nk * SF_ATOM);
-        tma_load_2d_hint(sA, &tmW, &full[s], kt * BK_BYTES, tile * BM, stream);
-        bulk_load_hint(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[s],
-                       stream);
-      }
-      // activations, their scales: only once the prologue grid has finished
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int u = u_begin; u < pre_end; ++u) {
-        const int tile = u / p.num_kt;
-        const int kt = gv_stage_k(u, tile, p.num_kt);
-        const int nk = min(4, ksteps_total - kt * 4);
-        const int s = u - u_begin;
-        uint8_t* sB = smem + s * GV_STAGE_BYTES + GV_A_BYTES;
-        uint8_t* sSFB = sB + GV_B_BYTES + 4 * SF_ATOM;
-        tma_load_2d(sB, &tmX, &full[s], kt * BK_BYTES, 0);
-        bulk_load(sSFB, p.xsf + static_cast<int64_t>(kt) * 4 * SF_ATOM, nk * SF_ATOM, &full[s]);
-        issued_mask |= 1u << s;
-        if (++stage == GV_STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      for (int u = pre_end; u < u_end; ++u) {
-        const int tile = u / p.num_kt;
-        const int kt = gv_stage_k(u, tile, p.num_kt);
-        if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
-        const int nk = min(4, ksteps_total - kt * 4);
-        uint8_t* sA = smem + stage * GV_STAGE_BYTES;
-        uint8_t* sB = sA + GV_A_BYTES;
-        uint8_t* sSFA = sB + GV_B_BYTES;
-        uint8_t* sSFB = sSFA + 4 * SF_ATOM;
-        mbar_arrive_expect_tx(&full[stage], GV_A_BYTES + GV_B_BYTES + 2 * nk * SF_ATOM);
-        tma_load_2d_hint(sA, &tmW, &full[stage], kt * BK_BYTES, tile * BM, stream);
-        tma_load_2d(sB, &tmX, &full[stage], kt * BK_BYTES, 0);
-        bulk_load_hint(sSFA, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM,
-                       &full[stage], stream);
-        bulk_load(sSFB, p.xsf + static_cast<int64_t>(kt) * 4 * SF_ATOM, nk * SF_ATOM, &full[stage]);
-        issued_mask |= 1u << stage;
-        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == GV_STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      for (int s = 0; s < GV_STAGES; ++s)
-        if (issued_mask & (1u << s)) {
-          volatile int no_abort = 0;
-          (void)mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &no_abort, p.wait_limit_ns, p.status);
-        }
-    }
-  } else if (warp == 1) {
-    if (elect_one()) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      const uint32_t idesc = idesc_mxf4nvf4(BM, GV_N);
-      int u = u_begin;
-      bool ok = true;
-      while (u < u_end && ok) {
-        const int tile = u / p.num_kt;
-        const int seg_end = min(u_end, (tile + 1) * p.num_kt);
-        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * GV_N;
-        bool first = true;
-        for (; u < seg_end; ++u) {
-          const int kt = gv_stage_k(u, tile, p.num_kt);
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int nk = min(4, ksteps_total - kt * 4);
-          const uint32_t sA = smem_u32(smem + stage * GV_STAGE_BYTES);
-          const uint32_t sB = sA + GV_A_BYTES;
-          const uint32_t sSFA = sB + GV_B_BYTES;
-          const uint32_t sSFB = sSFA + 4 * SF_ATOM;
-          const uint32_t tsfa = tmem_base + GV_SF_BASE + stage * GV_SF_COLS_PER_STAGE;
-          const uint32_t tsfb = tsfa + 16;
-          for (int j = 0; j < nk; ++j) {
-            tc_cp_32x128b_warpx4(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
-            tc_cp_32x128b_warpx4(tsfb + j * 4, sf_desc(sSFB + j * SF_ATOM));
-          }
-          for (int j = 0; j < nk; ++j) {
-            mma_mxf4nvf4(d_tmem, code_desc(sA + j * (MMA_K / 2)), code_desc(sB + j * (MMA_K / 2)), idesc,
-                         tsfa + j * 4, tsfb + j * 4, first ? 0u : 1u);
-            first = false;
-          }
-          tc_commit(&empty[stage]);
-          if (++stage == GV_STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) break;
-        tc_commit(&acc_full[acc]);
-        if (++acc == GV_ACC_BUFS) {
-          acc = 0;
-          acc_phase ^= 1;
-        }
-      }
-      tc_commit(mma_done);
-      volatile int no_abort = 0;
-      (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
-    }
-  } else {
-    // Stream-K fix-up.  Ranges hold at least num_kt units (grid <= tiles), so
-    // a weight tile has at most two contributors: the CTA holding its first
-    // stages and the next CTA holding the rest.  A CTA that covers a whole
-    // tile writes bf16 outputs directly; a split tile's two partial sums meet
-    // in the partial slots, and whichever contributor arrives second adds
-    // them (fp32 addition commutes: the result does not depend on who).
-    const int quad = warp & 3;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_w, *p.g_x));
-    const int cta = blockIdx.x;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    int u = u_begin;
-    while (u < u_end) {
-      const int tile = u / p.num_kt;
-      const int tile_begin = tile * p.num_kt;
-      const int seg_end = min(u_end, tile_begin + p.num_kt);
-      const bool has_head = u == tile_begin;                    // this segment holds the tile's first stage
-      const bool has_tail = seg_end == tile_begin + p.num_kt;   // ... and its last stage
-      u = seg_end;
-      if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * GV_N, v);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      if (++acc == GV_ACC_BUFS) {
-        acc = 0;
-        acc_phase ^= 1;
-      }
-      const int col = quad * 32 + lane;                         // row of the weight tile
-      const int n = tile * BM + col;                            // output column
-      if (has_head && has_tail) {
-        if (n < p.N) {
-#pragma unroll
-          for (int m = 0; m < GV_N; ++m)
-            if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(__uint_as_float(v[m]) * alpha);
-        }
-        continue;
-      }
-      // my slot: 2*cta for the tail of a tile I start in the middle of, 2*cta+1
-      // for the head of a tile I leave unfinished
-      float* mine = p.partials + (static_cast<int64_t>(2 * cta + (has_head ? 1 : 0)) * p.M) * BM;
-      const float* other = p.partials + (static_cast<int64_t>(has_head ? 2 * (cta + 1) : 2 * (cta - 1) + 1) * p.M) * BM;
-#pragma unroll
-      for (int m = 0; m < GV_N; ++m)
-        if (m < p.M) mine[m * BM + col] = __uint_as_float(v[m]);
-      __threadfence();
-      __syncwarp();
-      int arrived = 0;
-      if (lane == 0) arrived = atomicAdd(&p.counters[tile * 4 + quad], 1);
-      arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
-      if (arrived == 1) {                                       // second of the two: finish
-        __threadfence();
-        if (n < p.N) {
-#pragma unroll
-          for (int m = 0; m < GV_N; ++m)
-            if (m < p.M) {
-              const float sum = __uint_as_float(v[m]) + __ldcg(other + m * BM + col);
-              p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
-            }
-        }
-      }
-    }
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
-  }
-}
-
-// Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
-// clearing of the fix-up counters, in one cluster of GP_CLUSTER CTAs.  CTA c
-// owns activation rows c, c+8, c+16, c+24 (those below M): it reduces the
-// amax of its rows, the cluster exchanges the partial maxima through
-// distributed shared memory, then each CTA quantizes its rows (two whole
-// 16-element blocks per thread at a time).  Only real rows are written: a
-// padding row r (M <= r < 32) of the activation operand only feeds output
-// column r of the MMA, which is never stored, so its contents do not matter.
-// It lets the dependent GEMV grid launch at once (programmatic dependent
-// launch): the GEMV streams weights while this runs and waits for it only
-// before it touches the activations, g_x or the partial sums.
-constexpr int GP_THREADS = 256;
-constexpr int GP_CLUSTER = 8;
-constexpr int GP_ROWS = GV_N / GP_CLUSTER;    // activation rows per CTA
-static_assert(GP_ROWS == 4, "row selection below assumes four rows per CTA");
-
-__device__ __forceinline__ void gp_load_block(const uint16_t* p, uint32_t (&w)[8]) {
-  const uint4 a = reinterpret_cast<const uint4*>(p)[0];
-  const uint4 b = reinterpret_cast<const uint4*>(p)[1];
-  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-  w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-}
-
-__global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
-                                                                   int64_t ldx, uint8_t* __restrict__ xq,
-                                                                   uint8_t* __restrict__ xsf, float* __restrict__ g_x,
-                                                                   int* __restrict__ counters, int n_counters,
-                                                                   int* __restrict__ status) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ float2 table[128];
-  __shared__ uint32_t red[GP_THREADS / 32];
-  __shared__ uint32_t partial;
-  __shared__ uint32_t cluster_max;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int c = static_cast<int>(cluster_ctarank());
-  const int kb = K >> 4;                     // 16-element blocks per row
-
-  // amax of this CTA's rows.  Rows of up to 2 * GP_THREADS blocks stay in
-  // registers (two blocks per thread) for the quantization below; longer
-  // rows are read again from L2.
-  const bool resident = kb <= 2 * GP_THREADS;
-  uint32_t wr[GP_ROWS][2][8];
-  uint32_t mx = 0;
-  if (resident) {
-#pragma unroll
-    for (int i = 0; i < GP_ROWS; ++i) {
-      const int r = c + i * GP_CLUSTER;
-      const uint16_t* row = x + static_cast<int64_t>(r) * ldx;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int b = tid + h * GP_THREADS;
-        if (r < M && b < kb) {
-          gp_load_block(row + b * 16, wr[i][h]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) wr[i][h][q] = 0u;
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < GP_ROWS; ++i) mx = max(mx, max(abs_max_bits16(wr[i][0]), abs_max_bits16(wr[i][1])));
-  } else {
-    for (int r = c; r < M; r += GP_CLUSTER) {
-      const uint16_t* row = x + static_cast<int64_t>(r) * ldx;
-      for (int b = tid; b < kb; b += GP_THREADS) {
-        uint32_t w[8];
-        gp_load_block(row + b * 16, w);
-        mx = max(mx, abs_max_bits16(w));
-      }
-    }
-  }
-  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-  if (lane == 0) red[tid >> 5] = mx;
-  fill_scale_table(table);
-  __syncthreads();
-  if (tid < 32) {
-    uint32_t t = lane < GP_THREADS / 32 ? red[lane] : 0u;
-    t = __reduce_max_sync(0xFFFFFFFFu, t);
-    if (tid == 0) partial = t;
-  }
-  __syncwarp();
-  // No global store precedes this barrier, so its release arrive does not wait
-  // on memory traffic: it only publishes `partial` to the cluster.
-  cluster_sync_all();
-  if (tid < 32) {
-    uint32_t all = tid < GP_CLUSTER ? ld_shared_cluster_u32(mapa_shared(smem_u32(&partial), tid)) : 0u;
-    all = __reduce_max_sync(0xFFFFFFFFu, all);
-    if (tid == 0) cluster_max = all;
-  }
-  __syncthreads();                           // cluster_max visible to the CTA
-  cluster_sync_relaxed();                    // peers' partials read: CTAs may leave from here on
-  for (int i = c * GP_THREADS + tid; i < n_counters; i += GP_CLUSTER * GP_THREADS) counters[i] = 0;
-  bool valid;
-  float g = global_scale_from_amax(__uint_as_float(cluster_max << 16), valid);
-  if (c == 0 && tid == 0) {
-    *g_x = valid ? g : 0.0f;
-    if (!valid) record_status(status, kDevRange);
-  }
-  if (!valid) g = 0.0f;                      // all-zero codes and scales
-
-  // quantize this CTA's rows.  Scale of (row r < 32, block b) in the padded
-  // 128-row scale layout: byte (b / 4) * 512 + r * 16 + b % 4; the other 12
-  // bytes of that 16-B chunk belong to rows r + 32, r + 64, r + 96 (absent
-  // from the N = 32 operand) and are written as zeros.
-  for (int i = 0; i < GP_ROWS; ++i) {
-    const int r = c + i * GP_CLUSTER;
-    if (r >= M) break;
-    const uint16_t* row = x + static_cast<int64_t>(r) * ldx;
-    uint8_t* qrow = xq + static_cast<int64_t>(r) * (K >> 1);
-    for (int b0 = tid; b0 < kb; b0 += 2 * GP_THREADS) {
-      const int b1 = b0 + GP_THREADS;
-      uint32_t w0[8], w1[8];
-      if (resident) {
-        // wr[i] held by a run-time row index: select through a switch so the
-        // array stays in registers
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          w0[q] = i == 0 ? wr[0][0][q] : i == 1 ? wr[1][0][q] : i == 2 ? wr[2][0][q] : wr[3][0][q];
-          w1[q] = i == 0 ? wr[0][1][q] : i == 1 ? wr[1][1][q] : i == 2 ? wr[2][1][q] : wr[3][1][q];
-        }
-      } else {
-        gp_load_block(row + b0 * 16, w0);
-        if (b1 < kb) {
-          gp_load_block(row + b1 * 16, w1);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) w1[q] = 0u;
-        }
-      }
-      if (!valid) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          w0[q] = 0u;
-          w1[q] = 0u;
-        }
-      }
-      uint2 c0, c1;
-      uint32_t s0, s1;
-      quantize_two_blocks(w0, w1, g, table, c0, c1, s0, s1);
-      *reinterpret_cast<uint2*>(qrow + b0 * 8) = c0;
-      uint8_t* chunk0 = xsf + (b0 >> 2) * 512 + r * 16;
-      chunk0[b0 & 3] = static_cast<uint8_t>(s0);
-      if ((b0 & 3) == 0) {
-        uint32_t* z = reinterpret_cast<uint32_t*>(chunk0);
-        z[1] = 0u; z[2] = 0u; z[3] = 0u;
-      }
-      if (b1 < kb) {
-        *reinterpret_cast<uint2*>(qrow + b1 * 8) = c1;
-        uint8_t* chunk1 = xsf + (b1 >> 2) * 512 + r * 16;
-        chunk1[b1 & 3] = static_cast<uint8_t>(s1);
-        if ((b1 & 3) == 0) {
-          uint32_t* z = reinterpret_cast<uint32_t*>(chunk1);
-          z[1] = 0u; z[2] = 0u; z[3] = 0u;
-        }
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// [rows, k] E2M1 codes (k/2 bytes per row) as a 2-D uint8 tensor, boxes of
-// 128 B x box_rows, 128-B swizzle (the tcgen05 K-major SW128 operand layout).
-bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // Tensor-core scale array of a [rows, k] operand as a 3-D uint32 tensor
 // (128 words per 512-B atom, k/64 atoms per 128-row group, row groups);
 // a box of 4 atoms x `groups` row groups = one K stage of 256.
@@ -1253,103 +778,6 @@ nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a
   if (N <= 128) return run_gemm<128>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
   if (M <= 128) return run_gemm<256>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
   return run_gemm_pair(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
-}
-
-// Workspace of the GEMV: [32, K/2] activation codes | [128, K/16] activation
-// scales | g_x (16 B) | fp32 partial slots [2 * GV_MAX_CTAS][M][128] |
-// counters [tiles * 4].
-constexpr int GV_MAX_CTAS = 160;
-
-struct GemvWs {
-  size_t xq, xsf, gx, part, cnt, total;
-};
-
-static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
-  GemvWs w;
-  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
-  w.xq = 0;
-  w.xsf = al(w.xq + static_cast<size_t>(GV_N) * K / 2);
-  w.gx = al(w.xsf + static_cast<size_t>(128) * K / 16);
-  w.part = al(w.gx + 16);
-  w.cnt = al(w.part + static_cast<size_t>(2 * GV_MAX_CTAS) * M * BM * 4);
-  w.total = al(w.cnt + static_cast<size_t>((N + BM - 1) / BM) * 4 * 4);
-  return w;
-}
-
-size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) { return gemv_ws_layout(M, N, K).total; }
-
-nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
-                         const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s) {
-  const GemvWs L = gemv_ws_layout(M, N, K);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  uint8_t* xq = base + L.xq;
-  uint8_t* xsf = base + L.xsf;
-  float* gx = reinterpret_cast<float*>(base + L.gx);
-  float* partials = reinterpret_cast<float*>(base + L.part);
-  int* cnt = reinterpret_cast<int*>(base + L.cnt);
-  const int tiles = static_cast<int>((N + BM - 1) / BM);
-  const int sms = device_sm_count();
-  const int64_t num_kt = (K + BK - 1) / BK;
-  if (static_cast<int64_t>(tiles) * num_kt > (int64_t{1} << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-
-  int* status = device_status_ptr();
-  if (!status) return NVFP4_ERR_CUDA;
-  {
-    cudaLaunchConfig_t pcfg = {};
-    cudaLaunchAttribute pattr[1];
-    pattr[0].id = cudaLaunchAttributeClusterDimension;
-    pattr[0].val.clusterDim.x = GP_CLUSTER;
-    pattr[0].val.clusterDim.y = 1;
-    pattr[0].val.clusterDim.z = 1;
-    pcfg.gridDim = dim3(GP_CLUSTER);
-    pcfg.blockDim = dim3(GP_THREADS);
-    pcfg.stream = s;
-    pcfg.attrs = pattr;
-    pcfg.numAttrs = 1;
-    const cudaError_t pe = cudaLaunchKernelEx(&pcfg, gemv_prologue_kernel, static_cast<const uint16_t*>(x),
-                                              static_cast<int>(M), static_cast<int>(K), ldx, xq, xsf, gx, cnt,
-                                              tiles * 4, status);
-    if (pe != cudaSuccess) return launch_status(pe);
-  }
-
-  CUtensorMap tmW, tmX;
-  if (!make_code_map(&tmW, w_codes, N, K, BM) || !make_code_map(&tmX, xq, GV_N, K, GV_N)) return NVFP4_ERR_CUDA;
-  GemvParams p;
-  p.wsf = static_cast<const uint8_t*>(w_sf);
-  p.xsf = xsf;
-  p.g_w = g_w;
-  p.g_x = gx;
-  p.partials = partials;
-  p.counters = cnt;
-  p.y = static_cast<__nv_bfloat16*>(y);
-  p.ldy = ldy;
-  p.M = static_cast<int>(M);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
-  p.kb4 = static_cast<int>(K / 64);
-  p.tiles = tiles;
-  p.num_kt = static_cast<int>((K + BK - 1) / BK);
-  p.wait_limit_ns = wait_limit_ns();
-  p.status = device_status_ptr();
-  if (!p.status) return NVFP4_ERR_CUDA;
-  // grid <= tiles: every CTA's stream-K range spans at least one tile's worth
-  // of stages, so each tile has at most two contributors
-  int grid = tiles < sms ? tiles : sms;
-  if (grid > GV_MAX_CTAS) grid = GV_MAX_CTAS;
-  cudaError_t e = cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_BYTES);
-  if (e != cudaSuccess) return launch_status(e);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(GV_THREADS);
-  cfg.dynamicSmemBytes = GV_SMEM_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemv_kernel, tmW, tmX, p);
-  return launch_status(e);
 }
 
 }  // namespace nvfp4
