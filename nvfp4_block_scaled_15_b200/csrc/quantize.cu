@@ -30,6 +30,8 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // Pass 1: max |x|.  grid.x strides over rows, grid.y over row segments.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                         int64_t ldx, unsigned* __restrict__ amax_bits) {
+  // the quantize pass (a programmatic dependent) may take SMs as these CTAs leave
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int chunks = k >> 3;
   const int c0 = blockIdx.y * kSegChunks + threadIdx.x;
   uint32_t m = 0;
@@ -91,6 +93,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
 
+  // Launched as a programmatic dependent of the amax pass: everything before
+  // this point overlaps its tail; the amax (and x) are read only after it.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
   float g = global_scale_from_amax(*amax_in, valid);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
@@ -169,6 +174,21 @@ __global__ void swizzle_kernel(const uint8_t* __restrict__ src, int rows, int kb
   }
 }
 
+template <bool kTc, bool kWide>
+cudaError_t launch_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
+                                uint8_t* codes, uint8_t* sf, float* g_dev, const float* amax_dev, int* status) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_kernel<kTc, kWide>, x, rows, k, ldx, codes, sf, g_dev, amax_dev, status);
+}
+
 }  // namespace
 
 nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s) {
@@ -192,26 +212,20 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx
   uint8_t* ss = static_cast<uint8_t*>(sf);
   const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
   const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
-  if (grid_rows == 0 || segs == 0) {
-    // nothing to quantize: still publish g (from the given amax)
-    quantize_kernel<false, false><<<dim3(1, 1), kThreads, 0, s>>>(xs, 0, 0, ldx, cs, ss, g_dev, amax_dev, status);
-    return launch_status(cudaGetLastError());
-  }
+  const int ir = static_cast<int>(rows), ik = static_cast<int>(k);
+  if (grid_rows == 0 || segs == 0)   // nothing to quantize: still publish g (from the given amax)
+    return launch_status(launch_quantize_pdl<false, false>(dim3(1, 1), s, xs, 0, 0, ldx, cs, ss, g_dev, amax_dev,
+                                                           status));
   const dim3 grid(static_cast<unsigned>(grid_rows), segs);
   const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
-  const int ir = static_cast<int>(rows), ik = static_cast<int>(k);
-  if (layout == NVFP4_SF_TCGEN05) {
-    if (wide)
-      quantize_kernel<true, true><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
-    else
-      quantize_kernel<true, false><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
-  } else {
-    if (wide)
-      quantize_kernel<false, true><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
-    else
-      quantize_kernel<false, false><<<grid, kThreads, 0, s>>>(xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
-  }
-  return launch_status(cudaGetLastError());
+  cudaError_t e;
+  if (layout == NVFP4_SF_TCGEN05)
+    e = wide ? launch_quantize_pdl<true, true>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status)
+             : launch_quantize_pdl<true, false>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
+  else
+    e = wide ? launch_quantize_pdl<false, true>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status)
+             : launch_quantize_pdl<false, false>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
+  return launch_status(e);
 }
 
 nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst, cudaStream_t s) {
