@@ -130,6 +130,27 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t 
                             nvfp4_stream_t stream);
 
 /*
+ * MXFP4, the format the pages set against NVFP4 ("mxFP4/nvFP4 最小化知识",
+ * (一) mxFP4的技术局限; "low-precision-floats", FP4 / MXFP4 / NVFP4): one E8M0
+ * (power-of-two) scale per 32 consecutive elements along K and no global
+ * scale.  With A the block max |x|:
+ *     k  = ceil(log2(A / 6))   (A / 6 an fp32 RN divide; rounded up, as the page
+ *                               says TensorRT does; clamped to [-127, 127];
+ *                               A == 0 gives -127)
+ *     scale byte = k + 127     (torch.float8_e8m0fnu)
+ *     q  = e2m1_rne_sat(x * 2^-k)   (|x * 2^-k| <= 6)
+ * One pass over x.  codes: out, [rows, k/2] bytes (16-byte aligned); sf: out,
+ * nvfp4_mxfp4_sf_bytes(rows, k, layout) bytes.  k % 32 == 0 for
+ * NVFP4_SF_ROWMAJOR, k % 128 == 0 for NVFP4_SF_TCGEN05 (atoms of 128 rows x 4
+ * scales, laid out as in nvfp4_sf_bytes, each scale covering 32 elements).
+ * A block holding a non-finite value gets scale byte 0xFF and zero codes, and
+ * the device status records NVFP4_ERR_RANGE.
+ */
+NVFP4_API size_t nvfp4_mxfp4_sf_bytes(int64_t rows, int64_t k, nvfp4_sf_layout layout);
+NVFP4_API nvfp4_status nvfp4_mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, void* codes,
+                                  void* sf, nvfp4_sf_layout layout, nvfp4_stream_t stream);
+
+/*
  * Re-layout of row-major block scales [rows, k/16] into the TCGEN05 layout
  * (see nvfp4_sf_bytes), padding written as 0.  k % 64 == 0.  Pure byte
  * permutation; the pages are silent on the tensor core's scale layout.

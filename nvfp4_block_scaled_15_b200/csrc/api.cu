@@ -170,6 +170,26 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
   return launch_quantize(x_bf16, rows, k, ldx, codes, sf, layout, g_dev, amax_dev, s);
 }
 
+size_t nvfp4_mxfp4_sf_bytes(int64_t rows, int64_t k, nvfp4_sf_layout layout) {
+  if (rows < 0 || k < 0 || (k % 32) != 0) return 0;
+  const int64_t kbm = k / 32;
+  if (layout == NVFP4_SF_ROWMAJOR) return static_cast<size_t>(rows * kbm);
+  if (layout == NVFP4_SF_TCGEN05) return static_cast<size_t>(round_up(rows, 128) * round_up(kbm, 4));
+  return 0;
+}
+
+nvfp4_status nvfp4_mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                                  nvfp4_sf_layout layout, nvfp4_stream_t stream) {
+  nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
+  if (st != NVFP4_OK) return st;
+  if (!codes || !sf) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
+  if ((k % 32) != 0 || (layout == NVFP4_SF_TCGEN05 && (k % 128) != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes)) return NVFP4_ERR_MISALIGNED;
+  if ((st = check_arch()) != NVFP4_OK) return st;
+  return launch_mx_quantize(x_bf16, rows, k, ldx, codes, sf, layout, reinterpret_cast<cudaStream_t>(stream));
+}
+
 nvfp4_status nvfp4_swizzle_sf(const void* sf_rowmajor, int64_t rows, int64_t k, void* sf_tcgen05,
                               nvfp4_stream_t stream) {
   if (!sf_rowmajor || !sf_tcgen05 || rows < 0 || k < 0) return NVFP4_ERR_INVALID_ARG;

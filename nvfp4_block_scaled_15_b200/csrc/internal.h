@@ -33,6 +33,8 @@ nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, fl
 nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
                              nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, cudaStream_t s);
 nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst, cudaStream_t s);
+nvfp4_status launch_mx_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                                nvfp4_sf_layout layout, cudaStream_t s);
 nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                          const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                          int64_t ldd, nvfp4_out_dtype out, cudaStream_t s);

@@ -156,6 +156,94 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   }
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4 ("low-precision-floats", FP4 / MXFP4 / NVFP4; "mxFP4/nvFP4 最小化知识"
+// (一)): one E8M0 scale per 32 elements, s = 2^ceil(log2(A/6)) for the block
+// max |x| = A, codes e2m1_rne_sat(x * 2^-k), no global scale, so one pass.
+// One thread per 32-element block: blockIdx.x = row, blockIdx.y = segment of
+// kThreads blocks.
+// ---------------------------------------------------------------------------
+// k = ceil(log2 v) for v = RN(A/6) >= 0 (v == 0 gives -127), clamped to the
+// E8M0 range, from the bits of v (normal or subnormal).
+__device__ __forceinline__ int mx_exponent(float v) {
+  const uint32_t bits = __float_as_uint(v);
+  const uint32_t e = bits >> 23;             // v >= 0: no sign bit
+  const uint32_t mant = bits & 0x7FFFFFu;
+  int k;
+  if (bits == 0u) {
+    k = -127;
+  } else if (e == 0u) {                      // subnormal: v = mant * 2^-149
+    const int fl = (31 - __clz(static_cast<int>(mant))) - 149;
+    k = fl + (__popc(mant) == 1 ? 0 : 1);
+  } else {
+    k = static_cast<int>(e) - 127 + (mant != 0u ? 1 : 0);
+  }
+  return max(-127, min(127, k));
+}
+
+template <bool kTcLayout>
+__global__ void __launch_bounds__(kThreads) mx_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k,
+                                                               int64_t ldx, uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ sf, int* __restrict__ status) {
+  const int r = blockIdx.x;
+  const int kbm = k >> 5;                    // 32-element blocks per row
+  const int b = blockIdx.y * kThreads + static_cast<int>(threadIdx.x);
+  const bool real_row = r < rows;
+  const bool in_row = b < kbm;
+  uint32_t w[16];
+  if (real_row && in_row) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx + b * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = ld_stream(src + q);
+      w[4 * q + 0] = v.x;
+      w[4 * q + 1] = v.y;
+      w[4 * q + 2] = v.z;
+      w[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) w[q] = 0u;
+  }
+  uint32_t lo[8], hi[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    lo[q] = w[q];
+    hi[q] = w[8 + q];
+  }
+  const uint32_t amax_bits = max(abs_max_bits16(lo), abs_max_bits16(hi));
+  const float a = __uint_as_float(amax_bits << 16);
+  uint32_t scale_byte;
+  uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+  if (!isfinite(a)) {
+    scale_byte = 0xFFu;                      // E8M0 NaN; codes stay 0
+    record_status(status, kDevRange);
+  } else {
+    const float v = div_rn_by_recip(a, 6.0f, __frcp_rn(6.0f));   // RN(A / 6)
+    const int e = mx_exponent(v);
+    scale_byte = static_cast<uint32_t>(e + 127);
+    const float inv = e <= 126 ? __uint_as_float(static_cast<uint32_t>(127 - e) << 23)
+                               : __uint_as_float(0x00400000u);   // 2^-127, subnormal
+    const float2 inv2 = make_float2(inv, inv);
+    float2 u[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) u[q] = __fmul2_rn(make_float2(bf16_lo(w[q]), bf16_hi(w[q])), inv2);
+    packed.x = e2m1x8(u[0], u[1], u[2], u[3]);
+    packed.y = e2m1x8(u[4], u[5], u[6], u[7]);
+    packed.z = e2m1x8(u[8], u[9], u[10], u[11]);
+    packed.w = e2m1x8(u[12], u[13], u[14], u[15]);
+  }
+  if (real_row && in_row)
+    *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(r) * (k >> 1) + b * 16) = packed;
+  if (!kTcLayout) {
+    if (real_row && in_row) sf[static_cast<int64_t>(r) * kbm + b] = static_cast<uint8_t>(scale_byte);
+  } else if (in_row) {
+    // byte of (row r, block b) = row_base + (b / 4) * 512 + b % 4 (rows past `rows` get 0)
+    const int64_t row_base = (static_cast<int64_t>(r >> 7) * (kbm >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+    sf[row_base + ((b >> 2) << 9) + (b & 3)] = static_cast<uint8_t>(real_row ? scale_byte : 0u);
+  }
+}
+
 // Row-major [rows, kb] scales -> tensor-core atoms; one thread per output
 // 32-bit word (one row's 4 blocks of one atom).
 __global__ void swizzle_kernel(const uint8_t* __restrict__ src, int rows, int kb, int64_t words,
@@ -226,6 +314,24 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx
     e = wide ? launch_quantize_pdl<false, true>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status)
              : launch_quantize_pdl<false, false>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, status);
   return launch_status(e);
+}
+
+nvfp4_status launch_mx_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                                nvfp4_sf_layout layout, cudaStream_t s) {
+  int* status = device_status_ptr();
+  if (!status) return NVFP4_ERR_CUDA;
+  const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
+  const int segs = static_cast<int>((k / 32 + kThreads - 1) / kThreads);
+  if (grid_rows == 0 || segs == 0) return NVFP4_OK;
+  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  if (layout == NVFP4_SF_TCGEN05)
+    mx_quantize_kernel<true><<<grid, kThreads, 0, s>>>(xs, static_cast<int>(rows), static_cast<int>(k), ldx,
+                                                       static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), status);
+  else
+    mx_quantize_kernel<false><<<grid, kThreads, 0, s>>>(xs, static_cast<int>(rows), static_cast<int>(k), ldx,
+                                                        static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), status);
+  return launch_status(cudaGetLastError());
 }
 
 nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst, cudaStream_t s) {

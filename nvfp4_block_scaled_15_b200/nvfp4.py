@@ -51,6 +51,8 @@ _SIGS = {
     "nvfp4_gemv_batched": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _sz, _vp], _i32),
     "nvfp4_gemm_quant_a": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp], _i32),
     "nvfp4_gemv_batched_noalloc": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp], _i32),
+    "nvfp4_mxfp4_sf_bytes": ([_i64, _i64, _i32], _sz),
+    "nvfp4_mxfp4_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "nvfp4_check_device_status": ([_vp], _i32),
     "nvfp4_set_wait_limit_ns": ([_u64], None),
     "nvfp4_selftest_wait_timeout": ([_u64, _vp], _i32),
@@ -145,6 +147,15 @@ def nvfp4_gemm_quant_a(a, lda, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, w
                                    _p(workspace), ws_bytes, _s(stream)), "nvfp4_gemm_quant_a")
 
 
+def nvfp4_mxfp4_sf_bytes(rows: int, k: int, layout: int) -> int:
+    return _lib.nvfp4_mxfp4_sf_bytes(rows, k, layout)
+
+
+def nvfp4_mxfp4_quantize(x, rows, k, ldx, codes, sf, layout, stream=None) -> None:
+    _check(_lib.nvfp4_mxfp4_quantize(_p(x), rows, k, ldx, _p(codes), _p(sf), layout, _s(stream)),
+           "nvfp4_mxfp4_quantize")
+
+
 def nvfp4_check_device_status(stream=None) -> int:
     """Synchronises the stream; returns (and clears) the device status code."""
     return _lib.nvfp4_check_device_status(_s(stream))
@@ -226,3 +237,24 @@ def gemm_quant_a(a: torch.Tensor, b: Quantized, out_dtype=torch.bfloat16, out=No
     d = out if out is not None else torch.empty((m, n), dtype=out_dtype, device=a.device)
     nvfp4_gemm_quant_a(a, a.stride(0), b.codes, b.sf, b.g, m, n, k, d, d.stride(0), od, ws, ws.numel(), stream)
     return d
+
+
+class MXQuantized:
+    """MXFP4 tensor: codes [rows, k/2] uint8 and E8M0 scales (layout bytes); no global scale."""
+
+    def __init__(self, codes, sf, rows, k, layout):
+        self.codes, self.sf = codes, sf
+        self.rows, self.k, self.layout = rows, k, layout
+
+
+def mxfp4_quantize(x: torch.Tensor, layout: int = SF_TCGEN05, out: MXQuantized | None = None,
+                   stream=None) -> MXQuantized:
+    """bf16 [rows, k] (row pitch x.stride(0)) -> MXFP4 (one pass)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    if out is None:
+        codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=x.device)
+        sf = torch.empty(max(1, nvfp4_mxfp4_sf_bytes(rows, k, layout)), dtype=torch.uint8, device=x.device)
+        out = MXQuantized(codes, sf, rows, k, layout)
+    nvfp4_mxfp4_quantize(x, rows, k, x.stride(0), out.codes, out.sf, layout, stream)
+    return out

@@ -42,8 +42,13 @@ def test_gemv_tiles_split_between_ctas(lib, m):
 
 
 def test_gemv_repeated_calls_reuse_workspace(lib):
-    """The workspace is re-initialised by every call: two calls, same answer."""
-    m, n, k = 8, 640, 512
+    """The workspace is re-initialised by every call: two calls, same answer
+    (one shape with whole tiles per CTA, one with split tiles)."""
+    for m, n, k in [(8, 640, 512), (8, 2048, 512)]:
+        _repeated_calls(lib, m, n, k)
+
+
+def _repeated_calls(lib, m, n, k):
     x = inputs.gaussian_bf16((m, k), seed=501)
     w = inputs.gaussian_bf16((n, k), seed=502, std=0.02)
     qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
@@ -56,6 +61,22 @@ def test_gemv_repeated_calls_reuse_workspace(lib):
     d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, pw, sw, gw)
     check_bf16(host_bf16_bits(y1), d_ref, s_ref, alpha)
     check_bf16(host_bf16_bits(y2), d_ref, s_ref, alpha)
+
+
+@pytest.mark.parametrize("m,n,k", [(5, 1100, 960), (16, 1024, 8192), (1, 8192 + 40, 4160), (12, 4096, 64)],
+                         ids=lambda v: str(v))
+def test_gemv_more_shapes(lib, m, n, k):
+    """A partial last K stage (K % 256 != 0), ragged N, K = 64 (one MMA-K
+    step per tile), N = 1024 with K = 8192 (every CTA one whole tile)."""
+    x = inputs.activations_with_outliers(m, k, seed=950 + m, fraction=0.01, factor=30.0)
+    w = inputs.gaussian_bf16((n, k), seed=951 + n, std=0.02)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    y = lib.gemv_batched(dev_bf16(x), qw)
+    assert lib.nvfp4_check_device_status() == lib.OK
+    px, sx, gx, _ = O.quantize(x)
+    pw, sw, gw, _ = O.quantize(w)
+    d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, pw, sw, gw)
+    check_bf16(host_bf16_bits(y), d_ref, s_ref, alpha)
 
 
 @pytest.mark.parametrize("m", [1, 8, 16])
