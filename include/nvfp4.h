@@ -151,6 +151,18 @@ NVFP4_API nvfp4_status nvfp4_mxfp4_quantize(const void* x_bf16, int64_t rows, in
                                   void* sf, nvfp4_sf_layout layout, nvfp4_stream_t stream);
 
 /*
+ * MXFP4 block-scaled GEMM on tcgen05.mma kind::mxf4 (.scale_vec::2X, E8M0
+ * scales): D[m, n] = sum_k (s_a a)[m,k] (s_b b)[n,k], no global scales.
+ *   a_codes [M, K/2], a_sf_tc: TCGEN05 MXFP4 scales of A (nvfp4_mxfp4_quantize)
+ *   b_codes [N, K/2], b_sf_tc: the same for B
+ *   d: out, [M, N], pitch ldd >= N, bf16 or fp32 per out_dtype (as nvfp4_gemm).
+ * K % 128 == 0 (whole scale atoms), M, N >= 1.
+ */
+NVFP4_API nvfp4_status nvfp4_mxfp4_gemm(const void* a_codes, const void* a_sf_tc, const void* b_codes,
+                              const void* b_sf_tc, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                              nvfp4_out_dtype out_dtype, nvfp4_stream_t stream);
+
+/*
  * Re-layout of row-major block scales [rows, k/16] into the TCGEN05 layout
  * (see nvfp4_sf_bytes), padding written as 0.  k % 64 == 0.  Pure byte
  * permutation; the pages are silent on the tensor core's scale layout.

@@ -212,6 +212,23 @@ static nvfp4_status check_gemm_operands(const void* a_codes, const void* a_sf, c
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_mxfp4_gemm(const void* a_codes, const void* a_sf_tc, const void* b_codes, const void* b_sf_tc,
+                              int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out_dtype,
+                              nvfp4_stream_t stream) {
+  if (!a_codes || !a_sf_tc || !b_codes || !b_sf_tc || !d) return NVFP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1) return NVFP4_ERR_INVALID_ARG;
+  if ((K % 128) != 0 || M > 0x7FFFFF80 || N > 0x7FFFFF80 || K > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_sf_tc) || !aligned16(b_sf_tc))
+    return NVFP4_ERR_MISALIGNED;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+  if (ldd < N) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d) & (out_dtype == NVFP4_OUT_F32 ? 3u : 1u)) != 0) return NVFP4_ERR_MISALIGNED;
+  nvfp4_status st = check_arch();
+  if (st != NVFP4_OK) return st;
+  return launch_mx_gemm(a_codes, a_sf_tc, b_codes, b_sf_tc, M, N, K, d, ldd, out_dtype,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
 nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_sf_tc, const float* g_a_dev, const void* b_codes,
                         const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d,
                         int64_t ldd, nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {

@@ -59,18 +59,19 @@ namespace {
 // ---------------------------------------------------------------------------
 // GEMM configuration
 // ---------------------------------------------------------------------------
-template <int BN_>
+template <int BN_, bool kMx>
 struct GemmCfg {
+  using F = ScaleFmt<kMx>;
   static constexpr int BN = BN_;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
   static constexpr int A_BYTES = BM * BK_BYTES;
   static constexpr int B_BYTES = BN * BK_BYTES;
-  static constexpr int SFA_BYTES = 4 * SF_ATOM;
-  static constexpr int SFB_BYTES = (BN / 128) * 4 * SF_ATOM;
+  static constexpr int SFA_BYTES = F::ATOMS_PER_STAGE * SF_ATOM;
+  static constexpr int SFB_BYTES = (BN / 128) * F::ATOMS_PER_STAGE * SF_ATOM;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int ACC_BUFS = (BN == 256) ? 1 : 2;
-  static constexpr int SFB_COLS_PER_K = BN / 32;                       // TMEM columns of B scales per MMA
-  static constexpr int SF_COLS_PER_STAGE = 4 * 4 + 4 * SFB_COLS_PER_K;
+  static constexpr int SFB_COLS_PER_K = BN / 32;                       // TMEM columns of B scales per atom
+  static constexpr int SF_COLS_PER_STAGE = F::ATOMS_PER_STAGE * (4 + SFB_COLS_PER_K);
   static constexpr int TMEM_SF_BASE = ACC_BUFS * BN;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
@@ -138,11 +139,12 @@ __device__ __forceinline__ void store_row(const GemmParams& p, int row, int col0
   }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
+template <int BN, bool kMx>
+__global__ void __launch_bounds__(GemmCfg<BN, kMx>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, kMx>;
+  using F = typename C::F;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -201,7 +203,8 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
         for (int kt = 0; kt < num_kt; ++kt) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
           const int nk = min(4, ksteps_total - kt * 4);
-          const uint32_t bytes = C::A_BYTES + C::B_BYTES + nk * SF_ATOM * (1 + n_groups);
+          const int na = F::atoms_of(nk);
+          const uint32_t bytes = C::A_BYTES + C::B_BYTES + na * SF_ATOM * (1 + n_groups);
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
           uint8_t* sSFA = sB + C::B_BYTES;
@@ -209,10 +212,11 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_2d(sA, &tmA, &full[stage], kt * BK_BYTES, m0);
           tma_load_2d(sB, &tmB, &full[stage], kt * BK_BYTES, n0);
-          bulk_load(sSFA, p.sfa + (static_cast<int64_t>(tm) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM, &full[stage]);
+          const int atom0 = kt * F::ATOMS_PER_STAGE;
+          bulk_load(sSFA, p.sfa + (static_cast<int64_t>(tm) * p.kb4 + atom0) * SF_ATOM, na * SF_ATOM, &full[stage]);
           for (int g = 0; g < n_groups; ++g)
-            bulk_load(sSFB + g * 4 * SF_ATOM,
-                      p.sfb + (static_cast<int64_t>(n0 / 128 + g) * p.kb4 + kt * 4) * SF_ATOM, nk * SF_ATOM,
+            bulk_load(sSFB + g * F::ATOMS_PER_STAGE * SF_ATOM,
+                      p.sfb + (static_cast<int64_t>(n0 / 128 + g) * p.kb4 + atom0) * SF_ATOM, na * SF_ATOM,
                       &full[stage]);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -241,6 +245,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
         const int n0 = tn * BN;
         const int n_mma = min(BN, round_up_int(p.N - n0, 128));
         const uint32_t idesc = idesc_mxf4nvf4(BM, n_mma);
+        const uint32_t idesc_mx0 = idesc_mxf4(BM, n_mma, 0), idesc_mx1 = idesc_mxf4(BM, n_mma, 2);
         if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -257,15 +262,22 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
           const uint32_t sSFA = sB + C::B_BYTES;
           const uint32_t sSFB = sSFA + C::SFA_BYTES;
           const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE + stage * C::SF_COLS_PER_STAGE;
-          const uint32_t tsfb = tsfa + 16;
-          for (int j = 0; j < nk; ++j) {
-            tc_cp_32x128b_warpx4(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
+          const uint32_t tsfb = tsfa + 4 * F::ATOMS_PER_STAGE;
+          const int na = F::atoms_of(nk);
+          for (int a = 0; a < na; ++a) {
+            tc_cp_32x128b_warpx4(tsfa + a * 4, sf_desc(sSFA + a * SF_ATOM));
             for (int g = 0; g < n_mma / 128; ++g)
-              tc_cp_32x128b_warpx4(tsfb + j * C::SFB_COLS_PER_K + g * 4, sf_desc(sSFB + g * 4 * SF_ATOM + j * SF_ATOM));
+              tc_cp_32x128b_warpx4(tsfb + a * C::SFB_COLS_PER_K + g * 4,
+                                   sf_desc(sSFB + g * F::ATOMS_PER_STAGE * SF_ATOM + a * SF_ATOM));
           }
           for (int j = 0; j < nk; ++j) {
-            mma_mxf4nvf4(d_tmem, code_desc(sA + j * (MMA_K / 2)), code_desc(sB + j * (MMA_K / 2)), idesc,
-                         tsfa + j * 4, tsfb + j * C::SFB_COLS_PER_K, (kt | j) != 0);
+            const uint64_t ad = code_desc(sA + j * (MMA_K / 2)), bd = code_desc(sB + j * (MMA_K / 2));
+            const int a = F::atom_of_step(j);
+            if (kMx)
+              mma_mxf4(d_tmem, ad, bd, (j & 1) ? idesc_mx1 : idesc_mx0, tsfa + a * 4, tsfb + a * C::SFB_COLS_PER_K,
+                       (kt | j) != 0);
+            else
+              mma_mxf4nvf4(d_tmem, ad, bd, idesc, tsfa + a * 4, tsfb + a * C::SFB_COLS_PER_K, (kt | j) != 0);
           }
           tc_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -291,7 +303,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
     const int half = ew >> 2;                  // which half of the tile's columns
     constexpr int HALF = BN / 2;
-    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    const float alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -335,13 +347,15 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // the scale copies and MMAs for both; both CTAs' loads complete on the
 // leader's "full" barriers, and its commits arrive on both CTAs' barriers.
 // ---------------------------------------------------------------------------
+template <bool kMx>
 struct PairCfg {
+  using F = ScaleFmt<kMx>;
   static constexpr int BN = 256;                       // N per tile (both CTAs)
   static constexpr int STAGES = 5;
   static constexpr int A_BYTES = BM * BK_BYTES;        // this CTA's 128 rows of A
   static constexpr int B_BYTES = 128 * BK_BYTES;       // this CTA's half of B
-  static constexpr int SFA_BYTES = 4 * SF_ATOM;
-  static constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;    // scales of all 256 B rows
+  static constexpr int SFA_BYTES = F::ATOMS_PER_STAGE * SF_ATOM;
+  static constexpr int SFB_BYTES = 2 * F::ATOMS_PER_STAGE * SF_ATOM;    // scales of all 256 B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   // Two accumulators that share OVL columns: acc0 = [0, 256), acc1 =
   // [256 - OVL, 512 - OVL).  The epilogue drains the shared columns first and
@@ -349,7 +363,7 @@ struct PairCfg {
   // previous accumulator is still being drained.  The last OVL columns hold
   // the scale factors of the current K stage (one region, refreshed per stage:
   // tcgen05.cp and tcgen05.mma issued by one thread execute in order).
-  static constexpr int SF_COLS = 4 * 4 + 4 * 8;        // one K stage: SFA 16 + SFB 32 columns
+  static constexpr int SF_COLS = F::ATOMS_PER_STAGE * (4 + 8);   // one K stage: SFA + SFB columns
   static constexpr int OVL = 64;
   static constexpr int ACC1_COL = BN - OVL;
   static constexpr int TMEM_SF_BASE = 2 * BN - OVL;
@@ -366,11 +380,13 @@ struct PairCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+template <bool kMx>
+__global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                      const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-  using C = PairCfg;
+  using C = PairCfg<kMx>;
+  using F = typename C::F;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* epi_smem = smem + C::STAGES * C::STAGE_BYTES;
@@ -448,8 +464,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           tma_load_2d_pair(sA, &tmA, bar, kt * BK_BYTES, m_cta);
           tma_load_2d_pair(sB, &tmB, bar, kt * BK_BYTES, n0 + static_cast<int>(rank) * 128);
-          tma_load_3d_pair(sSFA, &tmSFA, bar, 0, kt * 4, m_cta / 128);
-          tma_load_3d_pair(sSFB, &tmSFB, bar, 0, kt * 4, n0 / 128);
+          tma_load_3d_pair(sSFA, &tmSFA, bar, 0, kt * F::ATOMS_PER_STAGE, m_cta / 128);
+          tma_load_3d_pair(sSFB, &tmSFB, bar, 0, kt * F::ATOMS_PER_STAGE, n0 / 128);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) {
@@ -470,10 +486,12 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     // ------------------------- MMA issuer (leader) -------------------------
     if (leader && elect_one()) {
       const uint32_t idesc = idesc_mxf4nvf4(256, C::BN);
+      const uint32_t idesc_mx0 = idesc_mxf4(256, C::BN, 0), idesc_mx1 = idesc_mxf4(256, C::BN, 2);
       const uint32_t smem_base = smem_u32(smem);
       const bool full_last_stage = (ksteps_total & 3) == 0;   // every K stage holds 4 MMA-K steps
       const uint32_t tsfa = tmem_base + C::TMEM_SF_BASE;
-      const uint32_t tsfb = tsfa + 16;
+      const uint32_t tsfb = tsfa + 4 * F::ATOMS_PER_STAGE;
+      constexpr int FB_GROUP = F::ATOMS_PER_STAGE * SF_ATOM / 16;   // second B row group, in descriptor units
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_phase = 0;                 // bit b: phase parity of acc_empty[b]
@@ -506,25 +524,37 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           const uint64_t fb = sf_desc(sA + C::A_BYTES + C::B_BYTES + C::SFA_BYTES);
           if (kt + 1 < num_kt || full_last_stage) {
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              tc_cp_32x128b_warpx4_pair(tsfa + jj * 4, fa + 32 * jj);
-              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8, fb + 32 * jj);
-              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8 + 4, fb + 128 + 32 * jj);
+            for (int aa = 0; aa < F::ATOMS_PER_STAGE; ++aa) {
+              tc_cp_32x128b_warpx4_pair(tsfa + aa * 4, fa + 32 * aa);
+              tc_cp_32x128b_warpx4_pair(tsfb + aa * 8, fb + 32 * aa);
+              tc_cp_32x128b_warpx4_pair(tsfb + aa * 8 + 4, fb + FB_GROUP + 32 * aa);
             }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-              mma_mxf4nvf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, idesc, tsfa + jj * 4, tsfb + jj * 8,
-                                (kt | jj) != 0);
+            for (int jj = 0; jj < 4; ++jj) {
+              const int a = F::atom_of_step(jj);
+              if (kMx)
+                mma_mxf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, (jj & 1) ? idesc_mx1 : idesc_mx0, tsfa + a * 4,
+                              tsfb + a * 8, (kt | jj) != 0);
+              else
+                mma_mxf4nvf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, idesc, tsfa + a * 4, tsfb + a * 8,
+                                  (kt | jj) != 0);
+            }
           } else {
             const int nk = ksteps_total - kt * 4;
-            for (int jj = 0; jj < nk; ++jj) {
-              tc_cp_32x128b_warpx4_pair(tsfa + jj * 4, fa + 32 * jj);
-              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8, fb + 32 * jj);
-              tc_cp_32x128b_warpx4_pair(tsfb + jj * 8 + 4, fb + 128 + 32 * jj);
+            for (int aa = 0; aa < F::atoms_of(nk); ++aa) {
+              tc_cp_32x128b_warpx4_pair(tsfa + aa * 4, fa + 32 * aa);
+              tc_cp_32x128b_warpx4_pair(tsfb + aa * 8, fb + 32 * aa);
+              tc_cp_32x128b_warpx4_pair(tsfb + aa * 8 + 4, fb + FB_GROUP + 32 * aa);
             }
-            for (int jj = 0; jj < nk; ++jj)
-              mma_mxf4nvf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, idesc, tsfa + jj * 4, tsfb + jj * 8,
-                                (kt | jj) != 0);
+            for (int jj = 0; jj < nk; ++jj) {
+              const int a = F::atom_of_step(jj);
+              if (kMx)
+                mma_mxf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, (jj & 1) ? idesc_mx1 : idesc_mx0, tsfa + a * 4,
+                              tsfb + a * 8, (kt | jj) != 0);
+              else
+                mma_mxf4nvf4_pair(d_tmem, ad + 2 * jj, bd + 2 * jj, idesc, tsfa + a * 4, tsfb + a * 8,
+                                  (kt | jj) != 0);
+            }
           }
           tc_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == C::STAGES) {
@@ -545,7 +575,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     const int quad = warp & 3;
     const int half = ew >> 2;
     constexpr int HALF = C::BN / 2;
-    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    const float alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     const uint32_t ovl_free_leader = mapa_shared(smem_u32(ovl_free), 0);
     int j = 0;
@@ -638,16 +668,16 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 // Host side
 // ---------------------------------------------------------------------------
 // Tensor-core scale array of a [rows, k] operand as a 3-D uint32 tensor
-// (128 words per 512-B atom, k/64 atoms per 128-row group, row groups);
-// a box of 4 atoms x `groups` row groups = one K stage of 256.
-bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int groups) {
+// (128 words per 512-B atom, k / k_per_atom atoms per 128-row group, row
+// groups); a box of the atoms of one 256-wide K stage x `groups` row groups.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int groups, int k_per_atom) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const int64_t kb4 = k / 64;
+  const int64_t kba = k / k_per_atom;
   const int64_t rg = (rows + 127) / 128;
-  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(kb4), static_cast<cuuint64_t>(rg)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(SF_ATOM), static_cast<cuuint64_t>(kb4 * SF_ATOM)};
-  cuuint32_t box[3] = {128, 4, static_cast<cuuint32_t>(groups)};
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(kba), static_cast<cuuint64_t>(rg)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(SF_ATOM), static_cast<cuuint64_t>(kba * SF_ATOM)};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(BK / k_per_atom), static_cast<cuuint32_t>(groups)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -662,7 +692,7 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(PairCfg::EPI_BOX_COLS), 32};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(PairCfg<false>::EPI_BOX_COLS), 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -670,13 +700,15 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   return r == CUDA_SUCCESS;
 }
 
+template <bool kMx>
 nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                            const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
                            nvfp4_out_dtype out, cudaStream_t s) {
-  using C = PairCfg;
+  using C = PairCfg<kMx>;
+  using F = typename C::F;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
   if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, 128) ||
-      !make_sf_map(&tmSFA, a_sf, M, K, 1) || !make_sf_map(&tmSFB, b_sf, N, K, 2))
+      !make_sf_map(&tmSFA, a_sf, M, K, 1, F::K_PER_ATOM) || !make_sf_map(&tmSFB, b_sf, N, K, 2, F::K_PER_ATOM))
     return NVFP4_ERR_CUDA;
   // bf16 D whose base, row pitch and row end (N) fall on 16-B boundaries leaves
   // through TMA stores.  The store clips boxes at the tensor's edge in whole
@@ -695,7 +727,7 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.kb4 = static_cast<int>(K / 64);
+  p.kb4 = static_cast<int>(K / F::K_PER_ATOM);
   p.tiles_m = static_cast<int>((M + 255) / 256);
   p.tiles_n = static_cast<int>((N + C::BN - 1) / C::BN);
   p.out_f32 = out == NVFP4_OUT_F32;
@@ -705,7 +737,8 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;
-  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<kMx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
   if (e != cudaSuccess) return launch_status(e);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -725,22 +758,22 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   if (dev < 64 && max_pairs[dev] == 0) {
     cfg.gridDim = dim3(2 * (device_sm_count() / 2));
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<kMx>, &cfg);
     if (e != cudaSuccess || clusters < 1) return launch_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
     max_pairs[dev] = clusters;
   }
   const int tiles = p.tiles_m * p.tiles_n;
   const int pairs = tiles < max_pairs[dev < 64 ? dev : 0] ? tiles : max_pairs[dev < 64 ? dev : 0];
   cfg.gridDim = dim3(2 * pairs);
-  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tmA, tmB, tmSFA, tmSFB, tmD, p);
+  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kMx>, tmA, tmB, tmSFA, tmSFB, tmD, p);
   return launch_status(e);
 }
 
-template <int BN>
+template <int BN, bool kMx>
 nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                       const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
                       nvfp4_out_dtype out, cudaStream_t s) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, kMx>;
   CUtensorMap tmA, tmB;
   if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, BN)) return NVFP4_ERR_CUDA;
   GemmParams p{};
@@ -753,7 +786,7 @@ nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, c
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.kb4 = static_cast<int>(K / 64);
+  p.kb4 = static_cast<int>(K / C::F::K_PER_ATOM);
   p.tiles_m = static_cast<int>((M + BM - 1) / BM);
   p.tiles_n = static_cast<int>((N + BN - 1) / BN);
   p.out_f32 = out == NVFP4_OUT_F32;
@@ -764,20 +797,34 @@ nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, c
   if (!p.status) return NVFP4_ERR_CUDA;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, kMx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
   if (e != cudaSuccess) return launch_status(e);
-  gemm_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tmA, tmB, p);
+  gemm_kernel<BN, kMx><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tmA, tmB, p);
   return launch_status(cudaGetLastError());
 }
 
 }  // namespace
 
+template <bool kMx>
+nvfp4_status dispatch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                           const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                           nvfp4_out_dtype out, cudaStream_t s) {
+  if (N <= 128) return run_gemm<128, kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  if (M <= 128) return run_gemm<256, kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  return run_gemm_pair<kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+}
+
 nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                          const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                          int64_t ldd, nvfp4_out_dtype out, cudaStream_t s) {
-  if (N <= 128) return run_gemm<128>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
-  if (M <= 128) return run_gemm<256>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
-  return run_gemm_pair(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  return dispatch_gemm<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+}
+
+nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,
+                            int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out,
+                            cudaStream_t s) {
+  return dispatch_gemm<true>(a_codes, a_sf, nullptr, b_codes, b_sf, nullptr, M, N, K, d, ldd, out, s);
 }
 
 }  // namespace nvfp4

@@ -38,6 +38,9 @@ nvfp4_status launch_mx_quantize(const void* x, int64_t rows, int64_t k, int64_t 
 nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                          const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                          int64_t ldd, nvfp4_out_dtype out, cudaStream_t s);
+nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,
+                            int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out,
+                            cudaStream_t s);
 nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
                          const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s);
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K);

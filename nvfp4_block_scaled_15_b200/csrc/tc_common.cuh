@@ -20,6 +20,22 @@ constexpr int MMA_K = 64;        // K per tcgen05.mma for kind::mxf4nvf4
 constexpr int SF_ATOM = 512;     // bytes of one 128-row x 4-block scale atom
 constexpr uint32_t TMEM_COLS = 512;
 
+// Scale format of the block-scaled MMA (both kernels are templated on it).
+//   NVFP4: E4M3 scale per 16 elements; one 512-B atom (128 rows x 4 scales)
+//          per 64-wide MMA-K step; kind::mxf4nvf4 .scale_vec::4X.
+//   MXFP4: E8M0 scale per 32 elements; one atom per two MMA-K steps, step j
+//          using the scale pair at byte 2 (j % 2) of each TMEM cell;
+//          kind::mxf4 .scale_vec::2X; no global scales (alpha = 1).
+template <bool kMx>
+struct ScaleFmt {
+  static constexpr int K_PER_ATOM = kMx ? 128 : 64;
+  static constexpr int ATOMS_PER_STAGE = BK / K_PER_ATOM;
+  // atom holding MMA-K step j of a stage
+  __host__ __device__ static constexpr int atom_of_step(int j) { return kMx ? j >> 1 : j; }
+  // scale atoms of a stage with nk MMA-K steps
+  __host__ __device__ static constexpr int atoms_of(int nk) { return kMx ? (nk + 1) >> 1 : nk; }
+};
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }

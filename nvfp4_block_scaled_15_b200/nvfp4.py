@@ -53,6 +53,7 @@ _SIGS = {
     "nvfp4_gemv_batched_noalloc": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp], _i32),
     "nvfp4_mxfp4_sf_bytes": ([_i64, _i64, _i32], _sz),
     "nvfp4_mxfp4_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
+    "nvfp4_mxfp4_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp], _i32),
     "nvfp4_check_device_status": ([_vp], _i32),
     "nvfp4_set_wait_limit_ns": ([_u64], None),
     "nvfp4_selftest_wait_timeout": ([_u64, _vp], _i32),
@@ -154,6 +155,11 @@ def nvfp4_mxfp4_sf_bytes(rows: int, k: int, layout: int) -> int:
 def nvfp4_mxfp4_quantize(x, rows, k, ldx, codes, sf, layout, stream=None) -> None:
     _check(_lib.nvfp4_mxfp4_quantize(_p(x), rows, k, ldx, _p(codes), _p(sf), layout, _s(stream)),
            "nvfp4_mxfp4_quantize")
+
+
+def nvfp4_mxfp4_gemm(a_codes, a_sf, b_codes, b_sf, m, n, k, d, ldd, out_dtype=OUT_BF16, stream=None) -> None:
+    _check(_lib.nvfp4_mxfp4_gemm(_p(a_codes), _p(a_sf), _p(b_codes), _p(b_sf), m, n, k, _p(d), ldd, out_dtype,
+                                 _s(stream)), "nvfp4_mxfp4_gemm")
 
 
 def nvfp4_check_device_status(stream=None) -> int:
@@ -258,3 +264,13 @@ def mxfp4_quantize(x: torch.Tensor, layout: int = SF_TCGEN05, out: MXQuantized |
         out = MXQuantized(codes, sf, rows, k, layout)
     nvfp4_mxfp4_quantize(x, rows, k, x.stride(0), out.codes, out.sf, layout, stream)
     return out
+
+
+def mxfp4_gemm(a: MXQuantized, b: MXQuantized, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """D [M, N] = (s_a A)(s_b B)^T for two TCGEN05-layout MXFP4 operands."""
+    assert a.layout == SF_TCGEN05 and b.layout == SF_TCGEN05 and a.k == b.k
+    od = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    d = out if out is not None else torch.empty((a.rows, b.rows), dtype=out_dtype, device=a.codes.device)
+    nvfp4_mxfp4_gemm(a.codes, a.sf, b.codes, b.sf, a.rows, b.rows, a.k, d, d.stride(0), od, stream)
+    return d

@@ -11,7 +11,7 @@ import torch
 from oracle import mxfp4_oracle as MX
 from oracle import nvfp4_oracle as NV
 from nvfp4_block_scaled_15_b200 import inputs
-from parity import dev_bf16, host_u8
+from parity import check_bf16, check_f32, dev_bf16, host_bf16_bits, host_u8
 
 pytestmark = pytest.mark.gpu
 
@@ -78,3 +78,134 @@ def test_mx_quantize_nonfinite_block_reports_range(lib):
     mask = np.ones_like(sf, dtype=bool)
     mask[2, 1] = False
     assert np.array_equal(sf[mask], want[mask])
+
+
+# --------------------------------------------------------------------------
+# MXFP4 block-scaled GEMM (tcgen05.mma kind::mxf4, E8M0 scales, no alpha)
+# --------------------------------------------------------------------------
+
+def _mx_gemm_case(lib, a_bits, b_bits, out_dtype):
+    qa = lib.mxfp4_quantize(dev_bf16(a_bits), lib.SF_TCGEN05)
+    qb = lib.mxfp4_quantize(dev_bf16(b_bits), lib.SF_TCGEN05)
+    d = lib.mxfp4_gemm(qa, qb, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    pa, sa = MX.quantize_mx(a_bits)
+    pb, sb = MX.quantize_mx(b_bits)
+    assert np.array_equal(host_u8(qa.codes), pa) and np.array_equal(host_u8(qb.codes), pb)
+    d_ref, s_ref = MX.gemm_ref_mx(pa, sa, pb, sb)
+    return d, d_ref, s_ref
+
+
+MX_SHAPES = [
+    (1, 1, 128),          # one element, one scale atom
+    (200, 136, 384),      # M and N tails, a last K stage with one 128-wide atom
+    (129, 257, 512),      # tails past one tile in both directions
+    (300, 100, 1152),     # N <= 128 kernel, odd atom count
+    (128, 384, 2048),     # M <= 128 kernel (256-wide N tiles + a tail)
+    (64, 512, 8192),      # long K
+    (300, 520, 384),      # CTA-pair kernel: odd 128-row groups, half stage at the end
+    (1000, 700, 1024),    # CTA-pair kernel: tails, several tiles
+    (2048, 2560, 256),    # more tiles than SMs
+]
+
+
+@pytest.mark.parametrize("m,n,k", MX_SHAPES, ids=lambda v: str(v))
+def test_mx_gemm_matches_oracle(lib, m, n, k):
+    a = inputs.activations_with_outliers(m, k, seed=m + 3 * k, fraction=0.01, factor=30.0)
+    b = inputs.gaussian_bf16((n, k), seed=n + 5 * k, std=0.02)
+    d32, d_ref, s_ref = _mx_gemm_case(lib, a, b, torch.float32)
+    check_f32(d32.cpu().numpy(), d_ref, s_ref, 1.0)
+    d16, _, _ = _mx_gemm_case(lib, a, b, torch.bfloat16)
+    check_bf16(host_bf16_bits(d16), d_ref, s_ref, 1.0)
+
+
+def test_mx_gemm_output_pitch(lib):
+    m, n, k = 130, 136, 256
+    a = inputs.gaussian_bf16((m, k), seed=191)
+    b = inputs.gaussian_bf16((n, k), seed=192)
+    qa = lib.mxfp4_quantize(dev_bf16(a), lib.SF_TCGEN05)
+    qb = lib.mxfp4_quantize(dev_bf16(b), lib.SF_TCGEN05)
+    big = torch.full((m + 40, 288), -7.0, dtype=torch.bfloat16, device="cuda")
+    lib.nvfp4_mxfp4_gemm(qa.codes, qa.sf, qb.codes, qb.sf, m, n, k, big, 288, lib.OUT_BF16)
+    torch.cuda.synchronize()
+    pa, sa = MX.quantize_mx(a)
+    pb, sb = MX.quantize_mx(b)
+    d_ref, s_ref = MX.gemm_ref_mx(pa, sa, pb, sb)
+    check_bf16(host_bf16_bits(big[:m, :n]), d_ref, s_ref, 1.0)
+    assert torch.all(big[:m, n:] == -7.0) and torch.all(big[m:, :] == -7.0)
+
+
+def _mx_probe(lib, m, n, k, sa, sb):
+    """All-ones codes (E2M1 1.0 = code 2) with the given row-major E8M0 scales."""
+    codes_a = torch.full((m, k // 2), 0x22, dtype=torch.uint8, device="cuda")
+    codes_b = torch.full((n, k // 2), 0x22, dtype=torch.uint8, device="cuda")
+    sfa = torch.from_numpy(NV.swizzle_sf_tcgen05(sa)).cuda()
+    sfb = torch.from_numpy(NV.swizzle_sf_tcgen05(sb)).cuda()
+    assert sfa.numel() == MX.sf_tcgen05_bytes_mx(m, k) == lib.nvfp4_mxfp4_sf_bytes(m, k, lib.SF_TCGEN05)
+    d = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    lib.nvfp4_mxfp4_gemm(codes_a, sfa, codes_b, sfb, m, n, k, d, n, lib.OUT_F32)
+    torch.cuda.synchronize()
+    return d.cpu().numpy()
+
+
+@pytest.mark.parametrize("m,n", [(256, 256), (128, 256), (256, 128)], ids=["cta_pair", "m128", "n128"])
+@pytest.mark.parametrize("side", ["a", "b"])
+def test_mx_scale_layout_probes(lib, side, m, n):
+    """Exactly one (row, block) E8M0 scale is 2.0 (byte 128), all others 1.0
+    (byte 127): only that row (A side) or column (B side) of D grows, by exactly
+    32 (one block of 32 products 1 x 1).  Pins the 32-element scale blocks and
+    their placement in the tensor-core layout, for each of the three kernels."""
+    k = 640                        # 20 scales per row: 5 atoms, the last stage half full
+    kb = k // 32
+    limit = m if side == "a" else n
+    for row, blk in [(0, 0), (37, 5), (77, 18), (100, 19), (161, 9), (255, 13), (127, 1)]:
+        if row >= limit:
+            continue
+        sa = np.full((m, kb), 127, np.uint8)
+        sb = np.full((n, kb), 127, np.uint8)
+        (sa if side == "a" else sb)[row, blk] = 128
+        d = _mx_probe(lib, m, n, k, sa, sb)
+        want = np.full((m, n), float(k))
+        if side == "a":
+            want[row, :] += 32.0
+        else:
+            want[:, row] += 32.0
+        assert np.array_equal(d, want), (side, row, blk, np.argwhere(d != want)[:4].tolist())
+
+
+def test_mx_gemm_full_size_sampled(lib):
+    """8192^3 with the prefill inputs in MXFP4: 512 sampled outputs against the
+    oracle, the sampled rows' codes and scales bit-exact, all outputs finite."""
+    a, w = inputs.prefill_gemm()
+    qa = lib.mxfp4_quantize(dev_bf16(a), lib.SF_ROWMAJOR)
+    qw = lib.mxfp4_quantize(dev_bf16(w), lib.SF_ROWMAJOR)
+    ta = lib.mxfp4_quantize(dev_bf16(a), lib.SF_TCGEN05)
+    tw = lib.mxfp4_quantize(dev_bf16(w), lib.SF_TCGEN05)
+    d = lib.mxfp4_gemm(ta, tw, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    assert torch.isfinite(d).all()
+    rng = np.random.default_rng(29)
+    rows = rng.choice(8192, 512)
+    cols = rng.choice(8192, 512)
+    ur, uc = np.unique(rows), np.unique(cols)
+    pa, sa = MX.quantize_mx(a[ur])
+    pw, sw = MX.quantize_mx(w[uc])
+    assert np.array_equal(host_u8(qa.codes)[ur], pa) and np.array_equal(host_u8(qw.codes)[uc], pw)
+    assert np.array_equal(host_u8(qa.sf).reshape(8192, -1)[ur], sa)
+    assert np.array_equal(host_u8(qw.sf).reshape(8192, -1)[uc], sw)
+    d_ref, s_ref = MX.gemm_ref_mx_entries(pa, sa, pw, sw, np.searchsorted(ur, rows), np.searchsorted(uc, cols))
+    check_bf16(host_bf16_bits(d)[rows, cols], d_ref, s_ref, 1.0)
+
+
+def test_mx_gemm_rejects_bad_arguments(lib):
+    q = lib.mxfp4_quantize(dev_bf16(inputs.gaussian_bf16((128, 256), seed=1)), lib.SF_TCGEN05)
+    d = torch.empty((128, 128), dtype=torch.bfloat16, device="cuda")
+    c, sf = q.codes, q.sf
+    for args, want in [((c, sf, c, sf, 128, 128, 192, d, 128), lib.ERR_UNSUPPORTED_SHAPE),   # K % 128 != 0
+                       ((c, sf, c, sf, 128, 128, 256, d, 64), lib.ERR_INVALID_ARG),          # ldd < N
+                       ((c[:, 8:], sf, c, sf, 128, 128, 256, d, 128), lib.ERR_MISALIGNED)]:  # codes + 8 B
+        with pytest.raises(lib.NVFP4Error) as e:
+            lib.nvfp4_mxfp4_gemm(*args, lib.OUT_BF16)
+        assert e.value.status == want
