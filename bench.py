@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--part", choices=["quantize", "gemv", "longk", "gemm"], default=None,
+    ap.add_argument("--part", choices=["quantize", "gemv", "longk", "gemm", "mxquantize", "mxgemm"], default=None,
                     help="run one workload alone, --steps times (for profiling); prints its timing")
     return ap.parse_args()
 
@@ -354,6 +354,7 @@ def main():
             "device_status": nv.nvfp4_status_string(status),
         }
     if rank == 0 and parts_inputs is not None:
+        parts_inputs["prefill"] = (a, w)
         result["parts"] = bench_parts(nv, torch, dev, flush, parts_inputs, hbm_peak, fp4_peak, peaks_src)
         result["parts"]["gemm_only"] = {"tflops": result["roofline"]["achieved"],
                                         "frac_fp4_peak": result["roofline"]["frac"]}
@@ -501,6 +502,24 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
     ms = _timed(torch, dev, flush, lambda: nv.gemm_quant_a(ad, wq, out=dd, workspace=ws), 10)
     fl = 2.0 * am * nn * k
     out["long_k_4096x8192x28672"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_fp4_peak": fl / ms / 1e9 / fp4_peak}
+    del wq, ad, dd, ws
+
+    # MXFP4 (E8M0 scale per 32, no global scale): one-pass quantize of the
+    # same [16384, 8192] input and the 8192^3 GEMM on MXFP4 operands
+    x = to_dev(pin["quant"])
+    rows, k = x.shape
+    qm = nv.mxfp4_quantize(x, nv.SF_TCGEN05)
+    ms = _timed(torch, dev, flush, lambda: nv.mxfp4_quantize(x, nv.SF_TCGEN05, out=qm), reps)
+    one_pass = rows * k * 2 + rows * k // 2 + rows * k // 32
+    out["mxfp4_quantize_16384x8192"] = {"ms": ms, "gbs": one_pass / ms / 1e6,
+                                        "frac_hbm": one_pass / ms / 1e6 / hbm_peak, "algorithmic_bytes": one_pass}
+    del x, qm
+    a, w = pin["prefill"]
+    qa, qw = nv.mxfp4_quantize(a, nv.SF_TCGEN05), nv.mxfp4_quantize(w, nv.SF_TCGEN05)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ms = _timed(torch, dev, flush, lambda: nv.mxfp4_gemm(qa, qw, out=d), reps)
+    out["mxfp4_gemm_8192"] = {"ms": ms, "tflops": FLOPS_STEP / ms / 1e9,
+                              "frac_fp4_peak": FLOPS_STEP / ms / 1e9 / fp4_peak}
     assert nv.nvfp4_check_device_status() == nv.OK
     return out
 
@@ -508,7 +527,7 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
 def run_part(args):
     """One workload alone: generate its inputs, run it ``--steps`` times with the
     L2 flushed in between, print the median time."""
-    if args.part == "quantize":
+    if args.part in ("quantize", "mxquantize"):
         x_bits = inputs.quantize_bandwidth()
     elif args.part == "gemv":
         xg, wg = inputs.decode_gemv(16)
@@ -545,6 +564,15 @@ def run_part(args):
         ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, al.shape[0], wl.shape[0], al.shape[1]),
                          dtype=torch.uint8, device=dev)
         out["ms"] = _timed(torch, dev, flush, lambda: nv.gemm_quant_a(ad, wq, out=dd, workspace=ws), args.steps)
+    elif args.part == "mxquantize":
+        x = to_dev(x_bits)
+        q = nv.mxfp4_quantize(x, nv.SF_TCGEN05)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.mxfp4_quantize(x, nv.SF_TCGEN05, out=q), args.steps)
+    elif args.part == "mxgemm":
+        qa = nv.mxfp4_quantize(to_dev(a_bits), nv.SF_TCGEN05)
+        qw = nv.mxfp4_quantize(to_dev(w_bits), nv.SF_TCGEN05)
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.mxfp4_gemm(qa, qw, out=d), args.steps)
     else:
         qa = nv.quantize(to_dev(a_bits), nv.SF_TCGEN05)
         qw = nv.quantize(to_dev(w_bits), nv.SF_TCGEN05)
