@@ -21,6 +21,11 @@ Definition (fp32 operation order is part of the definition):
   5. pack two codes per byte, first element in the low nibble            [P5 技術原理: ONNX FLOAT4E2M1 packing]
   6. D = alpha * (s_a (.) A)(s_b (.) W)^T with alpha = 1 / (g_a * g_b) in fp32,
      accumulated here in fp64                                            [P1 §三 scaled GEMM; P4 mixed-precision MMA]
+  7. output scale g_d (optional outputs of the GEMM)                    [P1 §三: D = g_d * (...), "output dequant by g_d",
+     v = fp32(alpha * acc) is the value the fp32 output holds;           the _scaled_mm example: scale_result=g_d,
+     FP8 output: e4m3_rne_satfinite(fp32(v * g_d)), sign kept;           out_dtype=float8_e4m3fn]
+     NVFP4 output: steps 3-5 on v with g := g_d (g_d is the output's
+     encode scale, given by the caller); amax_d = max |v|
 
 Readings taken where the pages are silent or disagree are listed in the design doc
 of the repository; each function below states the one it uses.
@@ -153,7 +158,13 @@ def quantize_with_scale(x_bits, g):
     Returns (codes [rows, K] uint8, one code per element, unpacked;
              sf [rows, K/16] uint8 E4M3 block scales, row-major).
     """
-    x = bf16_to_f32(x_bits)
+    return quantize_values_with_scale(bf16_to_f32(x_bits), g)
+
+
+def quantize_values_with_scale(x, g):
+    """Steps 3-4 for fp32 values x [rows, K] (any fp32, not only bf16 ones) and
+    a given fp32 encode scale g; the same returns as quantize_with_scale."""
+    x = np.asarray(x, dtype=np.float32)
     rows, k = x.shape
     if k % BLOCK:
         raise ValueError("K must be a multiple of 16")
@@ -248,6 +259,37 @@ def gemm_ref_entries(a_packed, a_sf, g_a, b_packed, b_sf, g_b, rows, cols):
         d[i] = np.float64(alpha) * np.dot(ar, bc)
         s[i] = np.dot(np.abs(ar), np.abs(bc))
     return d, s, alpha
+
+
+# --------------------------------------------------------------------------
+# Output scale g_d [P1 §三: D = g_d * ((g_a s_a A)(g_b s_b W)), "输出反量化由
+# g_d 完成（输出常以 FP8/FP16 落盘）", and the _scaled_mm example with
+# scale_result=g_d, out_dtype=torch.float8_e4m3fn]
+# --------------------------------------------------------------------------
+def e4m3_encode_signed_satfinite(v) -> np.ndarray:
+    """Signed fp32 values -> E4M3 bytes: the magnitude as e4m3_encode_satfinite
+    (nearest, ties to the even code, >= 448 gives 448), the sign in bit 7
+    (-0 gives 0x80)."""
+    v = np.asarray(v, dtype=np.float32)
+    if not np.all(np.isfinite(v)):
+        raise ValueError("output values are finite")
+    mag = e4m3_encode_satfinite(np.abs(v))
+    return (mag | (np.signbit(v).astype(np.uint8) << 7)).astype(np.uint8)
+
+
+def fp8_output(v, g_d) -> np.ndarray:
+    """FP8 output bytes: e4m3_rne_satfinite(fp32(v * g_d))."""
+    t = (np.asarray(v, dtype=np.float32) * np.float32(g_d)).astype(np.float32)
+    return e4m3_encode_signed_satfinite(t)
+
+
+def nvfp4_output(v, g_d):
+    """NVFP4 output of fp32 values v [rows, N] under the given encode scale
+    g_d: (packed codes [rows, N/2], E4M3 block scales [rows, N/16] row-major,
+    amax = max |v|)."""
+    v = np.asarray(v, dtype=np.float32)
+    codes, sf = quantize_values_with_scale(v, g_d)
+    return pack_codes(codes), sf, (np.float32(np.max(np.abs(v))) if v.size else np.float32(0.0))
 
 
 # --------------------------------------------------------------------------
