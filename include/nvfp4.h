@@ -187,6 +187,41 @@ NVFP4_API nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_sf_tc, cons
                         const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d,
                         int64_t ldd, nvfp4_out_dtype out_dtype, nvfp4_stream_t stream);
 
+/*
+ * The GEMM of nvfp4_gemm with its result landing under an output scale g_d
+ * ("NVIDIA NVFP4 与 Micro-Scaling" section 三: D = g_d * (...), "output
+ * dequantization by g_d, the output often landing as FP8"; its _scaled_mm
+ * example passes scale_result=g_d with a float8_e4m3fn output).  With
+ * v = fp32(alpha * acc), the value nvfp4_gemm's fp32 output holds:
+ *
+ * nvfp4_gemm_fp8_out: d_e4m3[m, n] = e4m3_rne_satfinite(fp32(v * g_d)), one
+ *   byte per element (float8_e4m3fn), row pitch ldd bytes >= N; d_e4m3 16-byte
+ *   aligned and ldd % 16 == 0.
+ *
+ * nvfp4_gemm_requant: D quantized to NVFP4 for the next layer, g_d being D's
+ *   global encode scale (given; e.g. 2688 / amax of a previous step): per 16
+ *   consecutive columns s = e4m3_rne_satfinite(fp32(fp32(ab * g_d) / 6)) with
+ *   ab = max |v| over the block, codes e2m1_rne_sat(fp32(fp32(v * g_d) / sd))
+ *   (zero codes when sd == 0), two per byte, first in the low nibble.
+ *   d_codes [M, N/2] with row pitch ldd_bytes >= N/2 (16-byte aligned rows);
+ *   d_sf: block scales in d_sf_layout (nvfp4_sf_bytes(M, N, layout) bytes; in
+ *   the TCGEN05 layout the rows past M of the last 128-row group are not
+ *   written).  N % 16 == 0, and N % 64 == 0 for the TCGEN05 layout.
+ *
+ * Both: g_d_dev one fp32 on the device; amax_d_dev (optional, may be null)
+ * receives max |v| over D (zeroed by the call first), the input of the next
+ * step's encode scale.  Other arguments, shapes and errors as nvfp4_gemm.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_fp8_out(const void* a_codes, const void* a_sf_tc, const float* g_a_dev,
+                              const void* b_codes, const void* b_sf_tc, const float* g_b_dev, int64_t M,
+                              int64_t N, int64_t K, const float* g_d_dev, void* d_e4m3, int64_t ldd,
+                              float* amax_d_dev, nvfp4_stream_t stream);
+NVFP4_API nvfp4_status nvfp4_gemm_requant(const void* a_codes, const void* a_sf_tc, const float* g_a_dev,
+                              const void* b_codes, const void* b_sf_tc, const float* g_b_dev, int64_t M,
+                              int64_t N, int64_t K, const float* g_d_dev, void* d_codes, int64_t ldd_bytes,
+                              void* d_sf, nvfp4_sf_layout d_sf_layout, float* amax_d_dev,
+                              nvfp4_stream_t stream);
+
 /* Workspace bytes needed by an op for the given sizes (0 for bad sizes). */
 NVFP4_API size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K);
 

@@ -242,6 +242,38 @@ nvfp4_status nvfp4_gemm(const void* a_codes, const void* a_sf_tc, const float* g
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status nvfp4_gemm_fp8_out(const void* a_codes, const void* a_sf_tc, const float* g_a_dev,
+                                const void* b_codes, const void* b_sf_tc, const float* g_b_dev, int64_t M,
+                                int64_t N, int64_t K, const float* g_d_dev, void* d_e4m3, int64_t ldd,
+                                float* amax_d_dev, nvfp4_stream_t stream) {
+  nvfp4_status st = check_gemm_operands(a_codes, a_sf_tc, g_a_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d_e4m3);
+  if (st != NVFP4_OK) return st;
+  if (!g_d_dev || ldd < N) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(d_e4m3) || (ldd % 16) != 0) return NVFP4_ERR_MISALIGNED;
+  if ((st = check_arch()) != NVFP4_OK) return st;
+  const QuantOut q{QUANT_OUT_E4M3, nullptr, 0, g_d_dev, amax_d_dev};
+  return launch_gemm_q(a_codes, a_sf_tc, g_a_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d_e4m3, ldd, q,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_gemm_requant(const void* a_codes, const void* a_sf_tc, const float* g_a_dev,
+                                const void* b_codes, const void* b_sf_tc, const float* g_b_dev, int64_t M,
+                                int64_t N, int64_t K, const float* g_d_dev, void* d_codes, int64_t ldd_bytes,
+                                void* d_sf, nvfp4_sf_layout d_sf_layout, float* amax_d_dev,
+                                nvfp4_stream_t stream) {
+  nvfp4_status st = check_gemm_operands(a_codes, a_sf_tc, g_a_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d_codes);
+  if (st != NVFP4_OK) return st;
+  if (!g_d_dev || !d_sf) return NVFP4_ERR_INVALID_ARG;
+  if (d_sf_layout != NVFP4_SF_ROWMAJOR && d_sf_layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
+  if ((N % 16) != 0 || (d_sf_layout == NVFP4_SF_TCGEN05 && (N % 64) != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (ldd_bytes < N / 2) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(d_codes) || (ldd_bytes % 16) != 0) return NVFP4_ERR_MISALIGNED;
+  if ((st = check_arch()) != NVFP4_OK) return st;
+  const QuantOut q{QUANT_OUT_NVFP4, d_sf, d_sf_layout == NVFP4_SF_TCGEN05 ? 1 : 0, g_d_dev, amax_d_dev};
+  return launch_gemm_q(a_codes, a_sf_tc, g_a_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d_codes, ldd_bytes, q,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1 || (K % 64) != 0) return 0;
   if (op == NVFP4_OP_GEMV_BATCHED) {

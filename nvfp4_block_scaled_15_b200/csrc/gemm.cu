@@ -24,6 +24,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_core.cuh"
 #include "tc_common.cuh"
 
 namespace nvfp4 {
@@ -94,11 +95,107 @@ struct GemmParams {
   int out_f32;
   int vec_store;    // rows of D are 16-byte aligned: vector stores allowed
   int tma_store;    // bf16 D written by TMA stores through shared memory (CTA-pair kernel)
+  // Quantized output under the output scale g_d (out_q != 0): D leaves as
+  // FP8 E4M3 bytes (QUANT_OUT_E4M3) or as NVFP4 codes + E4M3 block scales
+  // (QUANT_OUT_NVFP4); ldd is then the row pitch in bytes.
+  int out_q;
+  uint8_t* q_sf;    // NVFP4 output block scales
+  int q_sf_tc;      // 1: tensor-core layout, 0: row-major [M, N/16]
+  int q_kb_pad;     // blocks per row of the tensor-core layout (N/16 rounded up to 4)
+  const float* g_d;
+  float* amax_d;    // max |alpha acc| over D, or null
   uint64_t wait_limit_ns;
   int* status;
 };
 
 __host__ __device__ __forceinline__ int round_up_int(int a, int b) { return (a + b - 1) / b * b; }
+
+// Quantized output of 16 columns of one row ("NVIDIA NVFP4 与 Micro-Scaling",
+// section 三: D = g_d * (...), landing as FP8 or, for the next layer, as
+// NVFP4).  x holds v = fp32(alpha * acc) of columns c .. c+15 (n_valid of
+// them inside D).  FP8: e4m3_rne_satfinite(fp32(v * g_d)) per element.
+// NVFP4: the quantizer's rule with g := g_d: s = e4m3(fp32(fp32(ab * g_d) / 6)),
+// codes e2m1(fp32(fp32(v * g_d) / sd)), sd == 0 -> zero codes.
+__device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n\tcvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void store_block_e4m3(uint8_t* out, const float (&x)[16], float gd, int n_valid) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = e4m3x2_bits(__fmul_rn(x[4 * i], gd), __fmul_rn(x[4 * i + 1], gd)) |
+           (e4m3x2_bits(__fmul_rn(x[4 * i + 2], gd), __fmul_rn(x[4 * i + 3], gd)) << 16);
+  if (n_valid == 16) {
+    *reinterpret_cast<uint4*>(out) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < n_valid) out[i] = static_cast<uint8_t>(w[i >> 2] >> (8 * (i & 3)));
+  }
+}
+
+// NVFP4 codes (8 bytes, element 0 in the low nibble) and scale byte of one block.
+__device__ __forceinline__ uint2 block_nvfp4(const float (&x)[16], float ab, float gd, uint32_t& s8) {
+  const float sixth = __frcp_rn(6.0f);
+  const float t = __fmul_rn(ab, gd);
+  const float q = __fmul_rn(t, sixth);
+  const float sr = __fmaf_rn(__fmaf_rn(q, -6.0f, t), sixth, q);                // RN(t / 6)
+  s8 = e4m3x2_bits(sr, 0.0f) & 0xFFu;
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(s8), __NV_E4M3);
+  const float sd = __half2float(__half(h));
+  if (sd == 0.0f) return make_uint2(0u, 0u);
+  const float y = __frcp_rn(sd);
+  float2 u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float t0 = __fmul_rn(x[2 * i], gd), t1 = __fmul_rn(x[2 * i + 1], gd);
+    u[i] = make_float2(div_rn_by_recip(t0, sd, y), div_rn_by_recip(t1, sd, y));
+  }
+  return make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
+}
+
+template <int NV>
+__device__ __forceinline__ void store_row_q(const GemmParams& p, int row, int col0, const uint32_t (&v)[NV],
+                                            float alpha, float gd, float& amax_run) {
+  if (row >= p.M) return;
+  uint8_t* out = static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row) * p.ldd;
+#pragma unroll
+  for (int b = 0; b < NV / 16; ++b) {
+    const int c = col0 + b * 16;
+    if (c >= p.N) break;
+    const int n_valid = min(16, p.N - c);
+    float x[16];
+    float ab = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      x[i] = __fmul_rn(__uint_as_float(v[b * 16 + i]), alpha);
+      if (i < n_valid) ab = fmaxf(ab, fabsf(x[i]));
+    }
+    amax_run = fmaxf(amax_run, ab);
+    if (p.out_q == QUANT_OUT_E4M3) {
+      store_block_e4m3(out + c, x, gd, n_valid);
+    } else {
+      uint32_t s8;
+      const uint2 codes = block_nvfp4(x, ab, gd, s8);
+      *reinterpret_cast<uint2*>(out + c / 2) = codes;
+      const int blk = c >> 4;
+      p.q_sf[p.q_sf_tc ? sf_tc_offset(row, blk, p.q_kb_pad) : static_cast<int64_t>(row) * (p.N >> 4) + blk] =
+          static_cast<uint8_t>(s8);
+    }
+  }
+}
+
+// One atomic per warp: the running |v| maximum of the warp's rows.
+__device__ __forceinline__ void publish_amax(const GemmParams& p, float amax_run) {
+  if (!p.out_q || !p.amax_d) return;
+  const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax_run));
+  if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned int*>(p.amax_d), m);
+}
 
 
 template <int NV>
@@ -304,6 +401,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, kMx>::THREADS, 1)
     const int half = ew >> 2;                  // which half of the tile's columns
     constexpr int HALF = BN / 2;
     const float alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    const float gd = p.out_q ? *p.g_d : 0.0f;
+    float amax_run = 0.0f;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -325,8 +424,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, kMx>::THREADS, 1)
       }
       const int row = tm * BM + quad * 32 + lane;
       const int col0 = tn * BN + half * HALF;
-      if (col0 < p.N) store_row<HALF>(p, row, col0, v, alpha);
+      if (col0 < p.N) {
+        if (p.out_q)
+          store_row_q<HALF>(p, row, col0, v, alpha, gd, amax_run);
+        else
+          store_row<HALF>(p, row, col0, v, alpha);
+      }
     }
+    publish_amax(p, amax_run);
   }
 
   __syncwarp();
@@ -576,6 +681,8 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
     const int half = ew >> 2;
     constexpr int HALF = C::BN / 2;
     const float alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    const float gd = p.out_q ? *p.g_d : 0.0f;
+    float amax_run = 0.0f;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     const uint32_t ovl_free_leader = mapa_shared(smem_u32(ovl_free), 0);
     int j = 0;
@@ -618,7 +725,9 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
       if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader + 8u * b);
       const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const int col0 = tn * C::BN + half * HALF;
-      if (p.tma_store) {
+      if (p.out_q) {
+        if (col0 < p.N) store_row_q<HALF>(p, row0 + lane, col0, v, alpha, gd, amax_run);
+      } else if (p.tma_store) {
         // Coalesced output: each 32 x 32 box goes through one of this warp's
         // two staging buffers and leaves by a TMA store; rows and columns past
         // the end of D are clipped by the store.
@@ -653,6 +762,7 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
       }
     }
     if (p.tma_store && lane == 0) bulk_wait_group<0>();
+    publish_amax(p, amax_run);
   }
 
   __syncwarp();
@@ -700,10 +810,21 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   return r == CUDA_SUCCESS;
 }
 
+// Output-quantization fields of the parameters (none when q is null).
+void set_quant_out(GemmParams& p, const QuantOut* q, int64_t N) {
+  if (!q || q->mode == 0) return;
+  p.out_q = q->mode;
+  p.q_sf = static_cast<uint8_t*>(q->sf);
+  p.q_sf_tc = q->sf_tc;
+  p.q_kb_pad = static_cast<int>(((N / 16) + 3) / 4 * 4);
+  p.g_d = q->g_d;
+  p.amax_d = q->amax_d;
+}
+
 template <bool kMx>
 nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                            const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
-                           nvfp4_out_dtype out, cudaStream_t s) {
+                           nvfp4_out_dtype out, const QuantOut* q, cudaStream_t s) {
   using C = PairCfg<kMx>;
   using F = typename C::F;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
@@ -714,7 +835,8 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   // through TMA stores.  The store clips boxes at the tensor's edge in whole
   // 16-B chunks, so a row end inside a chunk would be overrun: such D takes
   // the direct-store path.
-  const bool tma_store = out == NVFP4_OUT_BF16 && aligned16(d) && (ldd * 2) % 16 == 0 && N % 8 == 0;
+  const bool tma_store =
+      !(q && q->mode) && out == NVFP4_OUT_BF16 && aligned16(d) && (ldd * 2) % 16 == 0 && N % 8 == 0;
   memset(&tmD, 0, sizeof(tmD));
   if (tma_store && !make_out_map(&tmD, d, M, N, ldd)) return NVFP4_ERR_CUDA;
   GemmParams p{};
@@ -734,6 +856,7 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   const int64_t row_bytes = ldd * (p.out_f32 ? 4 : 2);
   p.vec_store = aligned16(d) && (row_bytes % 16) == 0;
   p.tma_store = tma_store;
+  set_quant_out(p, q, N);
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;
@@ -772,7 +895,7 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
 template <int BN, bool kMx>
 nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                       const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
-                      nvfp4_out_dtype out, cudaStream_t s) {
+                      nvfp4_out_dtype out, const QuantOut* q, cudaStream_t s) {
   using C = GemmCfg<BN, kMx>;
   CUtensorMap tmA, tmB;
   if (!make_code_map(&tmA, a_codes, M, K, BM) || !make_code_map(&tmB, b_codes, N, K, BN)) return NVFP4_ERR_CUDA;
@@ -792,6 +915,7 @@ nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, c
   p.out_f32 = out == NVFP4_OUT_F32;
   const int64_t row_bytes = ldd * (p.out_f32 ? 4 : 2);
   p.vec_store = aligned16(d) && (row_bytes % 16) == 0;
+  set_quant_out(p, q, N);
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;
@@ -809,22 +933,32 @@ nvfp4_status run_gemm(const void* a_codes, const void* a_sf, const float* g_a, c
 template <bool kMx>
 nvfp4_status dispatch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                            const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
-                           nvfp4_out_dtype out, cudaStream_t s) {
-  if (N <= 128) return run_gemm<128, kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
-  if (M <= 128) return run_gemm<256, kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
-  return run_gemm_pair<kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+                           nvfp4_out_dtype out, const QuantOut* q, cudaStream_t s) {
+  if (N <= 128) return run_gemm<128, kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, q, s);
+  if (M <= 128) return run_gemm<256, kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, q, s);
+  return run_gemm_pair<kMx>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, q, s);
 }
 
 nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                          const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                          int64_t ldd, nvfp4_out_dtype out, cudaStream_t s) {
-  return dispatch_gemm<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, s);
+  return dispatch_gemm<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, nullptr, s);
+}
+
+nvfp4_status launch_gemm_q(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                           const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
+                           int64_t ldd_bytes, const QuantOut& q, cudaStream_t s) {
+  if (q.amax_d) {
+    cudaError_t e = cudaMemsetAsync(q.amax_d, 0, sizeof(float), s);
+    if (e != cudaSuccess) return launch_status(e);
+  }
+  return dispatch_gemm<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd_bytes, NVFP4_OUT_BF16, &q, s);
 }
 
 nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,
                             int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out,
                             cudaStream_t s) {
-  return dispatch_gemm<true>(a_codes, a_sf, nullptr, b_codes, b_sf, nullptr, M, N, K, d, ldd, out, s);
+  return dispatch_gemm<true>(a_codes, a_sf, nullptr, b_codes, b_sf, nullptr, M, N, K, d, ldd, out, nullptr, s);
 }
 
 }  // namespace nvfp4

@@ -38,6 +38,21 @@ nvfp4_status launch_mx_quantize(const void* x, int64_t rows, int64_t k, int64_t 
 nvfp4_status launch_gemm(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                          const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                          int64_t ldd, nvfp4_out_dtype out, cudaStream_t s);
+// Quantized GEMM output under the output scale g_d (mode 1: FP8 E4M3 bytes;
+// mode 2: NVFP4 codes + E4M3 block scales in `sf`, tensor-core layout when
+// sf_tc); amax_d (optional) receives max |alpha acc| over D.
+constexpr int QUANT_OUT_E4M3 = 1;
+constexpr int QUANT_OUT_NVFP4 = 2;
+struct QuantOut {
+  int mode;                // QUANT_OUT_E4M3 or QUANT_OUT_NVFP4
+  void* sf;
+  int sf_tc;
+  const float* g_d;
+  float* amax_d;
+};
+nvfp4_status launch_gemm_q(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
+                           const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
+                           int64_t ldd_bytes, const QuantOut& q, cudaStream_t s);
 nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,
                             int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out,
                             cudaStream_t s);

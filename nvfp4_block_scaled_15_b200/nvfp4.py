@@ -47,6 +47,9 @@ _SIGS = {
     "nvfp4_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _vp], _i32),
     "nvfp4_swizzle_sf": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "nvfp4_gemm": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp], _i32),
+    "nvfp4_gemm_fp8_out": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp], _i32),
+    "nvfp4_gemm_requant": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp],
+                           _i32),
     "nvfp4_workspace_bytes": ([_i32, _i64, _i64, _i64], _sz),
     "nvfp4_gemv_batched": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _sz, _vp], _i32),
     "nvfp4_gemm_quant_a": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp], _i32),
@@ -129,6 +132,19 @@ def nvfp4_swizzle_sf(sf_rowmajor, rows, k, sf_tc, stream=None) -> None:
 def nvfp4_gemm(a_codes, a_sf, g_a, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype=OUT_BF16, stream=None) -> None:
     _check(_lib.nvfp4_gemm(_p(a_codes), _p(a_sf), _p(g_a), _p(b_codes), _p(b_sf), _p(g_b), m, n, k, _p(d), ldd,
                            out_dtype, _s(stream)), "nvfp4_gemm")
+
+
+def nvfp4_gemm_fp8_out(a_codes, a_sf, g_a, b_codes, b_sf, g_b, m, n, k, g_d, d, ldd, amax_d=None,
+                       stream=None) -> None:
+    _check(_lib.nvfp4_gemm_fp8_out(_p(a_codes), _p(a_sf), _p(g_a), _p(b_codes), _p(b_sf), _p(g_b), m, n, k,
+                                   _p(g_d), _p(d), ldd, _p(amax_d), _s(stream)), "nvfp4_gemm_fp8_out")
+
+
+def nvfp4_gemm_requant(a_codes, a_sf, g_a, b_codes, b_sf, g_b, m, n, k, g_d, d_codes, ldd_bytes, d_sf, layout,
+                       amax_d=None, stream=None) -> None:
+    _check(_lib.nvfp4_gemm_requant(_p(a_codes), _p(a_sf), _p(g_a), _p(b_codes), _p(b_sf), _p(g_b), m, n, k,
+                                   _p(g_d), _p(d_codes), ldd_bytes, _p(d_sf), layout, _p(amax_d), _s(stream)),
+           "nvfp4_gemm_requant")
 
 
 def nvfp4_gemv_batched(x, m, ldx, w_codes, w_sf, g_w, n, k, y, ldy, workspace, ws_bytes, stream=None) -> None:
@@ -218,6 +234,28 @@ def gemm(a: Quantized, b: Quantized, out_dtype=torch.bfloat16, out: torch.Tensor
     od = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
     d = out if out is not None else torch.empty((a.rows, b.rows), dtype=out_dtype, device=a.codes.device)
     nvfp4_gemm(a.codes, a.sf, a.g, b.codes, b.sf, b.g, a.rows, b.rows, a.k, d, d.stride(0), od, stream)
+    return d
+
+
+def gemm_requant(a: Quantized, b: Quantized, g_d: torch.Tensor, layout: int = SF_TCGEN05,
+                 out: Quantized | None = None, stream=None) -> Quantized:
+    """D = alpha (s_a A)(s_b B)^T quantized to NVFP4 under the given encode
+    scale g_d (one fp32 on the device); out.amax receives max |D|."""
+    assert a.layout == SF_TCGEN05 and b.layout == SF_TCGEN05 and a.k == b.k
+    q = out if out is not None else empty_quantized(a.rows, b.rows, layout, a.codes.device)
+    q.g.copy_(g_d.reshape(1))
+    nvfp4_gemm_requant(a.codes, a.sf, a.g, b.codes, b.sf, b.g, a.rows, b.rows, a.k, q.g, q.codes,
+                       q.codes.stride(0), q.sf, q.layout, q.amax, stream)
+    return q
+
+
+def gemm_fp8_out(a: Quantized, b: Quantized, g_d: torch.Tensor, out: torch.Tensor | None = None,
+                 amax_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """FP8 (float8_e4m3fn) e4m3(v * g_d) for v = alpha (s_a A)(s_b B)^T; amax_out receives max |v|."""
+    assert a.layout == SF_TCGEN05 and b.layout == SF_TCGEN05 and a.k == b.k
+    d = out if out is not None else torch.empty((a.rows, b.rows), dtype=torch.float8_e4m3fn, device=a.codes.device)
+    nvfp4_gemm_fp8_out(a.codes, a.sf, a.g, b.codes, b.sf, b.g, a.rows, b.rows, a.k, g_d, d, d.stride(0), amax_out,
+                       stream)
     return d
 
 
