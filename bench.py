@@ -52,7 +52,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--part", choices=["quantize", "gemv", "longk", "gemm", "mxquantize", "mxgemm"], default=None,
+    ap.add_argument("--part", choices=["quantize", "gemv", "longk", "gemm", "mxquantize", "mxgemm", "requant"],
+                    default=None,
                     help="run one workload alone, --steps times (for profiling); prints its timing")
     return ap.parse_args()
 
@@ -520,6 +521,29 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
     ms = _timed(torch, dev, flush, lambda: nv.mxfp4_gemm(qa, qw, out=d), reps)
     out["mxfp4_gemm_8192"] = {"ms": ms, "tflops": FLOPS_STEP / ms / 1e9,
                               "frac_fp4_peak": FLOPS_STEP / ms / 1e9 / fp4_peak}
+    del qa, qw, d
+
+    # 8192^3 GEMM whose epilogue writes the output quantized for the next
+    # layer (NVFP4, tensor-core scales, amax) or as FP8, under an output scale
+    # g_d; against the unfused chain GEMM (bf16 D) + quantize of D
+    qa, qw = nv.quantize(a, nv.SF_TCGEN05), nv.quantize(w, nv.SF_TCGEN05)
+    h = nv.empty_quantized(M, N, nv.SF_TCGEN05, dev)
+    h.g.fill_(2688.0 / 40.0)
+    ms_rq = _timed(torch, dev, flush, lambda: nv.nvfp4_gemm_requant(
+        qa.codes, qa.sf, qa.g, qw.codes, qw.sf, qw.g, M, N, K, h.g, h.codes, N // 2, h.sf, nv.SF_TCGEN05, h.amax),
+        reps)
+    d8 = torch.empty((M, N), dtype=torch.float8_e4m3fn, device=dev)
+    ms_f8 = _timed(torch, dev, flush, lambda: nv.nvfp4_gemm_fp8_out(
+        qa.codes, qa.sf, qa.g, qw.codes, qw.sf, qw.g, M, N, K, h.g, d8, N, h.amax), reps)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    hq = nv.empty_quantized(M, N, nv.SF_TCGEN05, dev)
+    ms_unfused = _timed(torch, dev, flush, lambda: (nv.gemm(qa, qw, out=d), nv.quantize(d, nv.SF_TCGEN05, out=hq)),
+                        reps)
+    out["gemm_requant_8192"] = {
+        "nvfp4_out_ms": ms_rq, "nvfp4_out_tflops": FLOPS_STEP / ms_rq / 1e9,
+        "nvfp4_out_frac_fp4_peak": FLOPS_STEP / ms_rq / 1e9 / fp4_peak,
+        "fp8_out_ms": ms_f8, "fp8_out_tflops": FLOPS_STEP / ms_f8 / 1e9,
+        "unfused_gemm_bf16_then_quantize_ms": ms_unfused}
     assert nv.nvfp4_check_device_status() == nv.OK
     return out
 
@@ -568,6 +592,14 @@ def run_part(args):
         x = to_dev(x_bits)
         q = nv.mxfp4_quantize(x, nv.SF_TCGEN05)
         out["ms"] = _timed(torch, dev, flush, lambda: nv.mxfp4_quantize(x, nv.SF_TCGEN05, out=q), args.steps)
+    elif args.part == "requant":
+        qa = nv.quantize(to_dev(a_bits), nv.SF_TCGEN05)
+        qw = nv.quantize(to_dev(w_bits), nv.SF_TCGEN05)
+        h = nv.empty_quantized(M, N, nv.SF_TCGEN05, dev)
+        h.g.fill_(2688.0 / 40.0)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.nvfp4_gemm_requant(
+            qa.codes, qa.sf, qa.g, qw.codes, qw.sf, qw.g, M, N, K, h.g, h.codes, N // 2, h.sf, nv.SF_TCGEN05,
+            h.amax), args.steps)
     elif args.part == "mxgemm":
         qa = nv.mxfp4_quantize(to_dev(a_bits), nv.SF_TCGEN05)
         qw = nv.mxfp4_quantize(to_dev(w_bits), nv.SF_TCGEN05)

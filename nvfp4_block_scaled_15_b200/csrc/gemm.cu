@@ -124,12 +124,14 @@ __device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi) {
   return r;
 }
 
-__device__ __forceinline__ void store_block_e4m3(uint8_t* out, const float (&x)[16], float gd, int n_valid) {
+__device__ __forceinline__ float vf(const uint32_t* x, int i) { return __uint_as_float(x[i]); }
+
+__device__ __forceinline__ void store_block_e4m3(uint8_t* out, const uint32_t* x, float gd, int n_valid) {
   uint32_t w[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    w[i] = e4m3x2_bits(__fmul_rn(x[4 * i], gd), __fmul_rn(x[4 * i + 1], gd)) |
-           (e4m3x2_bits(__fmul_rn(x[4 * i + 2], gd), __fmul_rn(x[4 * i + 3], gd)) << 16);
+    w[i] = e4m3x2_bits(__fmul_rn(vf(x, 4 * i), gd), __fmul_rn(vf(x, 4 * i + 1), gd)) |
+           (e4m3x2_bits(__fmul_rn(vf(x, 4 * i + 2), gd), __fmul_rn(vf(x, 4 * i + 3), gd)) << 16);
   if (n_valid == 16) {
     *reinterpret_cast<uint4*>(out) = make_uint4(w[0], w[1], w[2], w[3]);
   } else {
@@ -140,7 +142,7 @@ __device__ __forceinline__ void store_block_e4m3(uint8_t* out, const float (&x)[
 }
 
 // NVFP4 codes (8 bytes, element 0 in the low nibble) and scale byte of one block.
-__device__ __forceinline__ uint2 block_nvfp4(const float (&x)[16], float ab, float gd, uint32_t& s8) {
+__device__ __forceinline__ uint2 block_nvfp4(const uint32_t* x, float ab, float gd, uint32_t& s8) {
   const float sixth = __frcp_rn(6.0f);
   const float t = __fmul_rn(ab, gd);
   const float q = __fmul_rn(t, sixth);
@@ -153,39 +155,58 @@ __device__ __forceinline__ uint2 block_nvfp4(const float (&x)[16], float ab, flo
   float2 u[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float t0 = __fmul_rn(x[2 * i], gd), t1 = __fmul_rn(x[2 * i + 1], gd);
+    const float t0 = __fmul_rn(vf(x, 2 * i), gd), t1 = __fmul_rn(vf(x, 2 * i + 1), gd);
     u[i] = make_float2(div_rn_by_recip(t0, sd, y), div_rn_by_recip(t1, sd, y));
   }
   return make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
 }
 
 template <int NV>
-__device__ __forceinline__ void store_row_q(const GemmParams& p, int row, int col0, const uint32_t (&v)[NV],
+__device__ __forceinline__ void store_row_q(const GemmParams& p, int row, int col0, uint32_t (&v)[NV],
                                             float alpha, float gd, float& amax_run) {
+  static_assert(NV % 32 == 0, "whole pairs of 16-column blocks");
   if (row >= p.M) return;
   uint8_t* out = static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row) * p.ldd;
+  const bool nv = p.out_q != QUANT_OUT_E4M3;
 #pragma unroll
-  for (int b = 0; b < NV / 16; ++b) {
-    const int c = col0 + b * 16;
+  for (int pr = 0; pr < NV / 32; ++pr) {         // two blocks (32 columns) at a time
+    const int c = col0 + pr * 32;
     if (c >= p.N) break;
-    const int n_valid = min(16, p.N - c);
-    float x[16];
-    float ab = 0.0f;
+    uint2 codes[2];
+    uint32_t s2 = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      x[i] = __fmul_rn(__uint_as_float(v[b * 16 + i]), alpha);
-      if (i < n_valid) ab = fmaxf(ab, fabsf(x[i]));
+    for (int h = 0; h < 2; ++h) {
+      const int n_valid = max(0, min(16, p.N - (c + h * 16)));
+      uint32_t* x = v + pr * 32 + h * 16;          // v = fp32(alpha * acc), in place
+      float ab = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        x[i] = __float_as_uint(__fmul_rn(__uint_as_float(x[i]), alpha));
+        if (i < n_valid) ab = fmaxf(ab, fabsf(__uint_as_float(x[i])));
+      }
+      amax_run = fmaxf(amax_run, ab);
+      if (!nv) {
+        if (n_valid > 0) store_block_e4m3(out + c + h * 16, x, gd, n_valid);
+      } else {
+        uint32_t s8;
+        codes[h] = block_nvfp4(x, ab, gd, s8);
+        s2 |= s8 << (8 * h);
+      }
     }
-    amax_run = fmaxf(amax_run, ab);
-    if (p.out_q == QUANT_OUT_E4M3) {
-      store_block_e4m3(out + c, x, gd, n_valid);
+    if (!nv) continue;
+    // NVFP4: N % 16 == 0, so a block is wholly inside D or wholly outside;
+    // the scales of blocks 2j, 2j+1 are adjacent bytes in both layouts
+    const int blk = c >> 4;
+    uint8_t* sf = p.q_sf + (p.q_sf_tc ? sf_tc_offset(row, blk, p.q_kb_pad) : static_cast<int64_t>(row) * (p.N >> 4) + blk);
+    if (c + 32 <= p.N) {
+      *reinterpret_cast<uint4*>(out + c / 2) = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+      if (p.q_sf_tc || ((p.N >> 4) & 1) == 0)
+        *reinterpret_cast<uint16_t*>(sf) = static_cast<uint16_t>(s2);
+      else
+        sf[0] = static_cast<uint8_t>(s2), sf[1] = static_cast<uint8_t>(s2 >> 8);
     } else {
-      uint32_t s8;
-      const uint2 codes = block_nvfp4(x, ab, gd, s8);
-      *reinterpret_cast<uint2*>(out + c / 2) = codes;
-      const int blk = c >> 4;
-      p.q_sf[p.q_sf_tc ? sf_tc_offset(row, blk, p.q_kb_pad) : static_cast<int64_t>(row) * (p.N >> 4) + blk] =
-          static_cast<uint8_t>(s8);
+      *reinterpret_cast<uint2*>(out + c / 2) = codes[0];
+      sf[0] = static_cast<uint8_t>(s2);
     }
   }
 }
@@ -485,7 +506,10 @@ struct PairCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <bool kMx>
+// kQ: the epilogue writes the quantized output (FP8 or NVFP4 under g_d)
+// instead of bf16 / fp32 D; a separate instantiation keeps the TMA-store
+// path's registers out of it.
+template <bool kMx, bool kQ>
 __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -681,7 +705,7 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
     const int half = ew >> 2;
     constexpr int HALF = C::BN / 2;
     const float alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
-    const float gd = p.out_q ? *p.g_d : 0.0f;
+    const float gd = kQ ? *p.g_d : 0.0f;
     float amax_run = 0.0f;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     const uint32_t ovl_free_leader = mapa_shared(smem_u32(ovl_free), 0);
@@ -725,7 +749,7 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
       if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_leader + 8u * b);
       const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quad * 32;
       const int col0 = tn * C::BN + half * HALF;
-      if (p.out_q) {
+      if constexpr (kQ) {
         if (col0 < p.N) store_row_q<HALF>(p, row0 + lane, col0, v, alpha, gd, amax_run);
       } else if (p.tma_store) {
         // Coalesced output: each 32 x 32 box goes through one of this warp's
@@ -761,8 +785,8 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
         store_row<HALF>(p, row0 + lane, col0, v, alpha);
       }
     }
-    if (p.tma_store && lane == 0) bulk_wait_group<0>();
-    publish_amax(p, amax_run);
+    if (!kQ && p.tma_store && lane == 0) bulk_wait_group<0>();
+    if constexpr (kQ) publish_amax(p, amax_run);
   }
 
   __syncwarp();
@@ -860,8 +884,12 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   p.wait_limit_ns = wait_limit_ns();
   p.status = device_status_ptr();
   if (!p.status) return NVFP4_ERR_CUDA;
-  cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<kMx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmParams) =
+      gemm_pair_kernel<kMx, false>;
+  if constexpr (!kMx) {
+    if (p.out_q) kern = gemm_pair_kernel<false, true>;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return launch_status(e);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -881,14 +909,14 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   if (dev < 64 && max_pairs[dev] == 0) {
     cfg.gridDim = dim3(2 * (device_sm_count() / 2));
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<kMx>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
     if (e != cudaSuccess || clusters < 1) return launch_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
     max_pairs[dev] = clusters;
   }
   const int tiles = p.tiles_m * p.tiles_n;
   const int pairs = tiles < max_pairs[dev < 64 ? dev : 0] ? tiles : max_pairs[dev < 64 ? dev : 0];
   cfg.gridDim = dim3(2 * pairs);
-  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kMx>, tmA, tmB, tmSFA, tmSFB, tmD, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmSFA, tmSFB, tmD, p);
   return launch_status(e);
 }
 
