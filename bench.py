@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--part", choices=["quantize", "gemv", "longk", "gemm", "mxquantize", "mxgemm", "requant"],
+    ap.add_argument("--part", choices=["quantize", "hadamard", "gemv", "longk", "gemm", "mxquantize", "mxgemm", "requant"],
                     default=None,
                     help="run one workload alone, --steps times (for profiling); prints its timing")
     return ap.parse_args()
@@ -454,6 +454,29 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
         "quantize_pass_frac_hbm": one_pass / ms_q1 / 1e6 / hbm_peak}
     del x, q
 
+    # Hadamard-rotated quantize of the same input (orders 16 and 128): two
+    # passes, the transform computed in both; same algorithmic bytes
+    x = to_dev(pin["quant"])
+    q = nv.empty_quantized(rows, k, nv.SF_TCGEN05, dev)
+    had = {}
+    for order in (16, 128):
+        ms_h = _timed(torch, dev, flush, lambda: nv.quantize_hadamard(x, order, nv.SF_TCGEN05, out=q), reps)
+        ms_h1 = _timed(torch, dev, flush, lambda: nv.nvfp4_quantize_hadamard(
+            x, rows, k, k, order, q.codes, q.sf, nv.SF_TCGEN05, q.g, q.amax, 1), reps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            nv.quantize_hadamard(x, order, nv.SF_TCGEN05, out=q)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_hb = e0.elapsed_time(e1) / 10
+        had[f"order={order}"] = {
+            "ms": ms_h, "gbs_two_pass": two_pass / ms_h / 1e6, "frac_hbm": two_pass / ms_h / 1e6 / hbm_peak,
+            "back_to_back_ms": ms_hb, "back_to_back_frac_hbm": two_pass / ms_hb / 1e6 / hbm_peak,
+            "quantize_pass_ms": ms_h1, "quantize_pass_frac_hbm": one_pass / ms_h1 / 1e6 / hbm_peak}
+    out["hadamard_quantize_16384x8192"] = had
+    del x, q
+
     # decode GEMV: W [28672, 8192] pre-quantized, x [M, 8192] quantized in the call
     xg, wg = pin["gemv"]
     wq = nv.quantize(to_dev(wg), nv.SF_TCGEN05)
@@ -551,7 +574,7 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
 def run_part(args):
     """One workload alone: generate its inputs, run it ``--steps`` times with the
     L2 flushed in between, print the median time."""
-    if args.part in ("quantize", "mxquantize"):
+    if args.part in ("quantize", "mxquantize", "hadamard"):
         x_bits = inputs.quantize_bandwidth()
     elif args.part == "gemv":
         xg, wg = inputs.decode_gemv(16)
@@ -572,6 +595,12 @@ def run_part(args):
         x = to_dev(x_bits)
         q = nv.empty_quantized(*x.shape, nv.SF_TCGEN05, dev)
         out["ms"] = _timed(torch, dev, flush, lambda: nv.quantize(x, nv.SF_TCGEN05, out=q), args.steps)
+    elif args.part == "hadamard":
+        x = to_dev(x_bits)
+        q = nv.empty_quantized(*x.shape, nv.SF_TCGEN05, dev)
+        for order in (16, 128):
+            out[f"ms_order{order}"] = _timed(torch, dev, flush,
+                                             lambda: nv.quantize_hadamard(x, order, nv.SF_TCGEN05, out=q), args.steps)
     elif args.part == "gemv":
         wq = nv.quantize(to_dev(wg), nv.SF_TCGEN05)
         n, k = wg.shape

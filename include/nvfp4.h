@@ -130,6 +130,32 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t 
                             nvfp4_stream_t stream);
 
 /*
+ * Hadamard-rotated NVFP4 quantization ("NVIDIA NVFP4 与 Micro-Scaling",
+ * section 4.1 旋转/阿达玛变换: x is multiplied by an orthogonal Walsh-Hadamard
+ * matrix before quantization, which spreads outlier channels over all
+ * channels; giving the weights the same rotation along K leaves the product
+ * A W^T unchanged, since (A H)(W H)^T = A W^T).
+ *   y = x H, H = blockdiag(H_n, ..., H_n) / sqrt(n), H_n the Sylvester-ordered
+ *   Walsh-Hadamard matrix of order n.  y is formed in fp32 by the fast
+ *   transform (stages h = 1, 2, 4, ..., n/2, each pair (i, i + h) with bit h of
+ *   i clear becoming (y_i + y_{i+h}, y_i - y_{i+h})), then y * fp32(1/sqrt(n)).
+ *   y is then quantized exactly as nvfp4_quantize quantizes x, with the amax
+ *   taken over y.
+ *   hadamard_order : n, a power of two from 1 to 512 dividing k (1 leaves x
+ *           unrotated and gives nvfp4_quantize's result).
+ *   codes, sf, g_dev, layout, k constraints: as nvfp4_quantize.
+ *   amax_dev : amax_given == 0: out, max |y| (two passes over x, the transform
+ *           recomputed in the second).  amax_given == 1: in, used as max |y|.
+ * Rotate both GEMM operands with the same n; nvfp4_gemm then gives
+ * approximately A W^T.  Errors: INVALID_ARG for an order that is not a power
+ * of two in [1, 512], UNSUPPORTED_SHAPE when it does not divide k; a non-finite
+ * max |y| behaves as in nvfp4_quantize (zero outputs, device status RANGE).
+ */
+NVFP4_API nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx,
+                                     int hadamard_order, void* codes, void* sf, nvfp4_sf_layout layout,
+                                     float* g_dev, float* amax_dev, int amax_given, nvfp4_stream_t stream);
+
+/*
  * MXFP4, the format the pages set against NVFP4 ("mxFP4/nvFP4 最小化知识",
  * (一) mxFP4的技术局限; "low-precision-floats", FP4 / MXFP4 / NVFP4): one E8M0
  * (power-of-two) scale per 32 consecutive elements along K and no global

@@ -194,6 +194,63 @@ __device__ __forceinline__ void quantize_two_blocks(const uint32_t (&w0)[8], con
   c1 = block_codes(w1, g, table[s1 & 0x7Fu]);
 }
 
+// ---------------------------------------------------------------------------
+// fp32 blocks (the rotated values of the Hadamard path): element 2i of a
+// block in p[i].x, element 2i+1 in p[i].y.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bf16_block_to_f32(const uint32_t (&w)[8], float2 (&p)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
+}
+
+// |y| maximum of 16 finite fp32 values (exact).
+__device__ __forceinline__ float abs_max16_f32(const float2 (&p)[8]) {
+  float m = fabsf(p[0].x);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(fmaxf(m, fabsf(p[i].x)), fabsf(p[i].y));
+  return m;
+}
+
+// 16 codes of one fp32 block for the scale entry e = {sd, RN(1/sd)}: the same
+// rule as block_codes, RN(RN(y * g) / sd) then E2M1 RNE with saturation.
+__device__ __forceinline__ uint2 block_codes_f32(const float2 (&p)[8], float g, float2 e) {
+  const float2 g2 = make_float2(g, g);
+  const float2 y2 = make_float2(e.y, e.y);
+  const float2 nsd2 = make_float2(-e.x, -e.x);
+  float2 u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 t = __fmul2_rn(p[i], g2);                                     // y * g
+    const float2 q = __fmul2_rn(t, y2);
+    const float2 r = __ffma2_rn(q, nsd2, t);                                   // exact remainder
+    const float2 d = __ffma2_rn(r, y2, q);                                     // RN(t / sd)
+    u[i] = make_float2(copysignf(d.x, t.x), copysignf(d.y, t.y));
+  }
+  uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
+  if (e.x == 0.0f) c = make_uint2(0u, 0u);
+  return c;
+}
+
+// Two fp32 blocks at once, as quantize_two_blocks.
+__device__ __forceinline__ void quantize_two_blocks_f32(const float2 (&p0)[8], const float2 (&p1)[8], float g,
+                                                        const float2* table, uint2& c0, uint2& c1, uint32_t& s0,
+                                                        uint32_t& s1) {
+  const float sixth = __frcp_rn(6.0f);
+  const float2 ab = make_float2(abs_max16_f32(p0), abs_max16_f32(p1));
+  const float2 t = __fmul2_rn(ab, make_float2(g, g));
+  const float2 q = __fmul2_rn(t, make_float2(sixth, sixth));
+  const float2 r = __ffma2_rn(q, make_float2(-6.0f, -6.0f), t);
+  const float2 sr = __ffma2_rn(r, make_float2(sixth, sixth), q);               // RN(t / 6)
+  uint32_t s2;
+  asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n\tcvt.u32.u16 %0, h;\n\t}"
+      : "=r"(s2)
+      : "f"(sr.y), "f"(sr.x));
+  s0 = s2 & 0xFFu;
+  s1 = (s2 >> 8) & 0xFFu;
+  c0 = block_codes_f32(p0, g, table[s0 & 0x7Fu]);
+  c1 = block_codes_f32(p1, g, table[s1 & 0x7Fu]);
+}
+
 // Byte offset of (row r, block b) in the tensor-core scale layout whose
 // padded block count is kb_pad (a multiple of 4).
 __host__ __device__ __forceinline__ int64_t sf_tc_offset(int64_t r, int64_t b, int64_t kb_pad) {

@@ -5,6 +5,8 @@
 // owns whole 16-element blocks ("NVIDIA NVFP4 与
 // Micro-Scaling" section 三: global scale from |X|_max, then per-block
 // micro-scales; "low-precision-floats" section FP4 / MXFP4 / NVFP4 formulas).
+#include <cmath>
+
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -81,6 +83,43 @@ __device__ __forceinline__ void load_block(const uint16_t* p, uint32_t (&w)[8]) 
   }
 }
 
+// Stores of one thread's two blocks (codes c0, c1 and scale bytes s0, s1 of
+// blocks b0, b1 of row r): codes row-major [rows, k/2], scales row-major or
+// in the tensor-core layout (where rows >= `rows` exist and get zero scales).
+template <bool kTcLayout>
+__device__ __forceinline__ void store_two_blocks(uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int r,
+                                                 bool real_row, int k, int kb, int b0, int b1, uint2 c0, uint2 c1,
+                                                 uint32_t s0, uint32_t s1) {
+  if (real_row) {
+    uint8_t* cr = codes + static_cast<int64_t>(r) * (k >> 1);
+    if ((reinterpret_cast<uintptr_t>(codes) & 7u) == 0) {
+      if (b0 < kb) *reinterpret_cast<uint2*>(cr + b0 * 8) = c0;
+      if (b1 < kb) *reinterpret_cast<uint2*>(cr + b1 * 8) = c1;
+    } else {
+      if (b0 < kb) {
+        reinterpret_cast<uint32_t*>(cr + b0 * 8)[0] = c0.x;
+        reinterpret_cast<uint32_t*>(cr + b0 * 8)[1] = c0.y;
+      }
+      if (b1 < kb) {
+        reinterpret_cast<uint32_t*>(cr + b1 * 8)[0] = c1.x;
+        reinterpret_cast<uint32_t*>(cr + b1 * 8)[1] = c1.y;
+      }
+    }
+  }
+  if (!kTcLayout) {
+    if (real_row) {
+      uint8_t* sr = sf + static_cast<int64_t>(r) * kb;
+      if (b0 < kb) sr[b0] = static_cast<uint8_t>(s0);
+      if (b1 < kb) sr[b1] = static_cast<uint8_t>(s1);
+    }
+  } else {
+    // byte of (row r, block b) = row_base + (b / 4) * 512 + b % 4
+    const int64_t row_base = (static_cast<int64_t>(r >> 7) * (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+    if (b0 < kb) sf[row_base + ((b0 >> 2) << 9) + (b0 & 3)] = static_cast<uint8_t>(s0);
+    if (b1 < kb) sf[row_base + ((b1 >> 2) << 9) + (b1 & 3)] = static_cast<uint8_t>(s1);
+  }
+}
+
 template <bool kTcLayout, bool kWide>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                             int64_t ldx, uint8_t* __restrict__ codes,
@@ -126,34 +165,173 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   uint32_t s0, s1;
   quantize_two_blocks(w0, w1, g, table, c0, c1, s0, s1);
 
-  if (real_row) {
-    uint8_t* cr = codes + static_cast<int64_t>(r) * (k >> 1);
-    if ((reinterpret_cast<uintptr_t>(codes) & 7u) == 0) {
-      if (b0 < kb) *reinterpret_cast<uint2*>(cr + b0 * 8) = c0;
-      if (b1 < kb) *reinterpret_cast<uint2*>(cr + b1 * 8) = c1;
-    } else {
-      if (b0 < kb) {
-        reinterpret_cast<uint32_t*>(cr + b0 * 8)[0] = c0.x;
-        reinterpret_cast<uint32_t*>(cr + b0 * 8)[1] = c0.y;
-      }
-      if (b1 < kb) {
-        reinterpret_cast<uint32_t*>(cr + b1 * 8)[0] = c1.x;
-        reinterpret_cast<uint32_t*>(cr + b1 * 8)[1] = c1.y;
+  store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
+}
+
+// ---------------------------------------------------------------------------
+// Hadamard-rotated NVFP4 ("NVIDIA NVFP4 与 Micro-Scaling", section 4.1: the
+// activations are multiplied by an orthogonal Walsh-Hadamard matrix before
+// quantization, which spreads outlier channels over all channels; the
+// adjacent weights take the same rotation, so the layer's product is
+// unchanged).  H = blockdiag(H_n, ..., H_n) / sqrt(n) with H_n the
+// Sylvester-ordered Walsh-Hadamard matrix of order n (a power of two, n <= 512,
+// n dividing k).  y = x H is formed in fp32 by the fast transform: stages
+// h = 1, 2, 4, ..., n/2, each turning (y_i, y_{i+h}) (bit h of i clear) into
+// (y_i + y_{i+h}, y_i - y_{i+h}), then y * fp32(1/sqrt(n)).  y is then
+// quantized like any fp32 tensor, its amax taken over y.
+//
+// Thread layout as in quantize_kernel: a thread owns blocks b0 = segment * 512
+// + tid and b1 = b0 + 256 of a row, 16 elements each.  Stages h < 16 run inside
+// the thread; a stage h >= 16 pairs the lanes that own blocks j and j + h/16,
+// i.e. lanes tid and tid ^ (h/16) of one warp (h/16 <= 16).
+// ---------------------------------------------------------------------------
+
+// Stages h = 1, 2, 4, 8 (those below n) on one thread's block.  h = 1 pairs
+// the two halves of a float2; h = 2, 4, 8 pair float2 entries hp = h/2 apart.
+// a - b is computed as a + (-b), which IEEE arithmetic rounds identically.
+__device__ __forceinline__ void fwht_in_thread(float2 (&p)[8], int n) {
+  if (n > 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      p[i] = __fadd2_rn(make_float2(p[i].x, p[i].x), make_float2(p[i].y, -p[i].y));
+  }
+#pragma unroll
+  for (int hp = 1; hp < 8; hp *= 2) {
+    if (n > 2 * hp) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i & hp) continue;
+        const float2 a = p[i], b = p[i + hp];
+        p[i] = __fadd2_rn(a, b);
+        p[i + hp] = __fadd2_rn(a, make_float2(-b.x, -b.y));
       }
     }
   }
-  if (!kTcLayout) {
-    if (real_row) {
-      uint8_t* sr = sf + static_cast<int64_t>(r) * kb;
-      if (b0 < kb) sr[b0] = static_cast<uint8_t>(s0);
-      if (b1 < kb) sr[b1] = static_cast<uint8_t>(s1);
+}
+
+// Stages h = 16, 32, ..., n/2 across lanes (lane mask lm = h/16).  The lane
+// holding y_i (bit lm clear) forms y_i + y_{i+h}, its partner y_i - y_{i+h};
+// fma(v, +-1, w) rounds exactly as w +- v.  n is uniform over the warp.
+__device__ __forceinline__ void fwht_cross_lanes(float2 (&p0)[8], float2 (&p1)[8], int n) {
+#pragma unroll
+  for (int lm = 1; lm < 32; lm <<= 1) {
+    if (16 * lm < n) {
+      const float sg = (threadIdx.x & lm) ? -1.0f : 1.0f;
+      const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 o0 = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p0[i].x, lm),
+                                      __shfl_xor_sync(0xFFFFFFFFu, p0[i].y, lm));
+        const float2 o1 = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p1[i].x, lm),
+                                      __shfl_xor_sync(0xFFFFFFFFu, p1[i].y, lm));
+        p0[i] = __ffma2_rn(p0[i], s2, o0);
+        p1[i] = __ffma2_rn(p1[i], s2, o1);
+      }
     }
+  }
+}
+
+// y = x H for the thread's two blocks (bf16 words in, fp32 out), c = fp32(1/sqrt(n)).
+__device__ __forceinline__ void rotate_two_blocks(const uint32_t (&w0)[8], const uint32_t (&w1)[8], int n, float c,
+                                                  float2 (&p0)[8], float2 (&p1)[8]) {
+  bf16_block_to_f32(w0, p0);
+  bf16_block_to_f32(w1, p1);
+  fwht_in_thread(p0, n);
+  fwht_in_thread(p1, n);
+  fwht_cross_lanes(p0, p1, n);
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    p0[i] = __fmul2_rn(p0[i], c2);
+    p1[i] = __fmul2_rn(p1[i], c2);
+  }
+}
+
+template <bool kWide>
+__device__ __forceinline__ void load_two_blocks(const uint16_t* xr, bool ok, int kb, int b0, int b1,
+                                                uint32_t (&w0)[8], uint32_t (&w1)[8]) {
+  if (ok && b0 < kb) {
+    load_block<kWide>(xr + b0 * 16, w0);
   } else {
-    // byte of (row r, block b) = row_base + (b / 4) * 512 + b % 4
-    const int64_t row_base = (static_cast<int64_t>(r >> 7) * (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
-    if (b0 < kb) sf[row_base + ((b0 >> 2) << 9) + (b0 & 3)] = static_cast<uint8_t>(s0);
-    if (b1 < kb) sf[row_base + ((b1 >> 2) << 9) + (b1 & 3)] = static_cast<uint8_t>(s1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w0[i] = 0u;
   }
+  if (ok && b1 < kb) {
+    load_block<kWide>(xr + b1 * 16, w1);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w1[i] = 0u;
+  }
+}
+
+// Pass 1 of the rotated quantizer: max |y| over the tensor.  grid.x strides
+// over rows, grid.y over segments of 512 blocks.  The maximum runs on the
+// fp32 magnitude bits, so a NaN or an infinity in y reaches the global amax
+// (and the quantize pass reports it) instead of being dropped.
+template <bool kWide>
+__global__ void __launch_bounds__(kThreads) hadamard_amax_kernel(const uint16_t* __restrict__ x, int rows, int k,
+                                                                 int64_t ldx, int n, float c,
+                                                                 unsigned* __restrict__ amax_bits) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int kb = k >> 4;
+  const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
+  const int b1 = b0 + kThreads;
+  uint32_t m = 0;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    uint32_t w0[8], w1[8];
+    load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, true, kb, b0, b1, w0, w1);
+    float2 p0[8], p1[8];
+    rotate_two_blocks(w0, w1, n, c, p0, p1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      m = max(m, max(__float_as_uint(p0[i].x) & 0x7FFFFFFFu, __float_as_uint(p0[i].y) & 0x7FFFFFFFu));
+      m = max(m, max(__float_as_uint(p1[i].x) & 0x7FFFFFFFu, __float_as_uint(p1[i].y) & 0x7FFFFFFFu));
+    }
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t red[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t t = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (threadIdx.x == 0 && t != 0) atomicMax(amax_bits, t);
+  }
+}
+
+// Pass 2: rotate again and quantize y (same grid and stores as quantize_kernel).
+template <bool kTcLayout, bool kWide>
+__global__ void __launch_bounds__(kThreads)
+    hadamard_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
+                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
+                             const float* __restrict__ amax_in, int* __restrict__ status) {
+  __shared__ float2 table[128];
+  const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
+  const int kb = k >> 4;
+  const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
+  const int b1 = b0 + kThreads;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  bool valid;
+  float g = global_scale_from_amax(*amax_in, valid);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    *g_out = valid ? g : 0.0f;
+    if (!valid) record_status(status, kDevRange);
+  }
+  if (!valid) g = 0.0f;
+  const bool real_row = r < rows;
+
+  uint32_t w0[8], w1[8];
+  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row && valid, kb, b0, b1, w0, w1);
+  fill_scale_table(table);
+  __syncthreads();
+
+  float2 p0[8], p1[8];
+  rotate_two_blocks(w0, w1, n, c, p0, p1);
+  uint2 c0, c1;
+  uint32_t s0, s1;
+  quantize_two_blocks_f32(p0, p1, g, table, c0, c1, s0, s1);
+  store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
 
 // ---------------------------------------------------------------------------
@@ -277,6 +455,27 @@ cudaError_t launch_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, in
   return cudaLaunchKernelEx(&cfg, quantize_kernel<kTc, kWide>, x, rows, k, ldx, codes, sf, g_dev, amax_dev, status);
 }
 
+template <bool kTc, bool kWide>
+cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
+                                         int n, float c, uint8_t* codes, uint8_t* sf, float* g_dev,
+                                         const float* amax_dev, int* status) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, hadamard_quantize_kernel<kTc, kWide>, x, rows, k, ldx, n, c, codes, sf, g_dev,
+                            amax_dev, status);
+}
+
+// fp32(1/sqrt(n)) for the transform's order n (a power of two): the double
+// quotient of the correctly rounded double square root, rounded to fp32.
+float hadamard_norm(int n) { return static_cast<float>(1.0 / std::sqrt(static_cast<double>(n))); }
+
 }  // namespace
 
 nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s) {
@@ -343,6 +542,57 @@ nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst,
   swizzle_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(src), static_cast<int>(rows),
                                       static_cast<int>(kb), words, static_cast<uint32_t*>(dst));
   return launch_status(cudaGetLastError());
+}
+
+nvfp4_status launch_hadamard_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, int n, float* amax_dev,
+                                  cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(amax_dev, 0, sizeof(float), s);
+  if (e != cudaSuccess) return launch_status(e);
+  if (rows == 0 || k == 0) return NVFP4_OK;
+  const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
+  const int64_t want = static_cast<int64_t>(device_sm_count()) * 8 / segs;
+  const int gx = static_cast<int>(rows < want ? rows : (want > 0 ? want : 1));
+  const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  unsigned* out = reinterpret_cast<unsigned*>(amax_dev);
+  const float c = hadamard_norm(n);
+  if (wide)
+    hadamard_amax_kernel<true><<<dim3(gx, segs), kThreads, 0, s>>>(xs, static_cast<int>(rows), static_cast<int>(k),
+                                                                   ldx, n, c, out);
+  else
+    hadamard_amax_kernel<false><<<dim3(gx, segs), kThreads, 0, s>>>(xs, static_cast<int>(rows), static_cast<int>(k),
+                                                                    ldx, n, c, out);
+  return launch_status(cudaGetLastError());
+}
+
+nvfp4_status launch_hadamard_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, int n, void* codes,
+                                      void* sf, nvfp4_sf_layout layout, float* g_dev, const float* amax_dev,
+                                      cudaStream_t s) {
+  int* status = device_status_ptr();
+  if (!status) return NVFP4_ERR_CUDA;
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  uint8_t* cs = static_cast<uint8_t*>(codes);
+  uint8_t* ss = static_cast<uint8_t*>(sf);
+  const float c = hadamard_norm(n);
+  const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
+  const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
+  const int ir = static_cast<int>(rows), ik = static_cast<int>(k);
+  if (grid_rows == 0 || segs == 0)   // nothing to quantize: still publish g (from the given amax)
+    return launch_status(launch_hadamard_quantize_pdl<false, false>(dim3(1, 1), s, xs, 0, 0, ldx, n, c, cs, ss,
+                                                                    g_dev, amax_dev, status));
+  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  cudaError_t e;
+  if (layout == NVFP4_SF_TCGEN05)
+    e = wide ? launch_hadamard_quantize_pdl<true, true>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev, status)
+             : launch_hadamard_quantize_pdl<true, false>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
+                                                         status);
+  else
+    e = wide ? launch_hadamard_quantize_pdl<false, true>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
+                                                         status)
+             : launch_hadamard_quantize_pdl<false, false>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
+                                                          status);
+  return launch_status(e);
 }
 
 }  // namespace nvfp4
