@@ -156,17 +156,17 @@ __device__ __forceinline__ uint32_t abs_max_bits16(const uint32_t (&w)[8]) {
 // entry e = {sd, RN(1/sd)}: RN(RN(x * g) / sd) by the FMA correction, then
 // E2M1 RNE with saturation; sd == 0 gives all-zero codes.
 __device__ __forceinline__ uint2 block_codes(const uint32_t (&w)[8], float g, float2 e) {
-  const float2 g2 = make_float2(g, g);
-  const float2 y2 = make_float2(e.y, e.y);
-  const float2 nsd2 = make_float2(-e.x, -e.x);
+  const float2 ng2 = make_float2(-g, -g);
+  const float2 nyr2 = make_float2(-e.y, -e.y);
+  const float2 sd2 = make_float2(e.x, e.x);
   float2 u[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 t = __fmul2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), g2);   // x * g
-    const float2 q = __fmul2_rn(t, y2);                                         // RN(t * RN(1/sd))
-    const float2 r = __ffma2_rn(q, nsd2, t);                                    // t - q * sd, exact
-    const float2 d = __ffma2_rn(r, y2, q);                                      // RN(t / sd)
-    u[i] = make_float2(copysignf(d.x, t.x), copysignf(d.y, t.y));
+    // negated operands as in block_codes_f32: no sign fix-up for x = -0
+    const float2 tn = __fmul2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), ng2);  // -(x * g)
+    const float2 q = __fmul2_rn(tn, nyr2);                                      // RN(t * RN(1/sd))
+    const float2 rr = __ffma2_rn(q, sd2, tn);                                   // q * sd - t, exact
+    u[i] = __ffma2_rn(rr, nyr2, q);                                             // RN(t / sd)
   }
   uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
   if (e.x == 0.0f) c = make_uint2(0u, 0u);
@@ -203,52 +203,51 @@ __device__ __forceinline__ void bf16_block_to_f32(const uint32_t (&w)[8], float2
   for (int i = 0; i < 8; ++i) p[i] = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
 }
 
+// Three-input fp32 maximum; the .NaN form returns NaN if any input is NaN.
+__device__ __forceinline__ float max3_f32(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3_nan_f32(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // |y| maximum of 16 finite fp32 values (exact).
 __device__ __forceinline__ float abs_max16_f32(const float2 (&p)[8]) {
-  float m = fabsf(p[0].x);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(fmaxf(m, fabsf(p[i].x)), fabsf(p[i].y));
-  return m;
+  float m = max3_f32(fabsf(p[0].x), fabsf(p[0].y), fabsf(p[1].x));
+  m = max3_f32(m, fabsf(p[1].y), fabsf(p[2].x));
+  m = max3_f32(m, fabsf(p[2].y), fabsf(p[3].x));
+  m = max3_f32(m, fabsf(p[3].y), fabsf(p[4].x));
+  m = max3_f32(m, fabsf(p[4].y), fabsf(p[5].x));
+  m = max3_f32(m, fabsf(p[5].y), fabsf(p[6].x));
+  m = max3_f32(m, fabsf(p[6].y), fabsf(p[7].x));
+  return fmaxf(m, fabsf(p[7].y));
 }
 
 // 16 codes of one fp32 block for the scale entry e = {sd, RN(1/sd)}: the same
 // rule as block_codes, RN(RN(y * g) / sd) then E2M1 RNE with saturation.
+// The division runs on negated operands: tn = RN(y * -g) = -t, q = RN(tn * -yr)
+// = RN(t * yr), rr = RN(q * sd + tn) = q * sd - t exactly, and
+// d = RN(q + rr * -yr) = RN(t / sd) (the FMA correction of div_rn_by_recip).
+// This order also gives t = -0 the quotient -0 (code 0x8) with no sign fix-up.
 __device__ __forceinline__ uint2 block_codes_f32(const float2 (&p)[8], float g, float2 e) {
-  const float2 g2 = make_float2(g, g);
-  const float2 y2 = make_float2(e.y, e.y);
-  const float2 nsd2 = make_float2(-e.x, -e.x);
+  const float2 ng2 = make_float2(-g, -g);
+  const float2 nyr2 = make_float2(-e.y, -e.y);
+  const float2 sd2 = make_float2(e.x, e.x);
   float2 u[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 t = __fmul2_rn(p[i], g2);                                     // y * g
-    const float2 q = __fmul2_rn(t, y2);
-    const float2 r = __ffma2_rn(q, nsd2, t);                                   // exact remainder
-    const float2 d = __ffma2_rn(r, y2, q);                                     // RN(t / sd)
-    u[i] = make_float2(copysignf(d.x, t.x), copysignf(d.y, t.y));
+    const float2 tn = __fmul2_rn(p[i], ng2);                                   // -(y * g)
+    const float2 q = __fmul2_rn(tn, nyr2);                                     // RN(t * RN(1/sd))
+    const float2 rr = __ffma2_rn(q, sd2, tn);                                  // q * sd - t, exact
+    u[i] = __ffma2_rn(rr, nyr2, q);                                            // RN(t / sd)
   }
   uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
   if (e.x == 0.0f) c = make_uint2(0u, 0u);
   return c;
-}
-
-// Two fp32 blocks at once, as quantize_two_blocks.
-__device__ __forceinline__ void quantize_two_blocks_f32(const float2 (&p0)[8], const float2 (&p1)[8], float g,
-                                                        const float2* table, uint2& c0, uint2& c1, uint32_t& s0,
-                                                        uint32_t& s1) {
-  const float sixth = __frcp_rn(6.0f);
-  const float2 ab = make_float2(abs_max16_f32(p0), abs_max16_f32(p1));
-  const float2 t = __fmul2_rn(ab, make_float2(g, g));
-  const float2 q = __fmul2_rn(t, make_float2(sixth, sixth));
-  const float2 r = __ffma2_rn(q, make_float2(-6.0f, -6.0f), t);
-  const float2 sr = __ffma2_rn(r, make_float2(sixth, sixth), q);               // RN(t / 6)
-  uint32_t s2;
-  asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n\tcvt.u32.u16 %0, h;\n\t}"
-      : "=r"(s2)
-      : "f"(sr.y), "f"(sr.x));
-  s0 = s2 & 0xFFu;
-  s1 = (s2 >> 8) & 0xFFu;
-  c0 = block_codes_f32(p0, g, table[s0 & 0x7Fu]);
-  c1 = block_codes_f32(p1, g, table[s1 & 0x7Fu]);
 }
 
 // Byte offset of (row r, block b) in the tensor-core scale layout whose

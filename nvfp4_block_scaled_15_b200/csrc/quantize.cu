@@ -187,14 +187,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
 // ---------------------------------------------------------------------------
 
 // Stages h = 1, 2, 4, 8 (those below n) on one thread's block.  h = 1 pairs
-// the two halves of a float2; h = 2, 4, 8 pair float2 entries hp = h/2 apart.
-// a - b is computed as a + (-b), which IEEE arithmetic rounds identically.
+// the two halves of a float2 (two scalar operations); h = 2, 4, 8 pair float2
+// entries hp = h/2 apart on the packed units, the difference as
+// fma(b, -1, a), which rounds exactly as a - b.
 __device__ __forceinline__ void fwht_in_thread(float2 (&p)[8], int n) {
   if (n > 1) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      p[i] = __fadd2_rn(make_float2(p[i].x, p[i].x), make_float2(p[i].y, -p[i].y));
+    for (int i = 0; i < 8; ++i) {
+      const float a = p[i].x, b = p[i].y;
+      p[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
   }
+  const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
   for (int hp = 1; hp < 8; hp *= 2) {
     if (n > 2 * hp) {
@@ -203,48 +207,95 @@ __device__ __forceinline__ void fwht_in_thread(float2 (&p)[8], int n) {
         if (i & hp) continue;
         const float2 a = p[i], b = p[i + hp];
         p[i] = __fadd2_rn(a, b);
-        p[i + hp] = __fadd2_rn(a, make_float2(-b.x, -b.y));
+        p[i + hp] = __ffma2_rn(b, m1, a);
       }
     }
   }
 }
 
-// Stages h = 16, 32, ..., n/2 across lanes (lane mask lm = h/16).  The lane
-// holding y_i (bit lm clear) forms y_i + y_{i+h}, its partner y_i - y_{i+h};
-// fma(v, +-1, w) rounds exactly as w +- v.  n is uniform over the warp.
-__device__ __forceinline__ void fwht_cross_lanes(float2 (&p0)[8], float2 (&p1)[8], int n) {
+// Stages h = 16, 32, ... below h_end across lanes (lane mask lm = h/16).  The
+// lane holding y_i (bit lm clear) forms y_i + y_{i+h}, its partner
+// y_i - y_{i+h}; fma(v, +-1, w) rounds exactly as w +- v.  h_end is uniform
+// over the warp.
+__device__ __forceinline__ void fwht_cross_lanes(float2 (&p)[8], int h_end) {
 #pragma unroll
   for (int lm = 1; lm < 32; lm <<= 1) {
-    if (16 * lm < n) {
+    if (16 * lm < h_end) {
       const float sg = (threadIdx.x & lm) ? -1.0f : 1.0f;
       const float2 s2 = make_float2(sg, sg);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float2 o0 = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p0[i].x, lm),
-                                      __shfl_xor_sync(0xFFFFFFFFu, p0[i].y, lm));
-        const float2 o1 = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p1[i].x, lm),
-                                      __shfl_xor_sync(0xFFFFFFFFu, p1[i].y, lm));
-        p0[i] = __ffma2_rn(p0[i], s2, o0);
-        p1[i] = __ffma2_rn(p1[i], s2, o1);
+        const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p[i].x, lm), __shfl_xor_sync(0xFFFFFFFFu, p[i].y, lm));
+        p[i] = __ffma2_rn(p[i], s2, o);
       }
     }
   }
 }
 
-// y = x H for the thread's two blocks (bf16 words in, fp32 out), c = fp32(1/sqrt(n)).
-__device__ __forceinline__ void rotate_two_blocks(const uint32_t (&w0)[8], const uint32_t (&w1)[8], int n, float c,
-                                                  float2 (&p0)[8], float2 (&p1)[8]) {
-  bf16_block_to_f32(w0, p0);
-  bf16_block_to_f32(w1, p1);
-  fwht_in_thread(p0, n);
-  fwht_in_thread(p1, n);
-  fwht_cross_lanes(p0, p1, n);
+// y = x H for one block of the thread (bf16 words in, fp32 out), c = fp32(1/sqrt(n)).
+__device__ __forceinline__ void rotate_block(const uint32_t (&w)[8], int n, float c, float2 (&p)[8]) {
+  bf16_block_to_f32(w, p);
+  fwht_in_thread(p, n);
+  fwht_cross_lanes(p, n);
   const float2 c2 = make_float2(c, c);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    p0[i] = __fmul2_rn(p0[i], c2);
-    p1[i] = __fmul2_rn(p1[i], c2);
+  for (int i = 0; i < 8; ++i) p[i] = __fmul2_rn(p[i], c2);
+}
+
+// Maximum magnitude after the last stage, without forming it: the last
+// stage turns (a, b) into RN(a + b) and RN(a - b), and since rounding to
+// nearest is monotone and odd, max(|RN(a + b)|, |RN(a - b)|) = RN(|a| + |b|).
+// The maxima propagate NaN, so a NaN or an infinity reaches the tensor amax.
+template <int H>
+__device__ __forceinline__ float last_stage_absmax(const float2 (&p)[8]) {
+  float v[8];
+  int j = 0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    if (e & H) continue;
+    const float a = (e & 1) ? p[e >> 1].y : p[e >> 1].x;
+    const float b = ((e + H) & 1) ? p[(e + H) >> 1].y : p[(e + H) >> 1].x;
+    v[j++] = __fadd_rn(fabsf(a), fabsf(b));
   }
+  const float m = max3_nan_f32(v[0], v[1], v[2]);
+  return max3_nan_f32(max3_nan_f32(m, v[3], v[4]), max3_nan_f32(v[5], v[6], v[7]), m);
+}
+
+// max |y / c| over one block of the thread, y = x H: every stage but the last
+// formed, the last one folded into the maximum.  For n > 16 the last stage
+// is across lanes: the lane with bit lm clear takes element positions 0..7
+// of the pair, its partner positions 8..15, so each lane sends 8 values.
+__device__ __forceinline__ float rotated_absmax(const uint32_t (&w)[8], int n) {
+  float2 p[8];
+  bf16_block_to_f32(w, p);
+  if (n <= 16) {
+    fwht_in_thread(p, n >> 1);
+    switch (n) {
+      case 2: return last_stage_absmax<1>(p);
+      case 4: return last_stage_absmax<2>(p);
+      case 8: return last_stage_absmax<4>(p);
+      case 16: return last_stage_absmax<8>(p);
+      default: {                                // n == 1: y = x
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = max3_nan_f32(m, fabsf(p[i].x), fabsf(p[i].y));
+        return m;
+      }
+    }
+  }
+  fwht_in_thread(p, 16);
+  fwht_cross_lanes(p, n >> 1);
+  const int lm = n >> 5;                        // last stage h = n/2
+  const bool upper = (threadIdx.x & lm) != 0;
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 send = upper ? p[i] : p[i + 4];
+    const float2 own = upper ? p[i + 4] : p[i];
+    const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, send.x, lm), __shfl_xor_sync(0xFFFFFFFFu, send.y, lm));
+    m = max3_nan_f32(m, __fadd_rn(fabsf(own.x), fabsf(o.x)), __fadd_rn(fabsf(own.y), fabsf(o.y)));
+  }
+  return m;
 }
 
 template <bool kWide>
@@ -265,9 +316,10 @@ __device__ __forceinline__ void load_two_blocks(const uint16_t* xr, bool ok, int
 }
 
 // Pass 1 of the rotated quantizer: max |y| over the tensor.  grid.x strides
-// over rows, grid.y over segments of 512 blocks.  The maximum runs on the
-// fp32 magnitude bits, so a NaN or an infinity in y reaches the global amax
-// (and the quantize pass reports it) instead of being dropped.
+// over rows, grid.y over segments of 512 blocks.  The maximum of |y / c|
+// propagates NaN (a NaN or an infinity in y reaches the global amax, and the
+// quantize pass reports it); the one multiply by c at the end gives max |y|
+// exactly, since RN(c v) is monotone in v.
 template <bool kWide>
 __global__ void __launch_bounds__(kThreads) hadamard_amax_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                                  int64_t ldx, int n, float c,
@@ -276,30 +328,41 @@ __global__ void __launch_bounds__(kThreads) hadamard_amax_kernel(const uint16_t*
   const int kb = k >> 4;
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
-  uint32_t m = 0;
+  float mf = 0.0f;
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
     uint32_t w0[8], w1[8];
     load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, true, kb, b0, b1, w0, w1);
-    float2 p0[8], p1[8];
-    rotate_two_blocks(w0, w1, n, c, p0, p1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      m = max(m, max(__float_as_uint(p0[i].x) & 0x7FFFFFFFu, __float_as_uint(p0[i].y) & 0x7FFFFFFFu));
-      m = max(m, max(__float_as_uint(p1[i].x) & 0x7FFFFFFFu, __float_as_uint(p1[i].y) & 0x7FFFFFFFu));
-    }
+    mf = max3_nan_f32(mf, rotated_absmax(w0, n), rotated_absmax(w1, n));
   }
-  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  // non-negative floats (NaN as the canonical positive pattern) order as their bits
+  uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mf));
   __shared__ uint32_t red[kThreads / 32];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x < 32) {
     uint32_t t = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0u;
     t = __reduce_max_sync(0xFFFFFFFFu, t);
-    if (threadIdx.x == 0 && t != 0) atomicMax(amax_bits, t);
+    if (threadIdx.x == 0 && t != 0) atomicMax(amax_bits, __float_as_uint(__fmul_rn(__uint_as_float(t), c)));
   }
 }
 
-// Pass 2: rotate again and quantize y (same grid and stores as quantize_kernel).
+// One rotated block: E4M3 scale RN_e4m3(RN(RN(ab * g) / 6)) and 16 codes.
+__device__ __forceinline__ uint2 quantize_rotated_block(const float2 (&p)[8], float g, const float2* table,
+                                                        uint32_t& s8) {
+  const float sixth = __frcp_rn(6.0f);
+  const float t = __fmul_rn(abs_max16_f32(p), g);
+  const float q = __fmul_rn(t, sixth);
+  const float sr = __fmaf_rn(__fmaf_rn(q, -6.0f, t), sixth, q);                // RN(t / 6)
+  uint32_t s2;
+  asm("{\n\t.reg .b16 h;\n\tcvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n\tcvt.u32.u16 %0, h;\n\t}"
+      : "=r"(s2)
+      : "f"(0.0f), "f"(sr));
+  s8 = s2 & 0xFFu;
+  return block_codes_f32(p, g, table[s8 & 0x7Fu]);
+}
+
+// Pass 2: rotate again and quantize y (same grid and stores as quantize_kernel),
+// one block at a time to keep register use low.
 template <bool kTcLayout, bool kWide>
 __global__ void __launch_bounds__(kThreads)
     hadamard_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
@@ -326,11 +389,18 @@ __global__ void __launch_bounds__(kThreads)
   fill_scale_table(table);
   __syncthreads();
 
-  float2 p0[8], p1[8];
-  rotate_two_blocks(w0, w1, n, c, p0, p1);
   uint2 c0, c1;
   uint32_t s0, s1;
-  quantize_two_blocks_f32(p0, p1, g, table, c0, c1, s0, s1);
+  {
+    float2 p[8];
+    rotate_block(w0, n, c, p);
+    c0 = quantize_rotated_block(p, g, table, s0);
+  }
+  {
+    float2 p[8];
+    rotate_block(w1, n, c, p);
+    c1 = quantize_rotated_block(p, g, table, s1);
+  }
   store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
 
