@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--part", choices=["quantize", "hadamard", "gemv", "longk", "gemm", "mxquantize", "mxgemm", "requant"],
+    ap.add_argument("--part", choices=["quantize", "hadamard", "stochastic", "gemv", "longk", "gemm", "mxquantize", "mxgemm", "requant"],
                     default=None,
                     help="run one workload alone, --steps times (for profiling); prints its timing")
     return ap.parse_args()
@@ -476,6 +476,16 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
             "quantize_pass_ms": ms_h1, "quantize_pass_frac_hbm": one_pass / ms_h1 / 1e6 / hbm_peak}
     out["hadamard_quantize_16384x8192"] = had
     del x, q
+    # stochastic rounding of the codes (Philox4x32-10 in the kernel), same input and bytes
+    x = to_dev(pin["quant"])
+    q = nv.empty_quantized(rows, k, nv.SF_TCGEN05, dev)
+    ms_s = _timed(torch, dev, flush, lambda: nv.quantize_stochastic(x, 1234, 0, nv.SF_TCGEN05, out=q), reps)
+    ms_s1 = _timed(torch, dev, flush, lambda: nv.nvfp4_quantize_stochastic(
+        x, rows, k, k, q.codes, q.sf, nv.SF_TCGEN05, q.g, q.amax, 1, 1234, 0), reps)
+    out["stochastic_quantize_16384x8192"] = {
+        "ms": ms_s, "gbs_two_pass": two_pass / ms_s / 1e6, "frac_hbm": two_pass / ms_s / 1e6 / hbm_peak,
+        "quantize_pass_ms": ms_s1, "quantize_pass_frac_hbm": one_pass / ms_s1 / 1e6 / hbm_peak}
+    del x, q
 
     # decode GEMV: W [28672, 8192] pre-quantized, x [M, 8192] quantized in the call
     xg, wg = pin["gemv"]
@@ -574,7 +584,7 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
 def run_part(args):
     """One workload alone: generate its inputs, run it ``--steps`` times with the
     L2 flushed in between, print the median time."""
-    if args.part in ("quantize", "mxquantize", "hadamard"):
+    if args.part in ("quantize", "mxquantize", "hadamard", "stochastic"):
         x_bits = inputs.quantize_bandwidth()
     elif args.part == "gemv":
         xg, wg = inputs.decode_gemv(16)
@@ -601,6 +611,11 @@ def run_part(args):
         for order in (16, 128):
             out[f"ms_order{order}"] = _timed(torch, dev, flush,
                                              lambda: nv.quantize_hadamard(x, order, nv.SF_TCGEN05, out=q), args.steps)
+    elif args.part == "stochastic":
+        x = to_dev(x_bits)
+        q = nv.empty_quantized(*x.shape, nv.SF_TCGEN05, dev)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.quantize_stochastic(x, 1234, 0, nv.SF_TCGEN05, out=q),
+                           args.steps)
     elif args.part == "gemv":
         wq = nv.quantize(to_dev(wg), nv.SF_TCGEN05)
         n, k = wg.shape

@@ -130,6 +130,27 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t 
                             nvfp4_stream_t stream);
 
 /*
+ * NVFP4 quantization with stochastic rounding of the element codes ("FP4"
+ * encyclopedia entry, 技術原理: NVFP4 quantization rounds stochastically
+ * instead of truncating).  amax, the global scale and the E4M3 block scales
+ * are those of nvfp4_quantize (round to nearest even).  Each element's
+ * u = fp32(fp32(x * g) / sd) lies between adjacent E2M1 magnitudes lo <= |u| < hi;
+ * it rounds to hi when R < f * 2^16, f = (|u| - lo) / (hi - lo), with R a 16-bit
+ * random integer, so E[x_hat] = x to within 2^-16 of a grid step; |u| >= 6 gives
+ * 6; the sign bit is kept.  R is drawn in the kernel by Philox4x32-10 (Salmon
+ * et al., "Parallel random numbers: as easy as 1, 2, 3", SC 2011): key =
+ * (seed mod 2^32, seed div 2^32); block b (16 elements) of row r uses the
+ * counters (2b + h, r, offset mod 2^32, offset div 2^32), h = 0, 1, and element
+ * 8h + 2i + m of the block takes bits 16m..16m+15 of output word i.  Equal
+ * (seed, offset) give equal codes; advance `offset` per call for fresh bits.
+ * Arguments, constraints and errors otherwise as nvfp4_quantize.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize_stochastic(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx,
+                                       void* codes, void* sf, nvfp4_sf_layout layout, float* g_dev,
+                                       float* amax_dev, int amax_given, uint64_t seed, uint64_t offset,
+                                       nvfp4_stream_t stream);
+
+/*
  * Hadamard-rotated NVFP4 quantization ("NVIDIA NVFP4 与 Micro-Scaling",
  * section 4.1 旋转/阿达玛变换: x is multiplied by an orthogonal Walsh-Hadamard
  * matrix before quantization, which spreads outlier channels over all

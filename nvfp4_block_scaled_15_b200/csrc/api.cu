@@ -170,6 +170,26 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
   return launch_quantize(x_bf16, rows, k, ldx, codes, sf, layout, g_dev, amax_dev, s);
 }
 
+nvfp4_status nvfp4_quantize_stochastic(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, void* codes,
+                                       void* sf, nvfp4_sf_layout layout, float* g_dev, float* amax_dev,
+                                       int amax_given, uint64_t seed, uint64_t offset, nvfp4_stream_t stream) {
+  nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
+  if (st != NVFP4_OK) return st;
+  if (!codes || !sf || !g_dev || !amax_dev) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
+  if (amax_given != 0 && amax_given != 1) return NVFP4_ERR_INVALID_ARG;
+  if ((k % 16) != 0 || (layout == NVFP4_SF_TCGEN05 && (k % 64) != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(sf) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  if ((st = check_arch()) != NVFP4_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!amax_given) {
+    st = launch_amax(x_bf16, rows, k, ldx, amax_dev, s);
+    if (st != NVFP4_OK) return st;
+  }
+  return launch_quantize_sr(x_bf16, rows, k, ldx, codes, sf, layout, g_dev, amax_dev, seed, offset, s);
+}
+
 nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, int hadamard_order,
                                      void* codes, void* sf, nvfp4_sf_layout layout, float* g_dev, float* amax_dev,
                                      int amax_given, nvfp4_stream_t stream) {

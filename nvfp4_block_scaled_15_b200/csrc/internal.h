@@ -32,6 +32,10 @@ inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s);
 nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
                              nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, cudaStream_t s);
+// Quantize pass with stochastic rounding of the codes (Philox4x32-10 bits).
+nvfp4_status launch_quantize_sr(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                                nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, uint64_t seed,
+                                uint64_t offset, cudaStream_t s);
 // Hadamard-rotated quantizer (order n: a power of two <= 512 dividing k).
 nvfp4_status launch_hadamard_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, int n, float* amax_dev,
                                   cudaStream_t s);

@@ -175,9 +175,9 @@ __device__ __forceinline__ uint2 block_codes(const uint32_t (&w)[8], float g, fl
 
 // Two blocks at once: their E4M3 scales (s = RN_e4m3(RN(RN(amax_b * g) / 6)),
 // satfinite) go through the packed units and one paired conversion.
-__device__ __forceinline__ void quantize_two_blocks(const uint32_t (&w0)[8], const uint32_t (&w1)[8], float g,
-                                                    const float2* table, uint2& c0, uint2& c1, uint32_t& s0,
-                                                    uint32_t& s1) {
+// E4M3 scale bytes of two bf16 blocks: RN_e4m3(RN(RN(amax_b * g) / 6)), satfinite.
+__device__ __forceinline__ void two_block_scales(const uint32_t (&w0)[8], const uint32_t (&w1)[8], float g,
+                                                 uint32_t& s0, uint32_t& s1) {
   const float sixth = __frcp_rn(6.0f);
   const float2 ab = make_float2(__uint_as_float(abs_max_bits16(w0) << 16), __uint_as_float(abs_max_bits16(w1) << 16));
   const float2 t = __fmul2_rn(ab, make_float2(g, g));
@@ -190,8 +190,76 @@ __device__ __forceinline__ void quantize_two_blocks(const uint32_t (&w0)[8], con
       : "f"(sr.y), "f"(sr.x));
   s0 = s2 & 0xFFu;
   s1 = (s2 >> 8) & 0xFFu;
+}
+
+__device__ __forceinline__ void quantize_two_blocks(const uint32_t (&w0)[8], const uint32_t (&w1)[8], float g,
+                                                    const float2* table, uint2& c0, uint2& c1, uint32_t& s0,
+                                                    uint32_t& s1) {
+  two_block_scales(w0, w1, g, s0, s1);
   c0 = block_codes(w0, g, table[s0 & 0x7Fu]);
   c1 = block_codes(w1, g, table[s1 & 0x7Fu]);
+}
+
+// ---------------------------------------------------------------------------
+// Stochastic rounding ("FP4" encyclopedia entry, 技術原理: NVFP4 quantization
+// rounds stochastically instead of truncating).
+// ---------------------------------------------------------------------------
+
+// Philox4x32 with 10 rounds (J. Salmon, M. Moraes, R. Dror, D. Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC 2011): each round maps
+// (c0, c1, c2, c3) to (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1,
+// lo(M0 c0)), and the key grows by the Weyl increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Stochastic rounding of u onto the E2M1 grid with the 16-bit random integer
+// r: the magnitude a lies between neighbours lo and hi = lo + step (step 0.5
+// below 2, 1 below 4, 2 below 6); it rounds up when r < f * 2^16, f = (a - lo)
+// / step; a >= 6 gives 6; the sign of u is kept.  Every step is exact in fp32:
+// v = a / step is a power-of-two scaling, floor(v) and v - floor(v) are exact,
+// and f * 2^16 and r are exact, so the comparison is the real one.
+__device__ __forceinline__ float e2m1_round_stochastic(float u, uint32_t r) {
+  const float a = fabsf(u);
+  const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+  const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+  const float v = a * inv_step;
+  const float fl = floorf(v);
+  const bool up = static_cast<float>(r) < (v - fl) * 65536.0f;
+  float m = (up ? fl + 1.0f : fl) * step;
+  if (a >= 6.0f) m = 6.0f;
+  return copysignf(m, u);
+}
+
+// 16 codes of one bf16 block for the scale entry e = {sd, RN(1/sd)} with
+// stochastic rounding: u = RN(RN(x * g) / sd) as in block_codes, then element
+// 8h + 2i + m takes bits 16m.. of word i of ra (h = 0) or rb (h = 1).  The
+// rounded values are E2M1 grid points, which the conversion keeps exactly.
+__device__ __forceinline__ uint2 block_codes_sr(const uint32_t (&w)[8], float g, float2 e, uint4 ra, uint4 rb) {
+  const float2 ng2 = make_float2(-g, -g);
+  const float2 nyr2 = make_float2(-e.y, -e.y);
+  const float2 sd2 = make_float2(e.x, e.x);
+  const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+  float2 u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 tn = __fmul2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), ng2);  // -(x * g)
+    const float2 q = __fmul2_rn(tn, nyr2);
+    const float2 rr = __ffma2_rn(q, sd2, tn);
+    const float2 d = __ffma2_rn(rr, nyr2, q);                                   // RN(t / sd)
+    u[i] = make_float2(e2m1_round_stochastic(d.x, rw[i] & 0xFFFFu), e2m1_round_stochastic(d.y, rw[i] >> 16));
+  }
+  uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
+  if (e.x == 0.0f) c = make_uint2(0u, 0u);
+  return c;
 }
 
 // ---------------------------------------------------------------------------

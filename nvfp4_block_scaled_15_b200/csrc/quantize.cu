@@ -168,6 +168,61 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
 
+// Pass 2 with stochastic rounding of the element codes: the same grid,
+// scales and stores as quantize_kernel; the random integers of block b of row
+// r come from Philox4x32-10 with key (seed_lo, seed_hi) and counters
+// (2b + h, r, offset_lo, offset_hi), h = 0, 1.
+template <bool kTcLayout, bool kWide>
+__global__ void __launch_bounds__(kThreads)
+    quantize_sr_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, uint8_t* __restrict__ codes,
+                       uint8_t* __restrict__ sf, float* __restrict__ g_out, const float* __restrict__ amax_in,
+                       uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo, uint32_t off_hi,
+                       int* __restrict__ status) {
+  __shared__ float2 table[128];
+  const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
+  const int kb = k >> 4;
+  const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
+  const int b1 = b0 + kThreads;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  bool valid;
+  float g = global_scale_from_amax(*amax_in, valid);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    *g_out = valid ? g : 0.0f;
+    if (!valid) record_status(status, kDevRange);
+  }
+  if (!valid) g = 0.0f;
+  const bool real_row = r < rows;
+
+  uint32_t w0[8], w1[8];
+  const uint16_t* xr = x + static_cast<int64_t>(r) * ldx;
+  if (real_row && valid && b0 < kb) {
+    load_block<kWide>(xr + b0 * 16, w0);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w0[i] = 0u;
+  }
+  if (real_row && valid && b1 < kb) {
+    load_block<kWide>(xr + b1 * 16, w1);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w1[i] = 0u;
+  }
+  fill_scale_table(table);
+  __syncthreads();
+
+  uint32_t s0, s1;
+  two_block_scales(w0, w1, g, s0, s1);
+  const uint32_t ur = static_cast<uint32_t>(r);
+  const uint2 c0 = block_codes_sr(w0, g, table[s0 & 0x7Fu],
+                                  philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi),
+                                  philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi));
+  const uint2 c1 = block_codes_sr(w1, g, table[s1 & 0x7Fu],
+                                  philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi),
+                                  philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi));
+  store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
+}
+
 // ---------------------------------------------------------------------------
 // Hadamard-rotated NVFP4 ("NVIDIA NVFP4 与 Micro-Scaling", section 4.1: the
 // activations are multiplied by an orthogonal Walsh-Hadamard matrix before
@@ -542,6 +597,24 @@ cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16
                             amax_dev, status);
 }
 
+template <bool kTc, bool kWide>
+cudaError_t launch_quantize_sr_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
+                                   uint8_t* codes, uint8_t* sf, float* g_dev, const float* amax_dev, uint64_t seed,
+                                   uint64_t offset, int* status) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_sr_kernel<kTc, kWide>, x, rows, k, ldx, codes, sf, g_dev, amax_dev,
+                            static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
+                            static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32), status);
+}
+
 // fp32(1/sqrt(n)) for the transform's order n (a power of two): the double
 // quotient of the correctly rounded double square root, rounded to fp32.
 float hadamard_norm(int n) { return static_cast<float>(1.0 / std::sqrt(static_cast<double>(n))); }
@@ -662,6 +735,36 @@ nvfp4_status launch_hadamard_quantize(const void* x, int64_t rows, int64_t k, in
                                                          status)
              : launch_hadamard_quantize_pdl<false, false>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
                                                           status);
+  return launch_status(e);
+}
+
+nvfp4_status launch_quantize_sr(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
+                                nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, uint64_t seed,
+                                uint64_t offset, cudaStream_t s) {
+  int* status = device_status_ptr();
+  if (!status) return NVFP4_ERR_CUDA;
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  uint8_t* cs = static_cast<uint8_t*>(codes);
+  uint8_t* ss = static_cast<uint8_t*>(sf);
+  const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
+  const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
+  const int ir = static_cast<int>(rows), ik = static_cast<int>(k);
+  if (grid_rows == 0 || segs == 0)
+    return launch_status(launch_quantize_sr_pdl<false, false>(dim3(1, 1), s, xs, 0, 0, ldx, cs, ss, g_dev, amax_dev,
+                                                              seed, offset, status));
+  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  cudaError_t e;
+  if (layout == NVFP4_SF_TCGEN05)
+    e = wide ? launch_quantize_sr_pdl<true, true>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, seed, offset,
+                                                  status)
+             : launch_quantize_sr_pdl<true, false>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, seed, offset,
+                                                   status);
+  else
+    e = wide ? launch_quantize_sr_pdl<false, true>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, seed, offset,
+                                                   status)
+             : launch_quantize_sr_pdl<false, false>(grid, s, xs, ir, ik, ldx, cs, ss, g_dev, amax_dev, seed, offset,
+                                                    status);
   return launch_status(e);
 }
 

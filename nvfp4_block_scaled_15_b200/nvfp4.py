@@ -45,6 +45,8 @@ _SIGS = {
     "nvfp4_sf_bytes": ([_i64, _i64, _i32], _sz),
     "nvfp4_amax": ([_vp, _i64, _i64, _i64, _vp, _vp], _i32),
     "nvfp4_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _vp], _i32),
+    "nvfp4_quantize_stochastic": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _u64, _u64, _vp],
+                                  _i32),
     "nvfp4_quantize_hadamard": ([_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp], _i32),
     "nvfp4_swizzle_sf": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "nvfp4_gemm": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp], _i32),
@@ -124,6 +126,13 @@ def nvfp4_amax(x, rows, k, ldx, amax_dev, stream=None) -> None:
 def nvfp4_quantize(x, rows, k, ldx, codes, sf, layout, g_dev, amax_dev, amax_given=0, stream=None) -> None:
     _check(_lib.nvfp4_quantize(_p(x), rows, k, ldx, _p(codes), _p(sf), layout, _p(g_dev), _p(amax_dev),
                                int(amax_given), _s(stream)), "nvfp4_quantize")
+
+
+def nvfp4_quantize_stochastic(x, rows, k, ldx, codes, sf, layout, g_dev, amax_dev, amax_given, seed, offset,
+                              stream=None) -> None:
+    _check(_lib.nvfp4_quantize_stochastic(_p(x), rows, k, ldx, _p(codes), _p(sf), layout, _p(g_dev), _p(amax_dev),
+                                          int(amax_given), int(seed), int(offset), _s(stream)),
+           "nvfp4_quantize_stochastic")
 
 
 def nvfp4_quantize_hadamard(x, rows, k, ldx, order, codes, sf, layout, g_dev, amax_dev, amax_given=0,
@@ -231,6 +240,19 @@ def quantize(x: torch.Tensor, layout: int = SF_TCGEN05, out: Quantized | None = 
         q.amax.copy_(amax)
     nvfp4_quantize(x, rows, k, x.stride(0), q.codes, q.sf, layout, q.g, q.amax, 1 if amax is not None else 0,
                    stream)
+    return q
+
+
+def quantize_stochastic(x: torch.Tensor, seed: int, offset: int, layout: int = SF_TCGEN05,
+                        out: Quantized | None = None, amax=None, stream=None) -> Quantized:
+    """bf16 [rows, k] -> NVFP4 with stochastically rounded codes (Philox4x32-10 bits from seed, offset)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    q = out if out is not None else empty_quantized(rows, k, layout, x.device)
+    if amax is not None:
+        q.amax.copy_(amax)
+    nvfp4_quantize_stochastic(x, rows, k, x.stride(0), q.codes, q.sf, layout, q.g, q.amax,
+                              1 if amax is not None else 0, seed, offset, stream)
     return q
 
 

@@ -64,12 +64,14 @@ def philox4x32_10(counter, key) -> np.ndarray:
     return np.stack([c0, c1, c2, c3], axis=-1).astype(np.uint32)
 
 
-def random16(rows: int, k: int, seed: int, offset: int) -> np.ndarray:
-    """The 16-bit random integers R [rows, k] of definition step 5."""
+def random16(rows: int, k: int, seed: int, offset: int, row_ids=None) -> np.ndarray:
+    """The 16-bit random integers R [rows, k] of definition step 5 (for the
+    tensor rows ``row_ids`` when given, else rows 0 .. rows-1)."""
     if k % NV.BLOCK:
         raise ValueError("K must be a multiple of 16")
     kb = k // NV.BLOCK
-    r = np.arange(rows, dtype=np.uint64)[:, None, None]
+    ids = np.arange(rows) if row_ids is None else np.asarray(row_ids)
+    r = ids.astype(np.uint64)[:, None, None]
     b = np.arange(kb, dtype=np.uint64)[None, :, None]
     h = np.arange(2, dtype=np.uint64)[None, None, :]
     ctr = np.empty((rows, kb, 2, 4), dtype=np.uint64)
@@ -98,8 +100,10 @@ def e2m1_encode_sr(u, r16) -> np.ndarray:
     return code | np.where(np.signbit(u), np.uint8(8), np.uint8(0))
 
 
-def quantize_sr(x_bits, seed: int, offset: int, amax_value=None):
-    """bf16 [rows, K] -> (packed codes [rows, K/2], row-major scales [rows, K/16], g, amax)."""
+def quantize_sr(x_bits, seed: int, offset: int, amax_value=None, row_ids=None):
+    """bf16 [rows, K] -> (packed codes [rows, K/2], row-major scales [rows, K/16], g, amax).
+    ``row_ids``: the tensor rows x_bits holds (a sample of a larger tensor, whose
+    amax is then given), which select the random integers."""
     x = NV.bf16_to_f32(x_bits)
     rows, k = x.shape
     a = NV.amax(x_bits) if amax_value is None else np.float32(amax_value)
@@ -113,7 +117,7 @@ def quantize_sr(x_bits, seed: int, offset: int, amax_value=None):
     zero = (sd == 0)[:, :, None]
     with np.errstate(divide="ignore", invalid="ignore"):
         u = np.where(zero, np.float32(0.0), t / np.where(zero, np.float32(1.0), sd[:, :, None])).astype(np.float32)
-    r16 = random16(rows, k, seed, offset).reshape(rows, k // NV.BLOCK, NV.BLOCK)
+    r16 = random16(rows, k, seed, offset, row_ids).reshape(rows, k // NV.BLOCK, NV.BLOCK)
     codes = e2m1_encode_sr(u, r16)
     codes = np.where(np.broadcast_to(zero, codes.shape), np.uint8(0), codes)
     return NV.pack_codes(codes.reshape(rows, k)), sf.astype(np.uint8), g, a

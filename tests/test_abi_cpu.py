@@ -83,6 +83,10 @@ def test_argument_errors_return_before_any_device_work(nv):
     assert raw("nvfp4_gemv_batched", fake, 4, 64, fake, fake, fake, 128, 64, fake, 128, fake, 16, None) == nv.ERR_WORKSPACE
     assert raw("nvfp4_gemm_quant_a", fake, 64, fake, fake, fake, 8, 8, 64, fake, 8, 0, fake, 16, None) == nv.ERR_WORKSPACE
     assert raw("nvfp4_swizzle_sf", fake, 4, 48, fake, None) == nv.ERR_UNSUPPORTED_SHAPE
+    qs = "nvfp4_quantize_stochastic"
+    assert raw(qs, fake, 4, 48, 48, fake, fake, 1, fake, fake, 0, 1, 2, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert raw(qs, fake, 4, 64, 64, fake, fake, 1, fake, fake, 2, 1, 2, None) == nv.ERR_INVALID_ARG
+    assert raw(qs, fake, 4, 64, 64, None, fake, 1, fake, fake, 0, 1, 2, None) == nv.ERR_INVALID_ARG
     # Hadamard order: a power of two in [1, 512] that divides k
     qh = "nvfp4_quantize_hadamard"
     for order in (0, 3, 1024, -16):
