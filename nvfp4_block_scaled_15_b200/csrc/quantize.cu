@@ -83,6 +83,24 @@ __device__ __forceinline__ void load_block(const uint16_t* p, uint32_t (&w)[8]) 
   }
 }
 
+// The thread's two blocks of row xr (zeros where ok is false or the block is past kb).
+template <bool kWide>
+__device__ __forceinline__ void load_two_blocks(const uint16_t* xr, bool ok, int kb, int b0, int b1,
+                                                uint32_t (&w0)[8], uint32_t (&w1)[8]) {
+  if (ok && b0 < kb) {
+    load_block<kWide>(xr + b0 * 16, w0);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w0[i] = 0u;
+  }
+  if (ok && b1 < kb) {
+    load_block<kWide>(xr + b1 * 16, w1);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w1[i] = 0u;
+  }
+}
+
 // Stores of one thread's two blocks (codes c0, c1 and scale bytes s0, s1 of
 // blocks b0, b1 of row r): codes row-major [rows, k/2], scales row-major or
 // in the tensor-core layout (where rows >= `rows` exist and get zero scales).
@@ -132,39 +150,33 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
 
-  // Launched as a programmatic dependent of the amax pass: everything before
-  // this point overlaps its tail; the amax (and x) are read only after it.
+  const bool real_row = r < rows;
+
+  // Launched as a programmatic dependent of the amax pass.  x is not written
+  // by that pass, so its loads and the scale table go out before the wait and
+  // overlap the pass's tail; only the amax is read after it, and every store
+  // comes after it.  (The kernels that release dependents early are the amax
+  // passes and the GEMV prologue, none of which writes x; the amax pass itself
+  // starts only after all earlier work on the stream has finished.)
+  uint32_t w0[8], w1[8];
+  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row, kb, b0, b1, w0, w1);
+  fill_scale_table(table);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
-  float g = global_scale_from_amax(*amax_in, valid);
+  const float g = global_scale_from_amax(*amax_in, valid);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     *g_out = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
-  if (!valid) g = 0.0f;                        // all-zero codes and scales
-  const bool real_row = r < rows;
-
-  uint32_t w0[8], w1[8];
-  const uint16_t* xr = x + static_cast<int64_t>(r) * ldx;
-  if (real_row && valid && b0 < kb) {
-    load_block<kWide>(xr + b0 * 16, w0);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w0[i] = 0u;
-  }
-  if (real_row && valid && b1 < kb) {
-    load_block<kWide>(xr + b1 * 16, w1);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w1[i] = 0u;
-  }
-  fill_scale_table(table);                    // overlaps the loads in flight
   __syncthreads();
 
   uint2 c0, c1;
   uint32_t s0, s1;
   quantize_two_blocks(w0, w1, g, table, c0, c1, s0, s1);
-
+  if (!valid) {                                // all-zero codes and scales
+    c0 = c1 = make_uint2(0u, 0u);
+    s0 = s1 = 0u;
+  }
   store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
 
@@ -184,6 +196,11 @@ __global__ void __launch_bounds__(kThreads)
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
 
+  const bool real_row = r < rows;
+
+  uint32_t w0[8], w1[8];                       // x and the table before the wait, as in quantize_kernel
+  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row, kb, b0, b1, w0, w1);
+  fill_scale_table(table);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
   float g = global_scale_from_amax(*amax_in, valid);
@@ -191,24 +208,11 @@ __global__ void __launch_bounds__(kThreads)
     *g_out = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
-  if (!valid) g = 0.0f;
-  const bool real_row = r < rows;
-
-  uint32_t w0[8], w1[8];
-  const uint16_t* xr = x + static_cast<int64_t>(r) * ldx;
-  if (real_row && valid && b0 < kb) {
-    load_block<kWide>(xr + b0 * 16, w0);
-  } else {
+  if (!valid) {                                // all-zero codes and scales
+    g = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w0[i] = 0u;
+    for (int i = 0; i < 8; ++i) w0[i] = w1[i] = 0u;
   }
-  if (real_row && valid && b1 < kb) {
-    load_block<kWide>(xr + b1 * 16, w1);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w1[i] = 0u;
-  }
-  fill_scale_table(table);
   __syncthreads();
 
   uint32_t s0, s1;
@@ -353,23 +357,6 @@ __device__ __forceinline__ float rotated_absmax(const uint32_t (&w)[8], int n) {
   return m;
 }
 
-template <bool kWide>
-__device__ __forceinline__ void load_two_blocks(const uint16_t* xr, bool ok, int kb, int b0, int b1,
-                                                uint32_t (&w0)[8], uint32_t (&w1)[8]) {
-  if (ok && b0 < kb) {
-    load_block<kWide>(xr + b0 * 16, w0);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w0[i] = 0u;
-  }
-  if (ok && b1 < kb) {
-    load_block<kWide>(xr + b1 * 16, w1);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w1[i] = 0u;
-  }
-}
-
 // Pass 1 of the rotated quantizer: max |y| over the tensor.  grid.x strides
 // over rows, grid.y over segments of 512 blocks.  The maximum of |y / c|
 // propagates NaN (a NaN or an infinity in y reaches the global amax, and the
@@ -429,6 +416,11 @@ __global__ void __launch_bounds__(kThreads)
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
 
+  const bool real_row = r < rows;
+
+  uint32_t w0[8], w1[8];                       // x and the table before the wait, as in quantize_kernel
+  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row, kb, b0, b1, w0, w1);
+  fill_scale_table(table);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
   float g = global_scale_from_amax(*amax_in, valid);
@@ -436,12 +428,11 @@ __global__ void __launch_bounds__(kThreads)
     *g_out = valid ? g : 0.0f;
     if (!valid) record_status(status, kDevRange);
   }
-  if (!valid) g = 0.0f;
-  const bool real_row = r < rows;
-
-  uint32_t w0[8], w1[8];
-  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row && valid, kb, b0, b1, w0, w1);
-  fill_scale_table(table);
+  if (!valid) {                                // all-zero codes and scales
+    g = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w0[i] = w1[i] = 0u;
+  }
   __syncthreads();
 
   uint2 c0, c1;
