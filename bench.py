@@ -10,8 +10,9 @@ over the device time of the step, summed over ranks (weak scaling: every
 rank runs its own replica; the path needs no exchange).
 
 Also reported on rank 0: the GEMM kernel's roofline (live CUDA events),
-end-to-end throughput through host buffers, the quantize-bandwidth,
-decode-GEMV and long-K workloads, SM clocks during the timed region, and
+end-to-end throughput through host buffers and SM clocks during the timed
+region; at N = 1 also the quantize-bandwidth, rotated and stochastic
+quantize, decode-GEMV, long-K, MXFP4 and requantizing-GEMM workloads, and
 the CPU oracle timed on a bounded sample of the same workload.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -202,6 +203,22 @@ def time_oracle(sample: OracleSample, reps: int = 1):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank timing (one process per GPU; replicas, no data-path collective)
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's step time: every rank contributes its own mean."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs one prefill step per step time."""
+    return world * FLOPS_STEP / (ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the oracle, timed on the host cores
 # ---------------------------------------------------------------------------
 def run_reference(args, rank):
@@ -258,7 +275,9 @@ def main():
     # host inputs first (the generator's process pool starts before CUDA)
     a_bits, w_bits = inputs.prefill_gemm()
     parts_inputs = None
-    if rank == 0 and not args.no_parts:
+    # the single-GPU workloads run at N = 1 only: with N > 1 the other ranks
+    # would sit in the closing barrier for their whole duration
+    if rank == 0 and world == 1 and not args.no_parts:
         parts_inputs = {"quant": inputs.quantize_bandwidth(),
                         "gemv": inputs.decode_gemv(16),
                         "longk": inputs.long_k()}
@@ -322,10 +341,8 @@ def main():
     gemm_ms = [e1.elapsed_time(e2) for e0, e1, e2 in ev]
     ms = statistics.mean(step_ms)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * FLOPS_STEP / (ms * 1e-3) / 1e12
+        ms = max_over_ranks(ms, dist, dev)
+    value = job_value(world, ms)
 
     # end to end through the public API with pinned host buffers
     e2e = None
