@@ -538,7 +538,25 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
         torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1) / calls
         algo = n * k // 2 + n * k // 16 + m * k * 2 + m * n * 2
-        thr[f"M={m}"] = {"ms_per_call": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak}
+        # the same 30 calls captured once in a CUDA graph and replayed (how a
+        # decode step issues its layers), so no per-launch host work sits between them
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(calls):
+                nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        stream = torch.cuda.current_stream(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        graph.replay()
+        graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_g = g0.elapsed_time(g1) / (2 * calls)
+        del graph
+        thr[f"M={m}"] = {"ms_per_call": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak,
+                         "graph_ms_per_call": ms_g, "graph_frac_hbm": algo / ms_g / 1e6 / hbm_peak}
     out["gemv_28672x8192_back_to_back"] = thr
     del wq, wqs
 
