@@ -122,6 +122,8 @@ NVFP4_API nvfp4_status nvfp4_amax(const void* x_bf16, int64_t rows, int64_t k, i
  *           computes the tensor amax into it (two passes over x).
  *           amax_given == 1: in, the callee uses *amax_dev as the amax (one pass).
  * k % 16 == 0 for NVFP4_SF_ROWMAJOR, k % 64 == 0 for NVFP4_SF_TCGEN05.
+ * An empty tensor (rows == 0 or k == 0) is valid: x, codes and sf may then be
+ * null; the amax is 0 and *g_dev is 1.
  * If 2688/amax is not finite, codes and scales are written as 0, *g_dev as 0,
  * and the device status records NVFP4_ERR_RANGE.
  */

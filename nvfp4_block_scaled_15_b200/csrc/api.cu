@@ -104,9 +104,13 @@ using namespace nvfp4;
 
 namespace {
 
+// An empty tensor (rows == 0 or k == 0) is read nowhere: its pointer may be
+// null and its pitch is not checked.
 nvfp4_status check_bf16_input(const void* x, int64_t rows, int64_t k, int64_t ld) {
-  if (!x || rows < 0 || k < 0 || ld < k) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned16(x) || (ld % 8) != 0) return NVFP4_ERR_MISALIGNED;
+  if (rows < 0 || k < 0 || ld < k) return NVFP4_ERR_INVALID_ARG;
+  const bool empty = rows == 0 || k == 0;
+  if (!x && !empty) return NVFP4_ERR_INVALID_ARG;
+  if (!empty && (!aligned16(x) || (ld % 8) != 0)) return NVFP4_ERR_MISALIGNED;
   if (rows > 0x7FFFFFFF || k > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   return NVFP4_OK;
 }
@@ -155,7 +159,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
                             nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
   if (st != NVFP4_OK) return st;
-  if (!codes || !sf || !g_dev || !amax_dev) return NVFP4_ERR_INVALID_ARG;
+  if (!g_dev || !amax_dev || ((!codes || !sf) && rows > 0 && k > 0)) return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
   if (amax_given != 0 && amax_given != 1) return NVFP4_ERR_INVALID_ARG;
   if ((k % 16) != 0 || (layout == NVFP4_SF_TCGEN05 && (k % 64) != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -175,7 +179,7 @@ nvfp4_status nvfp4_quantize_stochastic(const void* x_bf16, int64_t rows, int64_t
                                        int amax_given, uint64_t seed, uint64_t offset, nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
   if (st != NVFP4_OK) return st;
-  if (!codes || !sf || !g_dev || !amax_dev) return NVFP4_ERR_INVALID_ARG;
+  if (!g_dev || !amax_dev || ((!codes || !sf) && rows > 0 && k > 0)) return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
   if (amax_given != 0 && amax_given != 1) return NVFP4_ERR_INVALID_ARG;
   if ((k % 16) != 0 || (layout == NVFP4_SF_TCGEN05 && (k % 64) != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -195,7 +199,7 @@ nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows, int64_t k
                                      int amax_given, nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
   if (st != NVFP4_OK) return st;
-  if (!codes || !sf || !g_dev || !amax_dev) return NVFP4_ERR_INVALID_ARG;
+  if (!g_dev || !amax_dev || ((!codes || !sf) && rows > 0 && k > 0)) return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
   if (amax_given != 0 && amax_given != 1) return NVFP4_ERR_INVALID_ARG;
   const int n = hadamard_order;
@@ -225,7 +229,7 @@ nvfp4_status nvfp4_mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t k, i
                                   nvfp4_sf_layout layout, nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
   if (st != NVFP4_OK) return st;
-  if (!codes || !sf) return NVFP4_ERR_INVALID_ARG;
+  if ((!codes || !sf) && rows > 0 && k > 0) return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
   if ((k % 32) != 0 || (layout == NVFP4_SF_TCGEN05 && (k % 128) != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(codes)) return NVFP4_ERR_MISALIGNED;

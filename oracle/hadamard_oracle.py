@@ -59,7 +59,10 @@ def fwht_f32(x, b: int) -> np.ndarray:
 def quantize_hadamard(x_bits, b: int, amax_value=None):
     """bf16 [rows, C] -> rotated NVFP4: (packed codes, row-major scales, g, amax of y)."""
     y = fwht_f32(NV.bf16_to_f32(x_bits), b)
-    a = np.float32(np.max(np.abs(y))) if amax_value is None else np.float32(amax_value)
+    if amax_value is not None:
+        a = np.float32(amax_value)
+    else:                                   # an empty tensor has amax 0, so g = 1
+        a = np.float32(np.max(np.abs(y))) if y.size else np.float32(0.0)
     g = NV.global_scale(a)
     codes, sf = NV.quantize_values_with_scale(y, g)
     return NV.pack_codes(codes), sf, g, a

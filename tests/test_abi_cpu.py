@@ -104,3 +104,8 @@ def test_no_device_means_cuda_or_arch_error(nv):
     fake = 1 << 20
     st = nv.raw_status("nvfp4_quantize", fake, 4, 64, 64, fake, fake, 1, fake, fake, 0, None)
     assert st in (nv.ERR_CUDA, nv.ERR_ARCH)
+    # an empty tensor may come with null pointers: the arguments pass, the device check stops it
+    for rows, k in [(0, 64), (4, 0)]:
+        st = nv.raw_status("nvfp4_quantize", None, rows, k, 64, None, None, 1, fake, fake, 0, None)
+        assert st in (nv.ERR_CUDA, nv.ERR_ARCH)
+    assert nv.raw_status("nvfp4_quantize", None, 4, 64, 64, None, None, 1, fake, fake, 0, None) == nv.ERR_INVALID_ARG
