@@ -1,10 +1,12 @@
-// NVFP4 block quantization on a pair of lanes ("low-precision-floats",
+// NVFP4 block quantization steps shared by the quantize passes, the GEMV
+// prologue and the rotated and stochastic quantizers ("low-precision-floats",
 // section FP4 / MXFP4 / NVFP4: s_block = (block_amax / 6) / s_global and
 // x_hat = s_global * s_block * Q_E2M1(x / (s_global * s_block)), with the
 // encode scale g = 1 / s_global = 2688 / amax).
 //
-// Two adjacent lanes (2i, 2i+1) hold the two halves (8 bf16 each) of one
-// 16-element block; a single shuffle gives both the block amax.
+// One lane owns whole 16-element blocks, so a block's amax needs no shuffle.
+// Every fp32 step is the correctly rounded IEEE operation the CPU definition
+// states (divisions through Markstein's FMA correction).
 #pragma once
 #include <cstdint>
 #include <cuda_fp8.h>
@@ -34,18 +36,6 @@ __device__ __forceinline__ uint32_t abs_max_bits8(const uint4 v) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Two fp32 values -> one byte of two E2M1 codes (RNE, saturating): lo goes to
-// bits 0..3, hi to bits 4..7.
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(out)
-      : "f"(hi), "f"(lo));
-  return out;
-}
-
 // Eight fp32 values (element 2i in a[i].x, 2i+1 in a[i].y) -> 32 bits of
 // E2M1 codes, element 0 in bits 0..3.
 __device__ __forceinline__ uint32_t e2m1x8(float2 a0, float2 a1, float2 a2, float2 a3) {
@@ -61,24 +51,6 @@ __device__ __forceinline__ uint32_t e2m1x8(float2 a0, float2 a1, float2 a2, floa
   return out;
 }
 
-// Per-lane table for exact reciprocals of E4M3 scales: lane k (0 < k < 16)
-// holds RN(1/k).  An E4M3 value is k * 2^-s with k its integer significand
-// (8..15 for normals, 1..7 for subnormals), so RN(1/sd) = RN(1/k) * 2^s
-// exactly (scaling by a power of two does not change the rounding).
-__device__ __forceinline__ float recip_table_lane() {
-  const int k = static_cast<int>(threadIdx.x & 15);
-  return k == 0 ? 0.0f : __frcp_rn(static_cast<float>(k));
-}
-
-__device__ __forceinline__ float e4m3_recip_rn(uint32_t s8, float table_lane) {
-  const uint32_t e = (s8 >> 3) & 15u;
-  const uint32_t m = s8 & 7u;
-  const int k = e ? static_cast<int>(8u + m) : static_cast<int>(m);
-  const int sh = e ? 10 - static_cast<int>(e) : 9;           // sd = k * 2^-sh
-  const float rk = __shfl_sync(0xFFFFFFFFu, table_lane, k);
-  return __int_as_float(__float_as_int(rk) + (sh << 23));
-}
-
 // RN(t / d) given y = RN(1 / d): q = RN(t * y); r = t - q * d is exact with
 // one FMA; RN(q + r * y) equals RN(t / d) (Markstein's theorem on FMA-based
 // division, P. Markstein, "Computation of elementary functions on the IBM
@@ -88,40 +60,6 @@ __device__ __forceinline__ float div_rn_by_recip(float t, float d, float y) {
   const float q = __fmul_rn(t, y);
   const float r = __fmaf_rn(-q, d, t);
   return copysignf(__fmaf_rn(r, y, q), t);
-}
-
-// One half block: 8 bf16 in v.  Returns the 4 code bytes (element 0 in the
-// low nibble of byte 0) and, through sf, the block's E4M3 scale byte.  Every
-// lane of the warp must call this (it shuffles across the warp).  `sixth` is
-// RN(1/6) and `table_lane` this lane's recip_table_lane().
-// Pairs of elements go through the packed fp32x2 units; each lane of a
-// packed operation rounds exactly like its scalar counterpart.
-__device__ __forceinline__ uint32_t quantize_half_block(const uint4 v, const float g, uint32_t& sf, float sixth,
-                                                        float table_lane) {
-  uint32_t amax_bits = abs_max_bits8(v);
-  amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, 1));
-  const float ab = __uint_as_float(amax_bits << 16);
-  const float s_raw = div_rn_by_recip(__fmul_rn(ab, g), 6.0f, sixth);
-  const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(s_raw, __NV_SATFINITE, __NV_E4M3);
-  sf = static_cast<uint32_t>(s8);
-  const __half_raw hs = __nv_cvt_fp8_to_halfraw(s8, __NV_E4M3);
-  const float sd = __half2float(__half(hs));
-  const float y = e4m3_recip_rn(sf, table_lane);            // shuffles: every lane
-  if (sd == 0.0f) return 0u;
-  const float2 g2 = make_float2(g, g);
-  const float2 y2 = make_float2(y, y);
-  const float2 nsd2 = make_float2(-sd, -sd);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float2 u[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __fmul2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), g2);   // x * g
-    const float2 q = __fmul2_rn(t, y2);                                         // RN(t * RN(1/sd))
-    const float2 r = __ffma2_rn(q, nsd2, t);                                    // t - q * sd, exact
-    const float2 d = __ffma2_rn(r, y2, q);                                      // RN(t / sd)
-    u[i] = make_float2(copysignf(d.x, t.x), copysignf(d.y, t.y));
-  }
-  return e2m1x8(u[0], u[1], u[2], u[3]);
 }
 
 // ---------------------------------------------------------------------------
