@@ -25,11 +25,16 @@ Definition (readings marked):
      then y = fp32(y * c_b), c_b = fp32(1 / sqrt(b)) [reading: the rounding
      of the transform is fixed by this order, which the kernel follows];
   3. y is quantized to NVFP4 like any fp32 tensor (steps 1-5 of
-     nvfp4_oracle, the amax taken over y).
+     nvfp4_oracle, the amax taken over y);
+  4. with stochastic rounding ("FP4" encyclopedia entry, 技術原理, names the
+     rotation and stochastic rounding together): step 3 with the element
+     rounding of stochastic_oracle, its random integers indexed by the
+     position in y.
 """
 import numpy as np
 
 from oracle import nvfp4_oracle as NV
+from oracle import stochastic_oracle as SR
 
 
 def norm_constant(b: int) -> np.float32:
@@ -65,4 +70,17 @@ def quantize_hadamard(x_bits, b: int, amax_value=None):
         a = np.float32(np.max(np.abs(y))) if y.size else np.float32(0.0)
     g = NV.global_scale(a)
     codes, sf = NV.quantize_values_with_scale(y, g)
+    return NV.pack_codes(codes), sf, g, a
+
+
+def quantize_hadamard_sr(x_bits, b: int, seed: int, offset: int, amax_value=None, row_ids=None):
+    """bf16 [rows, C] -> rotated NVFP4 with stochastic rounding (definition step 4):
+    (packed codes, row-major scales, g, amax of y)."""
+    y = fwht_f32(NV.bf16_to_f32(x_bits), b)
+    if amax_value is not None:
+        a = np.float32(amax_value)
+    else:
+        a = np.float32(np.max(np.abs(y))) if y.size else np.float32(0.0)
+    g = NV.global_scale(a)
+    codes, sf = SR.quantize_values_sr(y, g, seed, offset, row_ids)
     return NV.pack_codes(codes), sf, g, a

@@ -100,24 +100,32 @@ def e2m1_encode_sr(u, r16) -> np.ndarray:
     return code | np.where(np.signbit(u), np.uint8(8), np.uint8(0))
 
 
-def quantize_sr(x_bits, seed: int, offset: int, amax_value=None, row_ids=None):
-    """bf16 [rows, K] -> (packed codes [rows, K/2], row-major scales [rows, K/16], g, amax).
-    ``row_ids``: the tensor rows x_bits holds (a sample of a larger tensor, whose
-    amax is then given), which select the random integers."""
-    x = NV.bf16_to_f32(x_bits)
-    rows, k = x.shape
-    a = NV.amax(x_bits) if amax_value is None else np.float32(amax_value)
-    g = NV.global_scale(a)
-    xb = x.reshape(rows, k // NV.BLOCK, NV.BLOCK)
-    ab = np.max(np.abs(xb), axis=2) if k else np.zeros((rows, 0), dtype=np.float32)
+def quantize_values_sr(y, g, seed: int, offset: int, row_ids=None):
+    """Steps 3-5 for fp32 values y [rows, K] under a given encode scale g:
+    (codes [rows, K] unpacked, row-major scales [rows, K/16])."""
+    y = np.asarray(y, dtype=np.float32)
+    rows, k = y.shape
+    g = np.float32(g)
+    yb = y.reshape(rows, k // NV.BLOCK, NV.BLOCK)
+    ab = np.max(np.abs(yb), axis=2) if k else np.zeros((rows, 0), dtype=np.float32)
     s_raw = (ab * g).astype(np.float32) / np.float32(6.0)
     sf = NV.e4m3_encode_satfinite(s_raw.astype(np.float32))
     sd = NV.e4m3_decode(sf)
-    t = (xb * g).astype(np.float32)
+    t = (yb * g).astype(np.float32)
     zero = (sd == 0)[:, :, None]
     with np.errstate(divide="ignore", invalid="ignore"):
         u = np.where(zero, np.float32(0.0), t / np.where(zero, np.float32(1.0), sd[:, :, None])).astype(np.float32)
     r16 = random16(rows, k, seed, offset, row_ids).reshape(rows, k // NV.BLOCK, NV.BLOCK)
     codes = e2m1_encode_sr(u, r16)
     codes = np.where(np.broadcast_to(zero, codes.shape), np.uint8(0), codes)
-    return NV.pack_codes(codes.reshape(rows, k)), sf.astype(np.uint8), g, a
+    return codes.reshape(rows, k).astype(np.uint8), sf.astype(np.uint8)
+
+
+def quantize_sr(x_bits, seed: int, offset: int, amax_value=None, row_ids=None):
+    """bf16 [rows, K] -> (packed codes [rows, K/2], row-major scales [rows, K/16], g, amax).
+    ``row_ids``: the tensor rows x_bits holds (a sample of a larger tensor, whose
+    amax is then given), which select the random integers."""
+    a = NV.amax(x_bits) if amax_value is None else np.float32(amax_value)
+    g = NV.global_scale(a)
+    codes, sf = quantize_values_sr(NV.bf16_to_f32(x_bits), g, seed, offset, row_ids)
+    return NV.pack_codes(codes), sf, g, a

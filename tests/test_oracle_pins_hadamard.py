@@ -184,3 +184,26 @@ def test_planted_mistakes(mutate, monkeypatch):
             caught = True
             break
     assert caught, f"no pin catches {mutate.__name__}"
+
+
+def test_rotated_stochastic_composition():
+    """Rotation followed by stochastic rounding: order 1 is the plain stochastic
+    quantizer; scales, g and amax are the rotated quantizer's; every code is a
+    neighbour of the rotated u; averaged over offsets, the dequantized values
+    approach y = x H (unbiased in the rotated domain)."""
+    from oracle import stochastic_oracle as S
+    x = _x(8, 256, 41)
+    assert all(np.array_equal(u, v) for u, v in zip(H.quantize_hadamard_sr(x, 1, 5, 6), S.quantize_sr(x, 5, 6)))
+    for b in (16, 128):
+        p, sf, g, a = H.quantize_hadamard_sr(x, b, 5, 6)
+        p2, sf2, g2, a2 = H.quantize_hadamard(x, b)
+        assert np.array_equal(sf, sf2) and g == g2 and a == a2
+        d_rn = np.abs(O.e2m1_decode(O.unpack_codes(p)) - O.e2m1_decode(O.unpack_codes(p2)))
+        assert np.all(d_rn <= 2.0)                                   # at most one grid step apart
+    y = H.fwht_f32(O.bf16_to_f32(x), 16).astype(np.float64)
+    acc = np.zeros_like(y)
+    for off in range(48):
+        p, sf, g, _ = H.quantize_hadamard_sr(x, 16, 9, off)
+        acc += O.dequantize(p, sf, g)
+    p2, sf2, g2, _ = H.quantize_hadamard(x, 16)
+    assert np.abs(acc / 48 - y).mean() < 0.4 * np.abs(O.dequantize(p2, sf2, g2) - y).mean()
