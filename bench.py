@@ -491,6 +491,10 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
             "ms": ms_h, "gbs_two_pass": two_pass / ms_h / 1e6, "frac_hbm": two_pass / ms_h / 1e6 / hbm_peak,
             "back_to_back_ms": ms_hb, "back_to_back_frac_hbm": two_pass / ms_hb / 1e6 / hbm_peak,
             "quantize_pass_ms": ms_h1, "quantize_pass_frac_hbm": one_pass / ms_h1 / 1e6 / hbm_peak}
+    ms_hs = _timed(torch, dev, flush, lambda: nv.quantize_hadamard_stochastic(x, 16, 1234, 0, nv.SF_TCGEN05, out=q),
+                   reps)
+    had["order=16_stochastic"] = {"ms": ms_hs, "gbs_two_pass": two_pass / ms_hs / 1e6,
+                                  "frac_hbm": two_pass / ms_hs / 1e6 / hbm_peak}
     out["hadamard_quantize_16384x8192"] = had
     del x, q
     # stochastic rounding of the codes (Philox4x32-10 in the kernel), same input and bytes

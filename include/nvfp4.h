@@ -179,6 +179,22 @@ NVFP4_API nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows,
                                      float* g_dev, float* amax_dev, int amax_given, nvfp4_stream_t stream);
 
 /*
+ * The rotated quantizer with stochastic rounding of the codes: y = x H as in
+ * nvfp4_quantize_hadamard, then y quantized as nvfp4_quantize_stochastic
+ * quantizes x (block scales round to nearest; each code rounds up with
+ * probability ceil(f * 2^16) / 2^16 from Philox4x32-10 bits, the counters of
+ * block b of row r being (2b + h, r, offset mod 2^32, offset div 2^32), key =
+ * seed).  The "FP4" encyclopedia entry (技術原理) names the two techniques
+ * together.  Arguments, constraints and errors as nvfp4_quantize_hadamard,
+ * plus seed and offset as nvfp4_quantize_stochastic.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize_hadamard_stochastic(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx,
+                                                int hadamard_order, void* codes, void* sf,
+                                                nvfp4_sf_layout layout, float* g_dev, float* amax_dev,
+                                                int amax_given, uint64_t seed, uint64_t offset,
+                                                nvfp4_stream_t stream);
+
+/*
  * MXFP4, the format the pages set against NVFP4 ("mxFP4/nvFP4 最小化知识",
  * (一) mxFP4的技术局限; "low-precision-floats", FP4 / MXFP4 / NVFP4): one E8M0
  * (power-of-two) scale per 32 consecutive elements along K and no global

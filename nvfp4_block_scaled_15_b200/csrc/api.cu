@@ -194,15 +194,15 @@ nvfp4_status nvfp4_quantize_stochastic(const void* x_bf16, int64_t rows, int64_t
   return launch_quantize_sr(x_bf16, rows, k, ldx, codes, sf, layout, g_dev, amax_dev, seed, offset, s);
 }
 
-nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, int hadamard_order,
-                                     void* codes, void* sf, nvfp4_sf_layout layout, float* g_dev, float* amax_dev,
-                                     int amax_given, nvfp4_stream_t stream) {
+static nvfp4_status quantize_hadamard_common(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, int n,
+                                             void* codes, void* sf, nvfp4_sf_layout layout, float* g_dev,
+                                             float* amax_dev, int amax_given, bool stochastic, uint64_t seed,
+                                             uint64_t offset, nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(x_bf16, rows, k, ldx);
   if (st != NVFP4_OK) return st;
   if (!g_dev || !amax_dev || ((!codes || !sf) && rows > 0 && k > 0)) return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
   if (amax_given != 0 && amax_given != 1) return NVFP4_ERR_INVALID_ARG;
-  const int n = hadamard_order;
   if (n < 1 || n > 512 || (n & (n - 1)) != 0) return NVFP4_ERR_INVALID_ARG;
   if ((k % 16) != 0 || (layout == NVFP4_SF_TCGEN05 && (k % 64) != 0) || (k % n) != 0)
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -214,7 +214,23 @@ nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows, int64_t k
     st = launch_hadamard_amax(x_bf16, rows, k, ldx, n, amax_dev, s);
     if (st != NVFP4_OK) return st;
   }
-  return launch_hadamard_quantize(x_bf16, rows, k, ldx, n, codes, sf, layout, g_dev, amax_dev, s);
+  return launch_hadamard_quantize(x_bf16, rows, k, ldx, n, codes, sf, layout, g_dev, amax_dev, stochastic, seed,
+                                  offset, s);
+}
+
+nvfp4_status nvfp4_quantize_hadamard(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx, int hadamard_order,
+                                     void* codes, void* sf, nvfp4_sf_layout layout, float* g_dev, float* amax_dev,
+                                     int amax_given, nvfp4_stream_t stream) {
+  return quantize_hadamard_common(x_bf16, rows, k, ldx, hadamard_order, codes, sf, layout, g_dev, amax_dev,
+                                  amax_given, false, 0, 0, stream);
+}
+
+nvfp4_status nvfp4_quantize_hadamard_stochastic(const void* x_bf16, int64_t rows, int64_t k, int64_t ldx,
+                                                int hadamard_order, void* codes, void* sf, nvfp4_sf_layout layout,
+                                                float* g_dev, float* amax_dev, int amax_given, uint64_t seed,
+                                                uint64_t offset, nvfp4_stream_t stream) {
+  return quantize_hadamard_common(x_bf16, rows, k, ldx, hadamard_order, codes, sf, layout, g_dev, amax_dev,
+                                  amax_given, true, seed, offset, stream);
 }
 
 size_t nvfp4_mxfp4_sf_bytes(int64_t rows, int64_t k, nvfp4_sf_layout layout) {

@@ -39,9 +39,10 @@ nvfp4_status launch_quantize_sr(const void* x, int64_t rows, int64_t k, int64_t 
 // Hadamard-rotated quantizer (order n: a power of two <= 512 dividing k).
 nvfp4_status launch_hadamard_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, int n, float* amax_dev,
                                   cudaStream_t s);
+// stochastic: round the codes stochastically (Philox4x32-10 bits from seed, offset).
 nvfp4_status launch_hadamard_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, int n, void* codes,
                                       void* sf, nvfp4_sf_layout layout, float* g_dev, const float* amax_dev,
-                                      cudaStream_t s);
+                                      bool stochastic, uint64_t seed, uint64_t offset, cudaStream_t s);
 nvfp4_status launch_swizzle(const void* src, int64_t rows, int64_t k, void* dst, cudaStream_t s);
 nvfp4_status launch_mx_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
                                 nvfp4_sf_layout layout, cudaStream_t s);

@@ -256,6 +256,27 @@ __device__ __forceinline__ uint2 block_codes_f32(const float2 (&p)[8], float g, 
   return c;
 }
 
+// 16 codes of one fp32 block with stochastic rounding (block_codes_f32's
+// quotient, block_codes_sr's rounding and random-bit layout).
+__device__ __forceinline__ uint2 block_codes_f32_sr(const float2 (&p)[8], float g, float2 e, uint4 ra, uint4 rb) {
+  const float2 ng2 = make_float2(-g, -g);
+  const float2 nyr2 = make_float2(-e.y, -e.y);
+  const float2 sd2 = make_float2(e.x, e.x);
+  const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+  float2 u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 tn = __fmul2_rn(p[i], ng2);
+    const float2 q = __fmul2_rn(tn, nyr2);
+    const float2 rr = __ffma2_rn(q, sd2, tn);
+    const float2 d = __ffma2_rn(rr, nyr2, q);                                   // RN(t / sd)
+    u[i] = make_float2(e2m1_round_stochastic(d.x, rw[i] & 0xFFFFu), e2m1_round_stochastic(d.y, rw[i] >> 16));
+  }
+  uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
+  if (e.x == 0.0f) c = make_uint2(0u, 0u);
+  return c;
+}
+
 // Byte offset of (row r, block b) in the tensor-core scale layout whose
 // padded block count is kb_pad (a multiple of 4).
 __host__ __device__ __forceinline__ int64_t sf_tc_offset(int64_t r, int64_t b, int64_t kb_pad) {

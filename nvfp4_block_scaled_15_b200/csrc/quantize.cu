@@ -388,9 +388,11 @@ __global__ void __launch_bounds__(kThreads) hadamard_amax_kernel(const uint16_t*
   }
 }
 
-// One rotated block: E4M3 scale RN_e4m3(RN(RN(ab * g) / 6)) and 16 codes.
+// One rotated block: E4M3 scale RN_e4m3(RN(RN(ab * g) / 6)) and 16 codes,
+// rounded to nearest, or stochastically (kSR) with the random words ra, rb.
+template <bool kSR>
 __device__ __forceinline__ uint2 quantize_rotated_block(const float2 (&p)[8], float g, const float2* table,
-                                                        uint32_t& s8) {
+                                                        uint32_t& s8, uint4 ra, uint4 rb) {
   const float sixth = __frcp_rn(6.0f);
   const float t = __fmul_rn(abs_max16_f32(p), g);
   const float q = __fmul_rn(t, sixth);
@@ -400,16 +402,21 @@ __device__ __forceinline__ uint2 quantize_rotated_block(const float2 (&p)[8], fl
       : "=r"(s2)
       : "f"(0.0f), "f"(sr));
   s8 = s2 & 0xFFu;
+  if (kSR) return block_codes_f32_sr(p, g, table[s8 & 0x7Fu], ra, rb);
   return block_codes_f32(p, g, table[s8 & 0x7Fu]);
 }
 
 // Pass 2: rotate again and quantize y (same grid and stores as quantize_kernel),
-// one block at a time to keep register use low.
-template <bool kTcLayout, bool kWide>
+// one block at a time to keep register use low.  kSR: stochastic rounding of
+// the codes, the random words of block b of row r from Philox4x32-10 with
+// key (seed_lo, seed_hi) and counters (2b + h, r, offset_lo, offset_hi), as in
+// quantize_sr_kernel (positions in y).
+template <bool kTcLayout, bool kWide, bool kSR>
 __global__ void __launch_bounds__(kThreads)
     hadamard_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
-                             const float* __restrict__ amax_in, int* __restrict__ status) {
+                             const float* __restrict__ amax_in, uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo,
+                             uint32_t off_hi, int* __restrict__ status) {
   __shared__ float2 table[128];
   const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
   const int kb = k >> 4;
@@ -437,15 +444,26 @@ __global__ void __launch_bounds__(kThreads)
 
   uint2 c0, c1;
   uint32_t s0, s1;
+  const uint32_t ur = static_cast<uint32_t>(r);
   {
     float2 p[8];
     rotate_block(w0, n, c, p);
-    c0 = quantize_rotated_block(p, g, table, s0);
+    uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+    if (kSR) {
+      ra = philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi);
+      rb = philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+    }
+    c0 = quantize_rotated_block<kSR>(p, g, table, s0, ra, rb);
   }
   {
     float2 p[8];
     rotate_block(w1, n, c, p);
-    c1 = quantize_rotated_block(p, g, table, s1);
+    uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+    if (kSR) {
+      ra = philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi);
+      rb = philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+    }
+    c1 = quantize_rotated_block<kSR>(p, g, table, s1, ra, rb);
   }
   store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
@@ -571,10 +589,10 @@ cudaError_t launch_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, in
   return cudaLaunchKernelEx(&cfg, quantize_kernel<kTc, kWide>, x, rows, k, ldx, codes, sf, g_dev, amax_dev, status);
 }
 
-template <bool kTc, bool kWide>
+template <bool kTc, bool kWide, bool kSR>
 cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
                                          int n, float c, uint8_t* codes, uint8_t* sf, float* g_dev,
-                                         const float* amax_dev, int* status) {
+                                         const float* amax_dev, uint64_t seed, uint64_t offset, int* status) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
@@ -584,8 +602,9 @@ cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, hadamard_quantize_kernel<kTc, kWide>, x, rows, k, ldx, n, c, codes, sf, g_dev,
-                            amax_dev, status);
+  return cudaLaunchKernelEx(&cfg, hadamard_quantize_kernel<kTc, kWide, kSR>, x, rows, k, ldx, n, c, codes, sf,
+                            g_dev, amax_dev, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
+                            static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32), status);
 }
 
 template <bool kTc, bool kWide>
@@ -699,9 +718,28 @@ nvfp4_status launch_hadamard_amax(const void* x, int64_t rows, int64_t k, int64_
   return launch_status(cudaGetLastError());
 }
 
+namespace {
+
+template <bool kSR>
+cudaError_t dispatch_hadamard_quantize(dim3 grid, bool tc, bool wide, cudaStream_t s, const uint16_t* x, int rows,
+                                       int k, int64_t ldx, int n, float c, uint8_t* codes, uint8_t* sf, float* g_dev,
+                                       const float* amax_dev, uint64_t seed, uint64_t offset, int* status) {
+  if (tc)
+    return wide ? launch_hadamard_quantize_pdl<true, true, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
+                                                                amax_dev, seed, offset, status)
+                : launch_hadamard_quantize_pdl<true, false, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
+                                                                 amax_dev, seed, offset, status);
+  return wide ? launch_hadamard_quantize_pdl<false, true, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
+                                                               amax_dev, seed, offset, status)
+              : launch_hadamard_quantize_pdl<false, false, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
+                                                                amax_dev, seed, offset, status);
+}
+
+}  // namespace
+
 nvfp4_status launch_hadamard_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, int n, void* codes,
                                       void* sf, nvfp4_sf_layout layout, float* g_dev, const float* amax_dev,
-                                      cudaStream_t s) {
+                                      bool stochastic, uint64_t seed, uint64_t offset, cudaStream_t s) {
   int* status = device_status_ptr();
   if (!status) return NVFP4_ERR_CUDA;
   const uint16_t* xs = static_cast<const uint16_t*>(x);
@@ -710,22 +748,16 @@ nvfp4_status launch_hadamard_quantize(const void* x, int64_t rows, int64_t k, in
   const float c = hadamard_norm(n);
   const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
   const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
-  const int ir = static_cast<int>(rows), ik = static_cast<int>(k);
-  if (grid_rows == 0 || segs == 0)   // nothing to quantize: still publish g (from the given amax)
-    return launch_status(launch_hadamard_quantize_pdl<false, false>(dim3(1, 1), s, xs, 0, 0, ldx, n, c, cs, ss,
-                                                                    g_dev, amax_dev, status));
-  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
-  const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
-  cudaError_t e;
-  if (layout == NVFP4_SF_TCGEN05)
-    e = wide ? launch_hadamard_quantize_pdl<true, true>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev, status)
-             : launch_hadamard_quantize_pdl<true, false>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
-                                                         status);
-  else
-    e = wide ? launch_hadamard_quantize_pdl<false, true>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
-                                                         status)
-             : launch_hadamard_quantize_pdl<false, false>(grid, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
-                                                          status);
+  const bool empty = grid_rows == 0 || segs == 0;   // nothing to quantize: still publish g (from the given amax)
+  const dim3 grid = empty ? dim3(1, 1) : dim3(static_cast<unsigned>(grid_rows), segs);
+  const int ir = empty ? 0 : static_cast<int>(rows), ik = empty ? 0 : static_cast<int>(k);
+  const bool tc = !empty && layout == NVFP4_SF_TCGEN05;
+  const bool wide = !empty && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  const cudaError_t e =
+      stochastic ? dispatch_hadamard_quantize<true>(grid, tc, wide, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev, amax_dev,
+                                                    seed, offset, status)
+                 : dispatch_hadamard_quantize<false>(grid, tc, wide, s, xs, ir, ik, ldx, n, c, cs, ss, g_dev,
+                                                     amax_dev, seed, offset, status);
   return launch_status(e);
 }
 

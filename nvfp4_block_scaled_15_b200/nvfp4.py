@@ -47,6 +47,8 @@ _SIGS = {
     "nvfp4_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _vp], _i32),
     "nvfp4_quantize_stochastic": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _u64, _u64, _vp],
                                   _i32),
+    "nvfp4_quantize_hadamard_stochastic": ([_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _vp, _vp, _i32, _u64, _u64,
+                                            _vp], _i32),
     "nvfp4_quantize_hadamard": ([_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp], _i32),
     "nvfp4_swizzle_sf": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "nvfp4_gemm": ([_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp], _i32),
@@ -139,6 +141,13 @@ def nvfp4_quantize_hadamard(x, rows, k, ldx, order, codes, sf, layout, g_dev, am
                             stream=None) -> None:
     _check(_lib.nvfp4_quantize_hadamard(_p(x), rows, k, ldx, int(order), _p(codes), _p(sf), layout, _p(g_dev),
                                         _p(amax_dev), int(amax_given), _s(stream)), "nvfp4_quantize_hadamard")
+
+
+def nvfp4_quantize_hadamard_stochastic(x, rows, k, ldx, order, codes, sf, layout, g_dev, amax_dev, amax_given,
+                                       seed, offset, stream=None) -> None:
+    _check(_lib.nvfp4_quantize_hadamard_stochastic(_p(x), rows, k, ldx, int(order), _p(codes), _p(sf), layout,
+                                                   _p(g_dev), _p(amax_dev), int(amax_given), int(seed), int(offset),
+                                                   _s(stream)), "nvfp4_quantize_hadamard_stochastic")
 
 
 def nvfp4_swizzle_sf(sf_rowmajor, rows, k, sf_tc, stream=None) -> None:
@@ -267,6 +276,19 @@ def quantize_hadamard(x: torch.Tensor, order: int, layout: int = SF_TCGEN05, out
         q.amax.copy_(amax)
     nvfp4_quantize_hadamard(x, rows, k, x.stride(0), order, q.codes, q.sf, layout, q.g, q.amax,
                             1 if amax is not None else 0, stream)
+    return q
+
+
+def quantize_hadamard_stochastic(x: torch.Tensor, order: int, seed: int, offset: int, layout: int = SF_TCGEN05,
+                                 out: Quantized | None = None, amax=None, stream=None) -> Quantized:
+    """bf16 [rows, k] -> NVFP4 of y = x H with stochastically rounded codes."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, k = x.shape
+    q = out if out is not None else empty_quantized(rows, k, layout, x.device)
+    if amax is not None:
+        q.amax.copy_(amax)
+    nvfp4_quantize_hadamard_stochastic(x, rows, k, x.stride(0), order, q.codes, q.sf, layout, q.g, q.amax,
+                                       1 if amax is not None else 0, seed, offset, stream)
     return q
 
 

@@ -94,6 +94,9 @@ def test_argument_errors_return_before_any_device_work(nv):
     assert raw(qh, fake, 4, 192, 192, 128, fake, fake, 1, fake, fake, 0, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert raw(qh, fake, 4, 48, 48, 16, fake, fake, 1, fake, fake, 0, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert raw(qh, fake, 4, 64, 64, 16, fake + 2, fake, 1, fake, fake, 0, None) == nv.ERR_MISALIGNED
+    qhs = "nvfp4_quantize_hadamard_stochastic"
+    assert raw(qhs, fake, 4, 256, 256, 3, fake, fake, 1, fake, fake, 0, 1, 2, None) == nv.ERR_INVALID_ARG
+    assert raw(qhs, fake, 4, 192, 192, 128, fake, fake, 1, fake, fake, 0, 1, 2, None) == nv.ERR_UNSUPPORTED_SHAPE
 
 
 def test_no_device_means_cuda_or_arch_error(nv):

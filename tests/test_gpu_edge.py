@@ -23,7 +23,7 @@ def test_empty_tensors(lib, rows, k, layout):
     _, _, g_ref, a_ref = O.quantize(np.zeros((rows, k), dtype=np.uint16))
     assert g_ref == np.float32(1.0) and a_ref == 0
     for q in (lib.quantize(x, layout), lib.quantize_hadamard(x, 16, layout),
-              lib.quantize_stochastic(x, 1, 2, layout)):
+              lib.quantize_stochastic(x, 1, 2, layout), lib.quantize_hadamard_stochastic(x, 16, 1, 2, layout)):
         torch.cuda.synchronize()
         assert lib.nvfp4_check_device_status() == lib.OK
         assert f32_scalar(q.g) == 1.0 and f32_scalar(q.amax) == 0.0

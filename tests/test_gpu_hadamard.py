@@ -138,3 +138,33 @@ def test_full_size_sampled_rows(lib, order):
     codes_ref, sf_ref, _, _ = H.quantize_hadamard(x[rows], order, amax_value=amax)
     assert np.array_equal(host_u8(q.codes)[rows], codes_ref)
     assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape)[rows], sf_ref)
+
+
+@pytest.mark.parametrize("order", [1, 16, 128, 512])
+@pytest.mark.parametrize("rows,k", [(200, 1536), (3, 12288)])
+@pytest.mark.parametrize("layout", [0, 1], ids=["rowmajor", "tcgen05"])
+def test_rotated_stochastic_matches_oracle(lib, order, rows, k, layout):
+    """Rotation then stochastic rounding, bit-exact: the Philox bits of each
+    position in y are drawn identically on both sides."""
+    x = inputs.activations_with_outliers(rows, k, seed=700 + order, fraction=0.01, factor=50.0)
+    seed, offset = 0xABCDEF0123456789, 77 + order
+    q = lib.quantize_hadamard_stochastic(dev_bf16(x), order, seed, offset, layout)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    _assert_same(lib, q, H.quantize_hadamard_sr(x, order, seed, offset), layout)
+
+
+def test_rotated_stochastic_full_size_sampled_rows(lib):
+    x = inputs.quantize_bandwidth()
+    q = lib.quantize_hadamard_stochastic(dev_bf16(x), 16, 42, 1, lib.SF_TCGEN05)
+    torch.cuda.synchronize()
+    assert lib.nvfp4_check_device_status() == lib.OK
+    amax = np.float32(0.0)
+    for r0 in range(0, x.shape[0], 2048):
+        y = H.fwht_f32(O.bf16_to_f32(x[r0:r0 + 2048]), 16)
+        amax = max(amax, np.float32(np.max(np.abs(y))))
+    assert f32_scalar(q.amax) == amax
+    rows = np.sort(np.random.default_rng(29).choice(x.shape[0], 64, replace=False))
+    codes_ref, sf_ref, _, _ = H.quantize_hadamard_sr(x[rows], 16, 42, 1, amax_value=amax, row_ids=rows)
+    assert np.array_equal(host_u8(q.codes)[rows], codes_ref)
+    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape)[rows], sf_ref)
