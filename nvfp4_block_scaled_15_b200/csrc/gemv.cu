@@ -287,13 +287,31 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       // for the head of a tile I leave unfinished
       float* mine = p.partials + (static_cast<int64_t>(2 * cta + (has_head ? 1 : 0)) * p.M) * BM;
       const float* other = p.partials + (static_cast<int64_t>(has_head ? 2 * (cta + 1) : 2 * (cta - 1) + 1) * p.M) * BM;
+      // The other contributor usually arrived long ago (a CTA works its tiles'
+      // tail segments first and head segments last).  If its arrival is on the
+      // counter, its partial was published before it (fence, then the atomic),
+      // so an acquire load of the counter makes it visible: finish the tile now,
+      // without writing this side's partial, fencing or counting.  Otherwise
+      // both take the counted path below and the second arrival finishes.
+      int* counter = &p.counters[tile * 4 + quad];
+      if (ld_acquire_gpu(counter) >= 1) {
+        if (n < p.N) {
+#pragma unroll
+          for (int m = 0; m < GV_N; ++m)
+            if (m < p.M) {
+              const float sum = __uint_as_float(v[m]) + __ldcg(other + m * BM + col);
+              p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
+            }
+        }
+        continue;
+      }
 #pragma unroll
       for (int m = 0; m < GV_N; ++m)
         if (m < p.M) mine[m * BM + col] = __uint_as_float(v[m]);
       __threadfence();
       __syncwarp();
       int arrived = 0;
-      if (lane == 0) arrived = atomicAdd(&p.counters[tile * 4 + quad], 1);
+      if (lane == 0) arrived = atomicAdd(counter, 1);
       arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
       if (arrived == 1) {                                       // second of the two: finish
         __threadfence();
