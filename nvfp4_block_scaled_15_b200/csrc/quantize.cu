@@ -138,19 +138,20 @@ __device__ __forceinline__ void store_two_blocks(uint8_t* __restrict__ codes, ui
   }
 }
 
-template <bool kTcLayout, bool kWide>
+// kRows rows per CTA (rows kRows * R .. kRows * R + kRows - 1 for the CTA's
+// row group R): the per-CTA work (scale table, global scale, barrier) is
+// shared by kRows rows and each thread has 2 * kRows loads in flight.
+template <bool kTcLayout, bool kWide, int kRows>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                             int64_t ldx, uint8_t* __restrict__ codes,
                                                             uint8_t* __restrict__ sf, float* __restrict__ g_out,
                                                             const float* __restrict__ amax_in,
                                                             int* __restrict__ status) {
   __shared__ float2 table[128];
-  const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
+  const int r0 = static_cast<int>(gridDim.x - 1 - blockIdx.x) * kRows;
   const int kb = k >> 4;                      // blocks per row
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
-
-  const bool real_row = r < rows;
 
   // Launched as a programmatic dependent of the amax pass.  x is not written
   // by that pass, so its loads and the scale table go out before the wait and
@@ -158,8 +159,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   // comes after it.  (The kernels that release dependents early are the amax
   // passes and the GEMV prologue, none of which writes x; the amax pass itself
   // starts only after all earlier work on the stream has finished.)
-  uint32_t w0[8], w1[8];
-  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row, kb, b0, b1, w0, w1);
+  uint32_t w0[kRows][8], w1[kRows][8];
+#pragma unroll
+  for (int j = 0; j < kRows; ++j)
+    load_two_blocks<kWide>(x + static_cast<int64_t>(r0 + j) * ldx, r0 + j < rows, kb, b0, b1, w0[j], w1[j]);
   fill_scale_table(table);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
@@ -170,14 +173,17 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
   }
   __syncthreads();
 
-  uint2 c0, c1;
-  uint32_t s0, s1;
-  quantize_two_blocks(w0, w1, g, table, c0, c1, s0, s1);
-  if (!valid) {                                // all-zero codes and scales
-    c0 = c1 = make_uint2(0u, 0u);
-    s0 = s1 = 0u;
+#pragma unroll
+  for (int j = 0; j < kRows; ++j) {
+    uint2 c0, c1;
+    uint32_t s0, s1;
+    quantize_two_blocks(w0[j], w1[j], g, table, c0, c1, s0, s1);
+    if (!valid) {                              // all-zero codes and scales
+      c0 = c1 = make_uint2(0u, 0u);
+      s0 = s1 = 0u;
+    }
+    store_two_blocks<kTcLayout>(codes, sf, r0 + j, r0 + j < rows, k, kb, b0, b1, c0, c1, s0, s1);
   }
-  store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
 
 // Pass 2 with stochastic rounding of the element codes: the same grid,
@@ -574,7 +580,9 @@ __global__ void swizzle_kernel(const uint8_t* __restrict__ src, int rows, int kb
   }
 }
 
-template <bool kTc, bool kWide>
+constexpr int kQuantRows = 2;                  // rows per CTA of the quantize pass
+
+template <bool kTc, bool kWide, int kRows = kQuantRows>
 cudaError_t launch_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
                                 uint8_t* codes, uint8_t* sf, float* g_dev, const float* amax_dev, int* status) {
   cudaLaunchConfig_t cfg = {};
@@ -586,7 +594,8 @@ cudaError_t launch_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_kernel<kTc, kWide>, x, rows, k, ldx, codes, sf, g_dev, amax_dev, status);
+  return cudaLaunchKernelEx(&cfg, quantize_kernel<kTc, kWide, kRows>, x, rows, k, ldx, codes, sf, g_dev, amax_dev,
+                            status);
 }
 
 template <bool kTc, bool kWide, bool kSR>
@@ -656,7 +665,7 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx
   if (grid_rows == 0 || segs == 0)   // nothing to quantize: still publish g (from the given amax)
     return launch_status(launch_quantize_pdl<false, false>(dim3(1, 1), s, xs, 0, 0, ldx, cs, ss, g_dev, amax_dev,
                                                            status));
-  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  const dim3 grid(static_cast<unsigned>((grid_rows + kQuantRows - 1) / kQuantRows), segs);
   const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
   cudaError_t e;
   if (layout == NVFP4_SF_TCGEN05)
