@@ -63,7 +63,8 @@ def _repeated_calls(lib, m, n, k):
     check_bf16(host_bf16_bits(y2), d_ref, s_ref, alpha)
 
 
-@pytest.mark.parametrize("m,n,k", [(5, 1100, 960), (16, 1024, 8192), (1, 8192 + 40, 4160), (12, 4096, 64)],
+@pytest.mark.parametrize("m,n,k", [(5, 1100, 960), (16, 1024, 8192), (1, 8192 + 40, 4160), (12, 4096, 64),
+                                   (3, 256, 12288), (4, 384, 8192), (20, 512, 10240)],
                          ids=lambda v: str(v))
 def test_gemv_more_shapes(lib, m, n, k):
     """A partial last K stage (K % 256 != 0), ragged N, K = 64 (one MMA-K
