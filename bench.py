@@ -392,31 +392,56 @@ def main():
 
 
 def bench_e2e(nv, torch, dev, a_bits, qw, qa, steps):
+    """The step through host buffers: every step copies A [8192, 8192] bf16 from
+    pinned host memory, quantizes it, runs the GEMM and copies D back to pinned
+    host memory.  Steps are double-buffered on three streams (upload, compute,
+    download), as a serving loop overlaps them: step i+1's upload and step
+    i-1's download run while step i computes, each buffer reused only after
+    the work that read it has finished."""
     a_host = torch.from_numpy(np.ascontiguousarray(a_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
-    d_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    a_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    d_dev = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    d_host = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    a_dev = [torch.empty((M, K), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    d_dev = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    qas = [qa, nv.empty_quantized(M, K, nv.SF_TCGEN05, dev)]
+    up, comp, down = (torch.cuda.Stream(dev) for _ in range(3))
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        a_dev.copy_(a_host, non_blocking=True)
-        nv.quantize(a_dev, nv.SF_TCGEN05, out=qa)
-        nv.gemm(qa, qw, out=d_dev)
-        d_host.copy_(d_dev, non_blocking=True)
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(computed[b])          # a_dev[b] no longer read
+                a_dev[b].copy_(a_host, non_blocking=True)
+                uploaded[b].record(up)
+            with torch.cuda.stream(comp):
+                comp.wait_event(uploaded[b])
+                if i >= 2:
+                    comp.wait_event(downloaded[b])      # d_dev[b] copied out
+                nv.quantize(a_dev[b], nv.SF_TCGEN05, out=qas[b], stream=comp)
+                nv.gemm(qas[b], qw, out=d_dev[b], stream=comp)
+                computed[b].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                d_host[b].copy_(d_dev[b], non_blocking=True)
+                downloaded[b].record(down)
 
-    for _ in range(3):
-        one()
+    run(4)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    e0.record(up)
+    run(steps)
+    down.wait_stream(up)
+    down.wait_stream(comp)
+    e1.record(down)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
     return {"value": FLOPS_STEP / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps,
-            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2}
+            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+            "pipelining": "double-buffered: upload, compute and download of consecutive steps overlap"}
 
 
 def _timed(torch, dev, flush, fn, reps):
