@@ -15,6 +15,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "internal.h"
 #include "ptx.cuh"
 #include "quant_core.cuh"
@@ -336,6 +338,369 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode GEMV without a prologue (M <= 4, K <= 8192): every CTA quantizes the
+// activations itself, at its start, into a resident operand image in shared
+// memory, so the quantized activations never pass through global memory.
+//   * Image: for each 256-wide K stage one 8-row x 128-B tile of codes in the
+//     128-B-swizzled K-major layout the tcgen05 operand expects (row r, 16-B
+//     chunk c at r * 128 + ((c ^ r) * 16)), and for each 64-wide MMA-K step
+//     one 8-row x 16-B group of E4M3 scales (row r at r * 16, block b % 4 at
+//     byte b % 4).  The MMA's N = 32 operand reads rows 8..31 through a zero
+//     8-row-group stride, i.e. as copies of rows 0..7: they only feed output
+//     columns >= 8, which are never stored.
+//   * The weight ring holds only weights and their scales.
+//   * The four epilogue warps build the image (zero it, amax of x, global
+//     scale, codes and scales of every block) before they turn to the
+//     epilogue; the MMA thread waits for the image on a named barrier.
+//   * Fix-up counters carry the call's tag in their high 32 bits, so a
+//     counter left by an earlier call reads as zero and nothing has to clear
+//     them between calls.
+// ---------------------------------------------------------------------------
+constexpr int GF_MAX_M = 4;                  // rows of x held in registers by the quantizer threads
+constexpr int GF_MAX_K = 8192;
+constexpr int GF_BLOCKS = GF_MAX_K / 16 / (GV_EPI_WARPS * 32);   // 16-element blocks per thread and row
+constexpr int GF_STAGES = 8;
+constexpr int GF_STAGE_BYTES = GV_A_BYTES + 4 * SF_ATOM;          // weights + their scales
+constexpr int GF_XIMG_BYTES = (GF_MAX_K / BK) * 1024;             // 8 rows x 128 B per K stage
+constexpr int GF_XSF_BYTES = (GF_MAX_K / MMA_K) * 128;            // 8 rows x 16 B per MMA-K step
+constexpr int GF_SMEM_BYTES = GF_STAGES * GF_STAGE_BYTES + GF_XIMG_BYTES + GF_XSF_BYTES + 1024 + 256 + 1024;
+constexpr int GF_QTHREADS = GV_EPI_WARPS * 32;
+constexpr uint32_t GF_BAR_IMAGE = 1;      // named barrier: image ready (quantizer threads + MMA warp)
+constexpr uint32_t GF_BAR_QUANT = 2;      // named barrier among the quantizer threads
+static_assert(GF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(GF_BLOCKS % 2 == 0, "blocks are quantized in pairs");
+
+struct GemvFusedParams {
+  const uint16_t* x;
+  int64_t ldx;
+  const uint8_t* wsf;      // weight scales, tensor-core layout
+  const float* g_w;
+  float* partials;         // [2 * grid][M][128] fp32 stream-K partial slots
+  unsigned long long* counters;   // [tiles * 4]: (tag << 32) | arrivals
+  uint32_t tag;            // this call's tag (never 0)
+  __nv_bfloat16* y;
+  int64_t ldy;
+  int M, N, K;
+  int kb4;
+  int tiles;
+  int num_kt;
+  uint64_t wait_limit_ns;
+  int* status;
+};
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Count this contributor's arrival on a tagged counter; returns the number
+// of earlier arrivals of the same call (0 or 1).
+__device__ __forceinline__ int tagged_arrive(unsigned long long* c, uint32_t tag) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(c);
+  for (int attempt = 0; attempt < 64; ++attempt) {
+    const bool same = static_cast<uint32_t>(cur >> 32) == tag;
+    const unsigned long long want = same ? cur + 1ull : ((static_cast<unsigned long long>(tag) << 32) | 1ull);
+    const unsigned long long prev = atomicCAS(c, cur, want);
+    if (prev == cur) return same ? static_cast<int>(cur & 0xFFFFFFFFull) : 0;
+    cur = prev;
+  }
+  return 0;   // two contributors per tile cannot contend 64 times; reached only on corruption
+}
+
+__global__ void __launch_bounds__(GV_THREADS, 1)
+    gemv_fused_kernel(const __grid_constant__ CUtensorMap tmW, const GemvFusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* ximg = smem + GF_STAGES * GF_STAGE_BYTES;                 // 1024-aligned
+  uint8_t* xsfimg = ximg + GF_XIMG_BYTES;
+  float2* table = reinterpret_cast<float2*>(xsfimg + GF_XSF_BYTES);  // 128 entries
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(table) + 1024);
+  uint64_t* empty = full + GF_STAGES;
+  uint64_t* acc_full = empty + GF_STAGES;
+  uint64_t* acc_empty = acc_full + GV_ACC_BUFS;
+  uint64_t* mma_done = acc_empty + GV_ACC_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* red = tmem_slot + 2;                                     // [GV_EPI_WARPS] amax partials
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GF_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < GV_ACC_BUFS; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], GV_EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmW);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int units = p.tiles * p.num_kt;
+  const int u_begin = static_cast<int>(static_cast<int64_t>(units) * blockIdx.x / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<int64_t>(units) * (blockIdx.x + 1) / gridDim.x);
+  const int ksteps_total = p.K / MMA_K;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      const uint64_t stream = l2_evict_first_policy();   // weights are read once
+      for (int u = u_begin; u < u_end; ++u) {
+        const int tile = u / p.num_kt;
+        const int kt = gv_stage_k(u, tile, p.num_kt);
+        if (u - u_begin >= GF_STAGES &&
+            !mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status))
+          break;
+        const int nk = min(4, ksteps_total - kt * 4);
+        uint8_t* sA = smem + stage * GF_STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], GV_A_BYTES + nk * SF_ATOM);
+        tma_load_2d_hint(sA, &tmW, &full[stage], kt * BK_BYTES, tile * BM, stream);
+        bulk_load_hint(sA + GV_A_BYTES, p.wsf + (static_cast<int64_t>(tile) * p.kb4 + kt * 4) * SF_ATOM,
+                       nk * SF_ATOM, &full[stage], stream);
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == GF_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      for (int s = 0; s < GF_STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          (void)mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &no_abort, p.wait_limit_ns, p.status);
+        }
+    }
+  } else if (warp == 1) {
+    named_barrier(GF_BAR_IMAGE, GF_QTHREADS + 32);   // the activation image is complete
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      const uint32_t idesc = idesc_mxf4nvf4(BM, GV_N);
+      const uint32_t sX = smem_u32(ximg);
+      const uint32_t sXSF = smem_u32(xsfimg);
+      int u = u_begin;
+      bool ok = true;
+      while (u < u_end && ok) {
+        const int tile = u / p.num_kt;
+        const int seg_end = min(u_end, (tile + 1) * p.num_kt);
+        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * GV_N;
+        bool first = true;
+        for (; u < seg_end; ++u) {
+          const int kt = gv_stage_k(u, tile, p.num_kt);
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_limit_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, ksteps_total - kt * 4);
+          const uint32_t sA = smem_u32(smem + stage * GF_STAGE_BYTES);
+          const uint32_t sSFA = sA + GV_A_BYTES;
+          const uint32_t tsfa = tmem_base + GV_SF_BASE + stage * GV_SF_COLS_PER_STAGE;
+          const uint32_t tsfb = tsfa + 16;
+          for (int j = 0; j < nk; ++j) {
+            tc_cp_32x128b_warpx4(tsfa + j * 4, sf_desc(sSFA + j * SF_ATOM));
+            // rows 8..31 of the activation scales read rows 0..7 (zero group stride)
+            tc_cp_32x128b_warpx4(tsfb + j * 4, smem_desc(sXSF + (kt * 4 + j) * 128, 0, 0, 0));
+          }
+          for (int j = 0; j < nk; ++j) {
+            mma_mxf4nvf4(d_tmem, code_desc(sA + j * (MMA_K / 2)),
+                         smem_desc(sX + kt * 1024 + j * (MMA_K / 2), 16, 0, 2), idesc, tsfa + j * 4,
+                         tsfb + j * 4, first ? 0u : 1u);
+            first = false;
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == GF_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == GV_ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      tc_commit(mma_done);
+      volatile int no_abort = 0;
+      (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
+    }
+  } else {
+    // ---- the activation image (quantizer threads 0..127) ----
+    const int qt = threadIdx.x - 64;
+    const int kb = p.K >> 4;
+    {
+      uint4* z = reinterpret_cast<uint4*>(ximg);
+      for (int i = qt; i < (GF_XIMG_BYTES + GF_XSF_BYTES) / 16; i += GF_QTHREADS) z[i] = make_uint4(0u, 0u, 0u, 0u);
+      fill_scale_table_from(table, qt, GF_QTHREADS);
+    }
+    // x, read once into registers: thread qt takes blocks j = qt + 128 i of
+    // every row, block j being x's block (j + rot) % kb.  The rotation differs
+    // from CTA to CTA, so the 148 CTAs, which all read the whole of x, do not
+    // all ask the same L2 lines for the same data at the same moment.
+    const int rot = (blockIdx.x * 16) % (kb > 0 ? kb : 1);
+    uint32_t w[GF_MAX_M][GF_BLOCKS][8];
+#pragma unroll
+    for (int r = 0; r < GF_MAX_M; ++r)
+#pragma unroll
+      for (int i = 0; i < GF_BLOCKS; ++i) {
+        const int j = qt + GF_QTHREADS * i;
+        if (r < p.M && j < kb) {
+          const int b = j + rot < kb ? j + rot : j + rot - kb;
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.ldx + b * 16);
+          const uint4 a = src[0], c = src[1];
+          w[r][i][0] = a.x; w[r][i][1] = a.y; w[r][i][2] = a.z; w[r][i][3] = a.w;
+          w[r][i][4] = c.x; w[r][i][5] = c.y; w[r][i][6] = c.z; w[r][i][7] = c.w;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) w[r][i][q] = 0u;
+        }
+      }
+    uint32_t mx = 0;
+#pragma unroll
+    for (int r = 0; r < GF_MAX_M; ++r)
+#pragma unroll
+      for (int i = 0; i < GF_BLOCKS; ++i) mx = max(mx, abs_max_bits16(w[r][i]));
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (lane == 0) red[warp - 2] = mx;
+    named_barrier(GF_BAR_QUANT, GF_QTHREADS);   // partials, the zeroed image and the table
+    uint32_t all = 0;
+#pragma unroll
+    for (int i = 0; i < GV_EPI_WARPS; ++i) all = max(all, red[i]);
+    bool valid;
+    float g = global_scale_from_amax(__uint_as_float(all << 16), valid);
+    if (blockIdx.x == 0 && qt == 0 && !valid) record_status(p.status, kDevRange);
+    // codes and scales of every block (two at a time), into the swizzled image:
+    // block b of row r lands in K stage b / 16, 16-B chunk (b % 16) / 2
+    // (swizzled with r), half b % 2, and its scale in MMA-K step b / 4
+    if (valid) {
+#pragma unroll
+      for (int r = 0; r < GF_MAX_M; ++r) {
+        if (r >= p.M) break;
+#pragma unroll
+        for (int i = 0; i < GF_BLOCKS; i += 2) {
+          const int j0 = qt + GF_QTHREADS * i, j1 = j0 + GF_QTHREADS;
+          uint2 c0, c1;
+          uint32_t s0, s1;
+          quantize_two_blocks(w[r][i], w[r][i + 1], g, table, c0, c1, s0, s1);
+          if (j0 < kb) {
+            const int b = j0 + rot < kb ? j0 + rot : j0 + rot - kb;
+            *reinterpret_cast<uint2*>(ximg + (b >> 4) * 1024 + r * 128 + ((((b & 15) >> 1) ^ r) << 4) + (b & 1) * 8) = c0;
+            xsfimg[(b >> 2) * 128 + r * 16 + (b & 3)] = static_cast<uint8_t>(s0);
+          }
+          if (j1 < kb) {
+            const int b = j1 + rot < kb ? j1 + rot : j1 + rot - kb;
+            *reinterpret_cast<uint2*>(ximg + (b >> 4) * 1024 + r * 128 + ((((b & 15) >> 1) ^ r) << 4) + (b & 1) * 8) = c1;
+            xsfimg[(b >> 2) * 128 + r * 16 + (b & 3)] = static_cast<uint8_t>(s1);
+          }
+        }
+      }
+    }
+    fence_proxy_async_shared();                 // generic-proxy writes, read by the tensor core
+    asm volatile("bar.arrive %0, %1;" ::"r"(GF_BAR_IMAGE), "r"(GF_QTHREADS + 32) : "memory");
+
+    // ---- epilogue and stream-K fix-up (as gemv_kernel, tagged counters) ----
+    const int quad = warp & 3;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_w, valid ? g : 0.0f));
+    const int cta = blockIdx.x;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int u = u_begin;
+    while (u < u_end) {
+      const int tile = u / p.num_kt;
+      const int tile_begin = tile * p.num_kt;
+      const int seg_end = min(u_end, tile_begin + p.num_kt);
+      const bool has_head = u == tile_begin;
+      const bool has_tail = seg_end == tile_begin + p.num_kt;
+      u = seg_end;
+      if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * GV_N, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == GV_ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+      const int col = quad * 32 + lane;
+      const int n = tile * BM + col;
+      if (has_head && has_tail) {
+        if (n < p.N) {
+#pragma unroll
+          for (int m = 0; m < GF_MAX_M; ++m)
+            if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(__uint_as_float(v[m]) * alpha);
+        }
+        continue;
+      }
+      float* mine = p.partials + (static_cast<int64_t>(2 * cta + (has_head ? 1 : 0)) * p.M) * BM;
+      const float* other = p.partials + (static_cast<int64_t>(has_head ? 2 * (cta + 1) : 2 * (cta - 1) + 1) * p.M) * BM;
+      unsigned long long* counter = &p.counters[tile * 4 + quad];
+      const unsigned long long seen = ld_acquire_gpu_u64(counter);
+      if (static_cast<uint32_t>(seen >> 32) == p.tag && (seen & 0xFFFFFFFFull) >= 1ull) {
+        if (n < p.N) {
+#pragma unroll
+          for (int m = 0; m < GF_MAX_M; ++m)
+            if (m < p.M) {
+              const float sum = __uint_as_float(v[m]) + __ldcg(other + m * BM + col);
+              p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
+            }
+        }
+        continue;
+      }
+#pragma unroll
+      for (int m = 0; m < GF_MAX_M; ++m)
+        if (m < p.M) mine[m * BM + col] = __uint_as_float(v[m]);
+      __threadfence();
+      __syncwarp();
+      int arrived = 0;
+      if (lane == 0) arrived = tagged_arrive(counter, p.tag);
+      arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
+      if (arrived == 1) {
+        __threadfence();
+        if (n < p.N) {
+#pragma unroll
+          for (int m = 0; m < GF_MAX_M; ++m)
+            if (m < p.M) {
+              const float sum = __uint_as_float(v[m]) + __ldcg(other + m * BM + col);
+              p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
+            }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
 // Activation quantization for the GEMV (same rule as nvfp4_quantize) plus
 // clearing of the fix-up counters, in one cluster of GP_CLUSTER CTAs.  CTA c
 // owns activation rows c, c+8, c+16, c+24 (those below M): it reduces the
@@ -500,7 +865,7 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
 
 // Workspace of the GEMV: [32, K/2] activation codes | [128, K/16] activation
 // scales | g_x (16 B) | fp32 partial slots [2 * GV_MAX_CTAS][M][128] |
-// counters [tiles * 4].
+// counters [tiles * 4] (8 bytes each: the prologue-free kernel tags them).
 constexpr int GV_MAX_CTAS = 160;
 
 struct GemvWs {
@@ -515,15 +880,57 @@ static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
   w.gx = al(w.xsf + static_cast<size_t>(128) * K / 16);
   w.part = al(w.gx + 16);
   w.cnt = al(w.part + static_cast<size_t>(2 * GV_MAX_CTAS) * M * BM * 4);
-  w.total = al(w.cnt + static_cast<size_t>((N + BM - 1) / BM) * 4 * 4);
+  w.total = al(w.cnt + static_cast<size_t>((N + BM - 1) / BM) * 4 * 8);   // 8-byte tagged counters
   return w;
 }
 
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) { return gemv_ws_layout(M, N, K).total; }
 
+// Tags of the prologue-free GEMV's fix-up counters: unique per call within
+// the process (never 0, so a zeroed counter is never taken for this call's).
+static std::atomic<uint32_t> g_gemv_tag{0};
+
+static nvfp4_status launch_gemv_fused(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
+                                      const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy,
+                                      const GemvWs& L, uint8_t* base, cudaStream_t s) {
+  const int tiles = static_cast<int>((N + BM - 1) / BM);
+  const int sms = device_sm_count();
+  CUtensorMap tmW;
+  if (!make_code_map(&tmW, w_codes, N, K, BM)) return NVFP4_ERR_CUDA;
+  GemvFusedParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.ldx = ldx;
+  p.wsf = static_cast<const uint8_t*>(w_sf);
+  p.g_w = g_w;
+  p.partials = reinterpret_cast<float*>(base + L.part);
+  p.counters = reinterpret_cast<unsigned long long*>(base + L.cnt);
+  uint32_t tag = g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (tag == 0) tag = g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1;   // skip 0 on wrap
+  p.tag = tag;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ldy = ldy;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.kb4 = static_cast<int>(K / 64);
+  p.tiles = tiles;
+  p.num_kt = static_cast<int>((K + BK - 1) / BK);
+  p.wait_limit_ns = wait_limit_ns();
+  p.status = device_status_ptr();
+  if (!p.status) return NVFP4_ERR_CUDA;
+  int grid = tiles < sms ? tiles : sms;       // grid <= tiles: at most two contributors per tile
+  if (grid > GV_MAX_CTAS) grid = GV_MAX_CTAS;
+  cudaError_t e = cudaFuncSetAttribute(gemv_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GF_SMEM_BYTES);
+  if (e != cudaSuccess) return launch_status(e);
+  gemv_fused_kernel<<<grid, GV_THREADS, GF_SMEM_BYTES, s>>>(tmW, p);
+  return launch_status(cudaGetLastError());
+}
+
 nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
                          const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s) {
   const GemvWs L = gemv_ws_layout(M, N, K);
+  if (M <= GF_MAX_M && K <= GF_MAX_K && static_cast<int64_t>((N + BM - 1) / BM) * ((K + BK - 1) / BK) < (int64_t{1} << 30))
+    return launch_gemv_fused(x, M, ldx, w_codes, w_sf, g_w, N, K, y, ldy, L, static_cast<uint8_t*>(ws), s);
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint8_t* xq = base + L.xq;
   uint8_t* xsf = base + L.xsf;

@@ -76,9 +76,12 @@ extern "C" NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16,
   if (st != NVFP4_OK) return st;
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch)) != NVFP4_OK) return st;
-  // The existing GEMV path, given the fixed scratch as its workspace.  Its
-  // prologue rewrites the quantized activations and clears the partial sums
-  // and counters on every call, so nothing from an earlier call is reused.
+  // The existing GEMV paths, given the fixed scratch as their workspace.
+  // Nothing from an earlier call is reused: with M > 4 the prologue rewrites
+  // the quantized activations and clears the counters on every call; with
+  // M <= 4 the activations stay in shared memory and the counters carry the
+  // call's tag, so an earlier call's counts read as zero; partial sums are
+  // always written before they are read.
   return launch_gemv(x_bf16, M, ldx, w_codes, w_sf_tc, g_w_dev, N, K, y_bf16, ldy, scratch,
                      reinterpret_cast<cudaStream_t>(stream));
 }

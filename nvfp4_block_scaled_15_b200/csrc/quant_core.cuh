@@ -70,12 +70,16 @@ __device__ __forceinline__ float div_rn_by_recip(float t, float d, float y) {
 // Shared-memory table of the positive E4M3 scales: entry s (0 <= s < 128)
 // holds {sd, RN(1/sd)} for sd the E4M3 value of byte s (RN(1/0) stored as 0).
 // __frcp_rn is the correctly rounded reciprocal.
-__device__ __forceinline__ void fill_scale_table(float2* table) {
-  for (int s = static_cast<int>(threadIdx.x); s < 128; s += static_cast<int>(blockDim.x)) {
+__device__ __forceinline__ void fill_scale_table_from(float2* table, int first, int stride) {
+  for (int s = first; s < 128; s += stride) {
     const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(s), __NV_E4M3);
     const float sd = __half2float(__half(h));
     table[s] = make_float2(sd, sd > 0.0f ? __frcp_rn(sd) : 0.0f);
   }
+}
+
+__device__ __forceinline__ void fill_scale_table(float2* table) {
+  fill_scale_table_from(table, static_cast<int>(threadIdx.x), static_cast<int>(blockDim.x));
 }
 
 // |x| maximum of 16 bf16 values as a bf16 bit pattern without sign.  The
