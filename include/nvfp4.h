@@ -299,8 +299,9 @@ NVFP4_API size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_
  * Micro-Scaling" section 六).  y: out, bf16 [M, N], pitch ldy.
  * workspace: device scratch of nvfp4_workspace_bytes(NVFP4_OP_GEMV_BATCHED, M, N, K)
  *   bytes (quantized x, its scales and g, fp32 partial sums, tile counters);
- *   every call re-initialises what it uses.  Calls sharing a workspace must not
- *   overlap on the device.
+ *   every call re-initialises what it reads, or marks it with a tag of its
+ *   own, so the workspace needs no clearing, before the first call or
+ *   between calls.  Calls sharing a workspace must not overlap on the device.
  * K % 64 == 0, 1 <= M <= 32.
  */
 NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t ldx, const void* w_codes,
@@ -323,9 +324,9 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t
  *     up the scratch's device address; make that first call before any stream
  *     capture.  Nothing is allocated or freed, then or later.
  *   Sharing: every call on a device uses the same scratch and overwrites what
- *     the previous call left there (each call clears what must start at
- *     zero).  Calls that overlap on the device race: serialise them, e.g. on
- *     one stream.
+ *     the previous call left there (each call clears, or marks with a tag of
+ *     its own, what must start at zero).  Calls that overlap on the device
+ *     race: serialise them, e.g. on one stream.
  * Other arguments, constraints and errors as nvfp4_gemv_batched.
  */
 NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M, int64_t ldx, const void* w_codes,
