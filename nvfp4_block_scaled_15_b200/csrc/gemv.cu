@@ -352,7 +352,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 //   * The weight ring holds only weights and their scales.
 //   * The four epilogue warps build the image (zero it, amax of x, global
 //     scale, codes and scales of every block) before they turn to the
-//     epilogue; the MMA thread waits for the image on a named barrier.
+//     epilogue.  They meet on an mbarrier (x_sync) after the zeroing and the
+//     amax partials, and each arrives on another (x_ready) once its image
+//     writes are fenced for the tensor core's proxy; the MMA thread waits on
+//     x_ready before its first MMA.
 //   * Fix-up counters carry the call's tag in their high 32 bits, so a
 //     counter left by an earlier call reads as zero and nothing has to clear
 //     them between calls.
@@ -366,8 +369,6 @@ constexpr int GF_XIMG_BYTES = (GF_MAX_K / BK) * 1024;             // 8 rows x 12
 constexpr int GF_XSF_BYTES = (GF_MAX_K / MMA_K) * 128;            // 8 rows x 16 B per MMA-K step
 constexpr int GF_SMEM_BYTES = GF_STAGES * GF_STAGE_BYTES + GF_XIMG_BYTES + GF_XSF_BYTES + 1024 + 256 + 1024;
 constexpr int GF_QTHREADS = GV_EPI_WARPS * 32;
-constexpr uint32_t GF_BAR_IMAGE = 1;      // named barrier: image ready (quantizer threads + MMA warp)
-constexpr uint32_t GF_BAR_QUANT = 2;      // named barrier among the quantizer threads
 static_assert(GF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(GF_BLOCKS % 2 == 0, "blocks are quantized in pairs");
 
@@ -421,7 +422,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
   uint64_t* acc_full = empty + GF_STAGES;
   uint64_t* acc_empty = acc_full + GV_ACC_BUFS;
   uint64_t* mma_done = acc_empty + GV_ACC_BUFS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* x_sync = mma_done + 1;          // quantizer threads: zeroed image, table, amax partials
+  uint64_t* x_ready = x_sync + 1;           // the activation image is written and fenced
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* red = tmem_slot + 2;                                     // [GV_EPI_WARPS] amax partials
 
@@ -437,6 +440,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       mbar_init(&acc_empty[b], GV_EPI_WARPS);
     }
     mbar_init(mma_done, 1);
+    mbar_init(x_sync, GF_QTHREADS);
+    mbar_init(x_ready, GF_QTHREADS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -487,7 +492,6 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         }
     }
   } else if (warp == 1) {
-    named_barrier(GF_BAR_IMAGE, GF_QTHREADS + 32);   // the activation image is complete
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
@@ -497,7 +501,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       const uint32_t sX = smem_u32(ximg);
       const uint32_t sXSF = smem_u32(xsfimg);
       int u = u_begin;
-      bool ok = true;
+      // the activation image must be complete before the first MMA reads it
+      bool ok = mbar_wait_bounded(x_ready, 0, abort_flag, p.wait_limit_ns, p.status);
       while (u < u_end && ok) {
         const int tile = u / p.num_kt;
         const int seg_end = min(u_end, (tile + 1) * p.num_kt);
@@ -583,7 +588,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       for (int i = 0; i < GF_BLOCKS; ++i) mx = max(mx, abs_max_bits16(w[r][i]));
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
     if (lane == 0) red[warp - 2] = mx;
-    named_barrier(GF_BAR_QUANT, GF_QTHREADS);   // partials, the zeroed image and the table
+    mbar_arrive(x_sync);                        // zeroed image, table and partials visible to all quantizers
+    (void)mbar_wait_bounded(x_sync, 0, abort_flag, p.wait_limit_ns, p.status);
     uint32_t all = 0;
 #pragma unroll
     for (int i = 0; i < GV_EPI_WARPS; ++i) all = max(all, red[i]);
@@ -617,7 +623,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       }
     }
     fence_proxy_async_shared();                 // generic-proxy writes, read by the tensor core
-    asm volatile("bar.arrive %0, %1;" ::"r"(GF_BAR_IMAGE), "r"(GF_QTHREADS + 32) : "memory");
+    mbar_arrive(x_ready);
 
     // ---- epilogue and stream-K fix-up (as gemv_kernel, tagged counters) ----
     const int quad = warp & 3;
