@@ -100,23 +100,25 @@ def test_gemv_decode_full_size_sampled(lib, m):
 
 @pytest.mark.parametrize("m", [1, 4])
 def test_gemv_weights_in_l2_repeated(lib, m):
-    """Weights small enough to stay in L2 reach the tensor core long before the
-    activations are quantized (K = 8192 takes the longest to quantize), so any
-    MMA issued before its activation operand is complete would show here: ten
-    calls in a row, each against the oracle and all identical."""
-    n, k = 2048, 8192
+    """All 148 CTAs running (160 weight tiles) with 94 MB of weights resident in
+    L2, so the weight stages reach the tensor core while the CTAs are still
+    quantizing the activations (the longest at K = 8192): an MMA issued before
+    its activation operand is complete would show as a gross error.  Ten calls
+    in a row must be identical and within 2 bf16 ulp of the block-scaled GEMM
+    on the same quantized operands (parity of both against the oracle is
+    tested elsewhere)."""
+    n, k = 20480, 8192
     x = inputs.activations_with_outliers(m, k, seed=970 + m, fraction=0.01, factor=30.0)
     w = inputs.gaussian_bf16((n, k), seed=971, std=0.02)
     qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
     xd = dev_bf16(x)
+    ref = lib.gemm(lib.quantize(xd, lib.SF_TCGEN05), qw)
     ws = torch.empty(lib.nvfp4_workspace_bytes(lib.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device="cuda")
     outs = [lib.gemv_batched(xd, qw, workspace=ws) for _ in range(10)]
     torch.cuda.synchronize()
     assert lib.nvfp4_check_device_status() == lib.OK
-    px, sx, gx, _ = O.quantize(x)
-    pw, sw, gw, _ = O.quantize(w)
-    d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, pw, sw, gw)
     first = host_bf16_bits(outs[0])
-    check_bf16(first, d_ref, s_ref, alpha)
     for y in outs[1:]:
         assert np.array_equal(host_bf16_bits(y), first)
+    ulps = np.abs(O.bf16_ordinal(first) - O.bf16_ordinal(host_bf16_bits(ref)))
+    assert int(ulps.max()) <= 2, int(ulps.max())
