@@ -163,22 +163,30 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
-// Stochastic rounding of u onto the E2M1 grid with the 16-bit random integer
-// r: the magnitude a lies between neighbours lo and hi = lo + step (step 0.5
-// below 2, 1 below 4, 2 below 6); it rounds up when r < f * 2^16, f = (a - lo)
-// / step; a >= 6 gives 6; the sign of u is kept.  Every step is exact in fp32:
-// v = a / step is a power-of-two scaling, floor(v) and v - floor(v) are exact,
-// and f * 2^16 and r are exact, so the comparison is the real one.
-__device__ __forceinline__ float e2m1_round_stochastic(float u, uint32_t r) {
-  const float a = fabsf(u);
-  const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-  const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-  const float v = a * inv_step;
-  const float fl = floorf(v);
-  const bool up = static_cast<float>(r) < (v - fl) * 65536.0f;
-  float m = (up ? fl + 1.0f : fl) * step;
-  if (a >= 6.0f) m = 6.0f;
-  return copysignf(m, u);
+// Stochastic rounding of two values onto the E2M1 grid, with 16-bit random
+// integers (element x's in bits 0..15 of r, y's in bits 16..31): a magnitude
+// a lies between neighbours lo and hi = lo + step (step 0.5 below 2, 1 below
+// 4, 2 below 6); it rounds up when r < f * 2^16, f = (a - lo) / step; a >= 6
+// gives 6; the sign of u is kept.  Every step is exact in fp32: v = a / step
+// is a power-of-two scaling, floor(v) and v - floor(v) are exact, and
+// f * 2^16 and r are exact, so the comparison is the real one.  The
+// multiplies, the fraction and the step product run on the packed fp32x2
+// units.
+__device__ __forceinline__ float2 e2m1_round_stochastic2(float2 u, uint32_t r) {
+  const float ax = fabsf(u.x), ay = fabsf(u.y);
+  const float2 inv = make_float2(ax < 2.0f ? 2.0f : (ax < 4.0f ? 1.0f : 0.5f),
+                                 ay < 2.0f ? 2.0f : (ay < 4.0f ? 1.0f : 0.5f));
+  const float2 v = __fmul2_rn(make_float2(ax, ay), inv);
+  const float2 fl = make_float2(floorf(v.x), floorf(v.y));
+  const float2 thr = __fmul2_rn(__ffma2_rn(fl, make_float2(-1.0f, -1.0f), v), make_float2(65536.0f, 65536.0f));
+  const float2 up = make_float2(static_cast<float>(r & 0xFFFFu) < thr.x ? 1.0f : 0.0f,
+                                static_cast<float>(r >> 16) < thr.y ? 1.0f : 0.0f);
+  // step = 1 / inv exactly: for a power of two 2^e, 2^-e has bits 0x7F000000 - bits(2^e);
+  // a >= 6 gives 6 through the minimum (a in [6, 8) lands on 6 or 8), inf included
+  const float2 step = make_float2(__uint_as_float(0x7F000000u - __float_as_uint(inv.x)),
+                                  __uint_as_float(0x7F000000u - __float_as_uint(inv.y)));
+  const float2 m = __fmul2_rn(__fadd2_rn(fl, up), step);
+  return make_float2(copysignf(fminf(m.x, 6.0f), u.x), copysignf(fminf(m.y, 6.0f), u.y));
 }
 
 // 16 codes of one bf16 block for the scale entry e = {sd, RN(1/sd)} with
@@ -197,7 +205,7 @@ __device__ __forceinline__ uint2 block_codes_sr(const uint32_t (&w)[8], float g,
     const float2 q = __fmul2_rn(tn, nyr2);
     const float2 rr = __ffma2_rn(q, sd2, tn);
     const float2 d = __ffma2_rn(rr, nyr2, q);                                   // RN(t / sd)
-    u[i] = make_float2(e2m1_round_stochastic(d.x, rw[i] & 0xFFFFu), e2m1_round_stochastic(d.y, rw[i] >> 16));
+    u[i] = e2m1_round_stochastic2(d, rw[i]);
   }
   uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
   if (e.x == 0.0f) c = make_uint2(0u, 0u);
@@ -274,7 +282,7 @@ __device__ __forceinline__ uint2 block_codes_f32_sr(const float2 (&p)[8], float 
     const float2 q = __fmul2_rn(tn, nyr2);
     const float2 rr = __ffma2_rn(q, sd2, tn);
     const float2 d = __ffma2_rn(rr, nyr2, q);                                   // RN(t / sd)
-    u[i] = make_float2(e2m1_round_stochastic(d.x, rw[i] & 0xFFFFu), e2m1_round_stochastic(d.y, rw[i] >> 16));
+    u[i] = e2m1_round_stochastic2(d, rw[i]);
   }
   uint2 c = make_uint2(e2m1x8(u[0], u[1], u[2], u[3]), e2m1x8(u[4], u[5], u[6], u[7]));
   if (e.x == 0.0f) c = make_uint2(0u, 0u);
