@@ -417,22 +417,22 @@ __device__ __forceinline__ uint2 quantize_rotated_block(const float2 (&p)[8], fl
 // the codes, the random words of block b of row r from Philox4x32-10 with
 // key (seed_lo, seed_hi) and counters (2b + h, r, offset_lo, offset_hi), as in
 // quantize_sr_kernel (positions in y).
-template <bool kTcLayout, bool kWide, bool kSR>
+template <bool kTcLayout, bool kWide, bool kSR, int kRows>
 __global__ void __launch_bounds__(kThreads)
     hadamard_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
                              const float* __restrict__ amax_in, uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo,
                              uint32_t off_hi, int* __restrict__ status) {
   __shared__ float2 table[128];
-  const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
+  const int r0 = static_cast<int>(gridDim.x - 1 - blockIdx.x) * kRows;
   const int kb = k >> 4;
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
 
-  const bool real_row = r < rows;
-
-  uint32_t w0[8], w1[8];                       // x and the table before the wait, as in quantize_kernel
-  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row, kb, b0, b1, w0, w1);
+  uint32_t w0[kRows][8], w1[kRows][8];         // x and the table before the wait, as in quantize_kernel
+#pragma unroll
+  for (int j = 0; j < kRows; ++j)
+    load_two_blocks<kWide>(x + static_cast<int64_t>(r0 + j) * ldx, r0 + j < rows, kb, b0, b1, w0[j], w1[j]);
   fill_scale_table(table);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
@@ -444,34 +444,40 @@ __global__ void __launch_bounds__(kThreads)
   if (!valid) {                                // all-zero codes and scales
     g = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w0[i] = w1[i] = 0u;
+    for (int j = 0; j < kRows; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w0[j][i] = w1[j][i] = 0u;
   }
   __syncthreads();
 
-  uint2 c0, c1;
-  uint32_t s0, s1;
-  const uint32_t ur = static_cast<uint32_t>(r);
-  {
-    float2 p[8];
-    rotate_block(w0, n, c, p);
-    uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
-    if (kSR) {
-      ra = philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi);
-      rb = philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+#pragma unroll
+  for (int j = 0; j < kRows; ++j) {
+    const int r = r0 + j;
+    const uint32_t ur = static_cast<uint32_t>(r);
+    uint2 c0, c1;
+    uint32_t s0, s1;
+    {
+      float2 p[8];
+      rotate_block(w0[j], n, c, p);
+      uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+      if (kSR) {
+        ra = philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi);
+        rb = philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+      }
+      c0 = quantize_rotated_block<kSR>(p, g, table, s0, ra, rb);
     }
-    c0 = quantize_rotated_block<kSR>(p, g, table, s0, ra, rb);
-  }
-  {
-    float2 p[8];
-    rotate_block(w1, n, c, p);
-    uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
-    if (kSR) {
-      ra = philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi);
-      rb = philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+    {
+      float2 p[8];
+      rotate_block(w1[j], n, c, p);
+      uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+      if (kSR) {
+        ra = philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi);
+        rb = philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+      }
+      c1 = quantize_rotated_block<kSR>(p, g, table, s1, ra, rb);
     }
-    c1 = quantize_rotated_block<kSR>(p, g, table, s1, ra, rb);
+    store_two_blocks<kTcLayout>(codes, sf, r, r < rows, k, kb, b0, b1, c0, c1, s0, s1);
   }
-  store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
 }
 
 // ---------------------------------------------------------------------------
@@ -611,7 +617,8 @@ cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, hadamard_quantize_kernel<kTc, kWide, kSR>, x, rows, k, ldx, n, c, codes, sf,
+  return cudaLaunchKernelEx(&cfg, hadamard_quantize_kernel<kTc, kWide, kSR, kSR ? 1 : kQuantRows>, x, rows, k, ldx,
+                            n, c, codes, sf,
                             g_dev, amax_dev, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
                             static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32), status);
 }
@@ -758,7 +765,10 @@ nvfp4_status launch_hadamard_quantize(const void* x, int64_t rows, int64_t k, in
   const int segs = static_cast<int>((k / 16 + kSegBlocks - 1) / kSegBlocks);
   const int64_t grid_rows = layout == NVFP4_SF_TCGEN05 ? round_up(rows, 128) : rows;
   const bool empty = grid_rows == 0 || segs == 0;   // nothing to quantize: still publish g (from the given amax)
-  const dim3 grid = empty ? dim3(1, 1) : dim3(static_cast<unsigned>(grid_rows), segs);
+  // two rows per CTA for the rounded-to-nearest pass; the stochastic pass,
+  // which needs twice the registers for two rows, takes one
+  const int per_cta = stochastic ? 1 : kQuantRows;
+  const dim3 grid = empty ? dim3(1, 1) : dim3(static_cast<unsigned>((grid_rows + per_cta - 1) / per_cta), segs);
   const int ir = empty ? 0 : static_cast<int>(rows), ik = empty ? 0 : static_cast<int>(k);
   const bool tc = !empty && layout == NVFP4_SF_TCGEN05;
   const bool wide = !empty && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
