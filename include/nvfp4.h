@@ -334,17 +334,39 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M,
                                 void* y_bf16, int64_t ldy, nvfp4_stream_t stream);
 
 /*
- * Long-K GEMM whose A operand arrives in bf16: A [M, K] (pitch lda) is
- * quantized to NVFP4 with the nvfp4_quantize rule (tensor amax first), then
- * multiplied by pre-quantized B as in nvfp4_gemm.
- * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_QUANT_A, M, N, K) bytes
- *   (A codes, A scales, g_a, amax_a).
+ * GEMM whose A operand arrives in bf16 (an activation): A [M, K] (pitch lda)
+ * is quantized to NVFP4 with the nvfp4_quantize rule (tensor amax first),
+ * then multiplied by pre-quantized B as in nvfp4_gemm ("NVIDIA NVFP4 与
+ * Micro-Scaling" section 三: activations quantized with a per-tensor global
+ * scale and per-block micro-scales, then the block-scaled product).
+ *   When M > 128, N > 128 and B's codes (N * K / 2 bytes) are at most 64 MiB,
+ *   one kernel does both after the amax pass: extra warps quantize A row by
+ *   row while the tensor cores multiply the row blocks already done.  Other
+ *   shapes run the quantize pass and the GEMM as two kernels.  Both give the
+ *   same codes, scales, g_a and D bit for bit.
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_QUANT_A, M, N, K) bytes:
+ *   A's codes [M, K/2] at byte 0, A's tensor-core scales from
+ *   round_up(M * K / 2, 256), then g_a (fp32) at the next 256-byte boundary,
+ *   amax_a 16 bytes after it and row-block counters from byte 64 there,
+ *   which the call zeroes itself.  It needs no clearing; calls sharing a
+ *   workspace must not overlap.
  * K % 64 == 0.
  */
 NVFP4_API nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,
                                 const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
                                 nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
                                 nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm_quant_a with A's tensor amax already on the device: amax_dev
+ * (one fp32, read-only) holds max |A|, e.g. from nvfp4_amax on the same A
+ * earlier on the stream; the call skips its own amax pass.  Null amax_dev:
+ * NVFP4_ERR_INVALID_ARG.  Everything else as nvfp4_gemm_quant_a.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_quant_a_amax(const void* a_bf16, int64_t lda, const float* amax_dev,
+                                const void* b_codes, const void* b_sf_tc, const float* g_b_dev, int64_t M,
+                                int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out_dtype,
+                                void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 
 /*
  * Synchronises the stream, then returns and clears the device status word of

@@ -115,6 +115,10 @@ nvfp4_status check_bf16_input(const void* x, int64_t rows, int64_t k, int64_t ld
   return NVFP4_OK;
 }
 
+// Scalar tail of the quantize-and-multiply workspace: g_a, the amax and one
+// 32-bit counter per 256-row block of A from byte 64.
+size_t quant_a_scalar_bytes(int64_t M) { return static_cast<size_t>(round_up(64 + 4 * ((M + 255) / 256), 256)); }
+
 }  // namespace
 
 extern "C" {
@@ -346,7 +350,7 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
   if (op == NVFP4_OP_GEMM_QUANT_A) {
     const size_t codes = static_cast<size_t>(round_up(M * (K / 2), 256));
     const size_t sf = static_cast<size_t>(round_up(nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05), 256));
-    return codes + sf + 256;
+    return codes + sf + quant_a_scalar_bytes(M);
   }
   return 0;
 }
@@ -367,10 +371,18 @@ nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t ldx, cons
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
-nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,
-                                const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
-                                nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
-                                nvfp4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Quantize a bf16 A and multiply (amax_given: A's amax already on the device;
+// else computed into the workspace).  Workspace: A's codes, A's tensor-core
+// scales, then the scalars (g_a at byte 0, amax at byte 16) and the
+// quantize-and-GEMM kernel's row-block counters from byte 64.
+nvfp4_status gemm_quant_a_common(const void* a_bf16, int64_t lda, const float* amax_given, const void* b_codes,
+                                 const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d,
+                                 int64_t ldd, nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
+                                 nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(a_bf16, M, K, lda);
   if (st != NVFP4_OK) return st;
   if (!workspace) return NVFP4_ERR_INVALID_ARG;
@@ -381,9 +393,10 @@ nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_c
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* a_codes = ws;
   uint8_t* a_sf = ws + round_up(M * (K / 2), 256);
-  float* scal = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05), 256));
-  float* g_a = scal;
-  float* amax_a = scal + 4;
+  uint8_t* scal_bytes = a_sf + round_up(nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05), 256);
+  float* g_a = reinterpret_cast<float*>(scal_bytes);
+  float* amax_ws = reinterpret_cast<float*>(scal_bytes + 16);
+  int* counters = reinterpret_cast<int*>(scal_bytes + 64);
   st = check_gemm_operands(a_codes, a_sf, g_a, b_codes, b_sf_tc, g_b_dev, M, N, K, d);
   if (st != NVFP4_OK) return st;
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
@@ -391,10 +404,46 @@ nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_c
   if ((reinterpret_cast<uintptr_t>(d) & (out_dtype == NVFP4_OUT_F32 ? 3u : 1u)) != 0) return NVFP4_ERR_MISALIGNED;
   if ((st = check_arch()) != NVFP4_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if ((st = launch_amax(a_bf16, M, K, lda, amax_a, s)) != NVFP4_OK) return st;
-  if ((st = launch_quantize(a_bf16, M, K, lda, a_codes, a_sf, NVFP4_SF_TCGEN05, g_a, amax_a, s)) != NVFP4_OK)
+  const bool fused = quant_a_fusable(M, N, K);
+  const float* amax = amax_given ? amax_given : amax_ws;
+  if (fused) {
+    // zero the row-block counters (and the amax when this call computes it) in one memset
+    const size_t first = amax_given ? 64 : 16;
+    const size_t end = 64 + 4 * static_cast<size_t>((M + 255) / 256);
+    cudaError_t e = cudaMemsetAsync(scal_bytes + first, 0, end - first, s);
+    if (e != cudaSuccess) return launch_status(e);
+    // the quantizers take the first rows first: leave those in L2
+    if (!amax_given && (st = launch_amax_reversed(a_bf16, M, K, lda, amax_ws, s)) != NVFP4_OK) return st;
+  } else if (!amax_given && (st = launch_amax(a_bf16, M, K, lda, amax_ws, s)) != NVFP4_OK) {
+    return st;
+  }
+  if (fused)
+    return launch_gemm_quant_a_fused(a_bf16, lda, amax, a_codes, a_sf, g_a, counters, b_codes, b_sf_tc, g_b_dev, M,
+                                     N, K, d, ldd, out_dtype, s);
+  if ((st = launch_quantize(a_bf16, M, K, lda, a_codes, a_sf, NVFP4_SF_TCGEN05, g_a, amax, s)) != NVFP4_OK)
     return st;
   return launch_gemm(a_codes, a_sf, g_a, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,
+                                const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                                nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
+                                nvfp4_stream_t stream) {
+  return gemm_quant_a_common(a_bf16, lda, nullptr, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype, workspace,
+                             ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_quant_a_amax(const void* a_bf16, int64_t lda, const float* amax_dev, const void* b_codes,
+                                     const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K,
+                                     void* d, int64_t ldd, nvfp4_out_dtype out_dtype, void* workspace,
+                                     size_t ws_bytes, nvfp4_stream_t stream) {
+  if (!amax_dev) return NVFP4_ERR_INVALID_ARG;
+  return gemm_quant_a_common(a_bf16, lda, amax_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype,
+                             workspace, ws_bytes, stream);
 }
 
 nvfp4_status nvfp4_check_device_status(nvfp4_stream_t stream) {

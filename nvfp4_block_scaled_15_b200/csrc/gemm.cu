@@ -106,6 +106,19 @@ struct GemmParams {
   float* amax_d;    // max |alpha acc| over D, or null
   uint64_t wait_limit_ns;
   int* status;
+  // Quantize-and-GEMM kernel only: A arrives as bf16 rows (qa_x, pitch
+  // qa_ldx elements; qa_wide: 32-B aligned blocks) and is quantized in the
+  // kernel into qa_codes / qa_sf (tensor-core layout) with the global scale
+  // from qa_amax (also written to qa_g); qa_ready holds one counter per
+  // 256-row block of A, zero at launch: the rows of the block quantized.
+  const uint16_t* qa_x;
+  int64_t qa_ldx;
+  int qa_wide;
+  uint8_t* qa_codes;
+  uint8_t* qa_sf;
+  float* qa_g;
+  const float* qa_amax;
+  int* qa_ready;
 };
 
 __host__ __device__ __forceinline__ int round_up_int(int a, int b) { return (a + b - 1) / b * b; }
@@ -473,6 +486,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, kMx>::THREADS, 1)
 // the scale copies and MMAs for both; both CTAs' loads complete on the
 // leader's "full" barriers, and its commits arrive on both CTAs' barriers.
 // ---------------------------------------------------------------------------
+// Quantize-and-GEMM kernel: warps that quantize A, and the 16-element blocks
+// each lane takes per unit of work (a unit: 32 x QA_BLOCKS blocks of a row).
+constexpr int QA_WARPS = 4;
+constexpr int QA_BLOCKS = 8;
+constexpr int QA_UNIT_BLOCKS = 32 * QA_BLOCKS;
+
 template <bool kMx>
 struct PairCfg {
   using F = ScaleFmt<kMx>;
@@ -501,16 +520,101 @@ struct PairCfg {
   static constexpr int EPI_BOX_BYTES = 32 * EPI_BOX_COLS * 2;
   static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BOX_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 256 + 1024;
+  // Quantize-and-GEMM kernel: QA_WARPS more warps quantize A's rows; the
+  // E4M3 scale table takes 1 KB more.
+  static constexpr int THREADS_QA = THREADS + QA_WARPS * 32;
+  static constexpr int SMEM_BYTES_QA = SMEM_BYTES + 128 * 8;
   static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-B aligned");
   static_assert(TMEM_SF_BASE + SF_COLS <= (int)TMEM_COLS, "TMEM budget");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(SMEM_BYTES_QA <= 232448, "shared memory budget");
 };
+
+// Wait (bounded) until all units of 256-row block tm of A are quantized
+// (upr units per row), then order the TMA loads that follow after the
+// quantizers' stores.
+__device__ __forceinline__ bool wait_rows_quantized(const GemmParams& p, int tm, int rows_pad, int upr,
+                                                    volatile int* abort_flag) {
+  const int want = min(256, rows_pad - tm * 256) * upr;
+  const int* c = p.qa_ready + tm;
+  if (ld_acquire_gpu(c) < want) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(c) >= want) break;
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        *abort_flag = 1;
+        record_status(p.status, kDevTimeout);
+        return false;
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+// Units quantized at start-up, one per quantizer and epilogue warp of the
+// grid (the epilogue warps have nothing to drain before the first tile):
+// enough for the first row blocks the first tiles need.
+__device__ __forceinline__ int64_t qa_startup_units(int64_t units, int grid, int epi_warps) {
+  const int64_t h = static_cast<int64_t>(grid) * (QA_WARPS + epi_warps);
+  return units < h ? units : h;
+}
+
+// Quantizer warp: 16-element blocks b0 + 32 j (j < QA_BLOCKS) of A row r into
+// w (zeros past the row's end or for rows past M).
+__device__ __forceinline__ void qa_load(const GemmParams& p, int r, int b0, int kb, bool wide,
+                                        uint32_t (&w)[QA_BLOCKS][8]) {
+  const bool real = r < p.M;
+  const uint16_t* xr = p.qa_x + static_cast<int64_t>(r) * p.qa_ldx;
+#pragma unroll
+  for (int j = 0; j < QA_BLOCKS; ++j) {
+    const int b = b0 + 32 * j;
+    if (real && b < kb) {
+      load_bf16_block(xr + b * 16, w[j], wide);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[j][i] = 0u;
+    }
+  }
+}
+
+// Codes and scales of those blocks (the quantize pass's rule; all zero when
+// g is not finite); codes only for rows inside A, scales for every row of
+// the tensor-core layout.
+__device__ __forceinline__ void qa_quantize_store(const GemmParams& p, int r, int b0, int kb, float g, bool valid,
+                                                  const float2* table, const uint32_t (&w)[QA_BLOCKS][8]) {
+  const bool real = r < p.M;
+  uint8_t* cr = p.qa_codes + static_cast<int64_t>(r) * (p.K >> 1);
+  uint8_t* sr = p.qa_sf + static_cast<int64_t>(r >> 7) * (kb >> 2) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+#pragma unroll
+  for (int j = 0; j < QA_BLOCKS; j += 2) {
+    const int ba = b0 + 32 * j, bb = ba + 32;
+    uint2 ka, kb2;
+    uint32_t sa, sb;
+    quantize_two_blocks(w[j], w[j + 1], g, table, ka, kb2, sa, sb);
+    if (!valid) {
+      ka = kb2 = make_uint2(0u, 0u);
+      sa = sb = 0u;
+    }
+    if (ba < kb) {
+      if (real) *reinterpret_cast<uint2*>(cr + ba * 8) = ka;
+      sr[((ba >> 2) << 9) + (ba & 3)] = static_cast<uint8_t>(sa);
+    }
+    if (bb < kb) {
+      if (real) *reinterpret_cast<uint2*>(cr + bb * 8) = kb2;
+      sr[((bb >> 2) << 9) + (bb & 3)] = static_cast<uint8_t>(sb);
+    }
+  }
+}
 
 // kQ: the epilogue writes the quantized output (FP8 or NVFP4 under g_d)
 // instead of bf16 / fp32 D; a separate instantiation keeps the TMA-store
 // path's registers out of it.
-template <bool kMx, bool kQ>
-__global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
+// kQA: the quantize-and-GEMM kernel (bf16 A quantized by extra warps, tiles
+// taken in row-major order so the first tiles need only the first rows).
+template <bool kMx, bool kQ, bool kQA = false>
+__global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                      const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
@@ -527,6 +631,7 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
   uint64_t* mma_done = ovl_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* qa_table = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(full) + 256);   // kQA only
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -534,6 +639,7 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
+  if constexpr (kQA) fill_scale_table_from(qa_table, static_cast<int>(threadIdx.x), static_cast<int>(blockDim.x));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -564,12 +670,16 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
   cluster_sync_all();                         // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent of the amax pass: everything above
+  // overlapped its tail; nothing below runs before it has finished.
+  if constexpr (kQA) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int tiles_m = (p.M + 255) / 256;
   const int tiles_n = (p.N + C::BN - 1) / C::BN;
   const int num_tiles = tiles_m * tiles_n;
   const int num_kt = (p.K + BK - 1) / BK;
   const int ksteps_total = p.K / MMA_K;
+  const int rows_pad = round_up_int(p.M, 128);   // rows of A's tensor-core scale layout
 
   if (warp == 0) {
     // ------------------------- producer (both CTAs) -------------------------
@@ -578,11 +688,19 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
+      int ready_tm = -1;                        // kQA: A rows known quantized up to this row block
       for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
-        const int tm = t % tiles_m;
-        const int tn = t / tiles_m;
+        const int tm = kQA ? t / tiles_n : t % tiles_m;
+        const int tn = kQA ? t - tm * tiles_n : t / tiles_m;
         const int m_cta = tm * 256 + static_cast<int>(rank) * 128;
         const int n0 = tn * C::BN;
+        if constexpr (kQA) {
+          if (tm > ready_tm) {
+            if (!wait_rows_quantized(p, tm, rows_pad, (p.K / 16 + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS, abort_flag))
+              break;
+            ready_tm = tm;
+          }
+        }
         for (int kt = 0; kt < num_kt; ++kt) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
@@ -698,13 +816,39 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
       volatile int no_abort = 0;
       (void)mbar_wait_bounded(mma_done, 0, &no_abort, p.wait_limit_ns, p.status);
     }
-  } else {
+  } else if (!kQA || warp < 2 + C::EPI_WARPS) {
     // ------------------------- epilogue (both CTAs) -------------------------
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int half = ew >> 2;
     constexpr int HALF = C::BN / 2;
-    const float alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    float alpha;
+    if constexpr (kQA) {
+      // the g_a the quantizers use and publish: 0 when it is not finite
+      bool valid;
+      const float ga = global_scale_from_amax(*p.qa_amax, valid);
+      alpha = __fdiv_rn(1.0f, __fmul_rn(valid ? ga : 0.0f, *p.g_b));
+    } else {
+      alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
+    }
+    if constexpr (kQA) {
+      // start-up: this warp's unit of the first row blocks of A
+      bool valid;
+      const float g = global_scale_from_amax(*p.qa_amax, valid);
+      const int kb = p.K >> 4;
+      const int upr = (kb + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS;
+      const int64_t units = static_cast<int64_t>(rows_pad) * upr;
+      const int64_t u = static_cast<int64_t>(blockIdx.x) * (QA_WARPS + C::EPI_WARPS) + QA_WARPS + ew;
+      if (u < qa_startup_units(units, static_cast<int>(gridDim.x), C::EPI_WARPS)) {
+        const int r = static_cast<int>(u / upr), c0 = static_cast<int>(u % upr) * QA_UNIT_BLOCKS;
+        uint32_t w[QA_BLOCKS][8];
+        qa_load(p, r, c0 + lane, kb, p.qa_wide != 0, w);
+        qa_quantize_store(p, r, c0 + lane, kb, g, valid, qa_table, w);
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) red_release_add_gpu(p.qa_ready + (r >> 8), 1);
+      }
+    }
     const float gd = kQ ? *p.g_d : 0.0f;
     float amax_run = 0.0f;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
@@ -712,13 +856,67 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
     int j = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++j) {
       const int b = j & 1;
-      const int tm = t % tiles_m;
-      const int tn = t / tiles_m;
+      const int tm = kQA ? t / tiles_n : t % tiles_m;
+      const int tn = kQA ? t - tm * tiles_n : t / tiles_m;
       if (!mbar_wait_bounded(acc_full, static_cast<uint32_t>(j & 1), abort_flag, p.wait_limit_ns, p.status)) break;
       tc_fence_after();
       uint32_t v[HALF];
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (b ? C::ACC1_COL : 0) + half * HALF;
+      if constexpr (kQA) {
+        // 64 columns at a time (the quantizer warps take the registers a
+        // 128-column drain would hold), the columns shared with the other
+        // accumulator first; bf16 or fp32 D, no quantized output.
+        const bool shared_cols = (b == 0 && half == 1) || (b == 1 && half == 0);
+        const int first = (b == 0 && half == 1) ? 64 : 0;
+        const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quad * 32;
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {
+          const int c_off = part == 0 ? first : 64 - first;
+          uint32_t v[64];
+          tmem_ld_32x32b_x32(taddr + c_off, v);
+          tmem_ld_32x32b_x32(taddr + c_off + 32, v + 32);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (part == 0 && shared_cols) mbar_arrive_cluster_relaxed(ovl_free_leader);
+            if (part == 1) mbar_arrive_cluster_relaxed(acc_empty_leader + 8u * b);
+          }
+          const int col0 = tn * C::BN + half * HALF + c_off;
+          if (p.tma_store) {
+            if (row0 < p.M) {
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                if (col0 + cc * C::EPI_BOX_COLS >= p.N) break;
+                const int box_id = c_off / C::EPI_BOX_COLS + cc;     // staging buffers alternate by box
+                uint8_t* box = epi_smem + (ew * 2 + (box_id & 1)) * C::EPI_BOX_BYTES;
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const uint32_t* f = v + cc * C::EPI_BOX_COLS + q * 8;
+                  uint4 wv;
+                  wv.x = pack_bf16x2(__uint_as_float(f[0]) * alpha, __uint_as_float(f[1]) * alpha);
+                  wv.y = pack_bf16x2(__uint_as_float(f[2]) * alpha, __uint_as_float(f[3]) * alpha);
+                  wv.z = pack_bf16x2(__uint_as_float(f[4]) * alpha, __uint_as_float(f[5]) * alpha);
+                  wv.w = pack_bf16x2(__uint_as_float(f[6]) * alpha, __uint_as_float(f[7]) * alpha);
+                  *reinterpret_cast<uint4*>(box + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = wv;
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_2d(&tmD, box, col0 + cc * C::EPI_BOX_COLS, row0);
+                  bulk_commit_group();
+                }
+              }
+            }
+          } else if (col0 < p.N) {
+            store_row<64>(p, row0 + lane, col0, v, alpha);
+          }
+        }
+        continue;
+      }
       // The shared columns [256-OVL, 256) are the last OVL of accumulator 0
       // (held by half 1) and the first OVL of accumulator 1 (held by half 0).
       if (b == 0 && half == 1) {
@@ -787,6 +985,49 @@ __global__ void __launch_bounds__(PairCfg<kMx>::THREADS, 1)
     }
     if (!kQ && p.tma_store && lane == 0) bulk_wait_group<0>();
     if constexpr (kQ) publish_amax(p, amax_run);
+  } else if constexpr (kQA) {
+    // ------------------- A quantizers (quantize-and-GEMM) -------------------
+    // Units (row r, blocks c * QA_UNIT_BLOCKS ..) numbered row-major and
+    // taken in order (a start-up unit, then every nqw-th), so the row blocks
+    // complete roughly first to last, the order the row-major tiles need them.  Each unit: the quantize pass's rule (block
+    // scales RN_e4m3(RN(RN(amax_b g) / 6)), codes RN_e2m1(RN(RN(x g) / s)));
+    // rows past M (up to the 128-row group) get zero scales.  After a unit
+    // the warp counts it on its row block's counter with release semantics.
+    const int qw = warp - (2 + C::EPI_WARPS);
+    bool valid;
+    const float g = global_scale_from_amax(*p.qa_amax, valid);
+    if (blockIdx.x == 0 && qw == 0 && lane == 0) {
+      *p.qa_g = valid ? g : 0.0f;
+      if (!valid) record_status(p.status, kDevRange);
+    }
+    const int kb = p.K >> 4;
+    const int upr = (kb + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS;   // units per row
+    const int64_t units = static_cast<int64_t>(rows_pad) * upr;
+    const int nqw = static_cast<int>(gridDim.x) * QA_WARPS;
+    const bool wide = p.qa_wide != 0;
+    // Pipelined over units: the next unit's loads go out before this one is
+    // published, so the release waits while they are in flight.
+    // Units [0, S) are the start-up units, one per quantizer and epilogue
+    // warp; this warp then takes S + gw, S + gw + nqw, ...
+    const int64_t S = qa_startup_units(units, static_cast<int>(gridDim.x), C::EPI_WARPS);
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * QA_WARPS + qw;
+    uint32_t w[QA_BLOCKS][8];
+    int64_t u = static_cast<int64_t>(blockIdx.x) * (QA_WARPS + C::EPI_WARPS) + qw;
+    if (u >= S) u = S + gw;
+    int r = static_cast<int>(u / upr), c0 = static_cast<int>(u % upr) * QA_UNIT_BLOCKS;
+    if (u < units) qa_load(p, r, c0 + lane, kb, wide, w);
+    while (u < units && !*abort_flag) {
+      qa_quantize_store(p, r, c0 + lane, kb, g, valid, qa_table, w);
+      const int64_t un = u < S ? S + gw : u + nqw;
+      const int rn = static_cast<int>(un / upr), cn = static_cast<int>(un % upr) * QA_UNIT_BLOCKS;
+      if (un < units) qa_load(p, rn, cn + lane, kb, wide, w);
+      fence_proxy_async_global();   // the unit's bytes are read next by TMA loads
+      __syncwarp();
+      if (lane == 0) red_release_add_gpu(p.qa_ready + (r >> 8), 1);
+      u = un;
+      r = rn;
+      c0 = cn;
+    }
   }
 
   __syncwarp();
@@ -845,10 +1086,18 @@ void set_quant_out(GemmParams& p, const QuantOut* q, int64_t N) {
   p.amax_d = q->amax_d;
 }
 
+// In-kernel quantization of a bf16 A (the quantize-and-GEMM kernel).
+struct QuantA {
+  const void* x;
+  int64_t ldx;
+  const float* amax;
+  int* counters;
+};
+
 template <bool kMx>
 nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                            const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
-                           nvfp4_out_dtype out, const QuantOut* q, cudaStream_t s) {
+                           nvfp4_out_dtype out, const QuantOut* q, cudaStream_t s, const QuantA* qa = nullptr) {
   using C = PairCfg<kMx>;
   using F = typename C::F;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
@@ -886,35 +1135,54 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
   if (!p.status) return NVFP4_ERR_CUDA;
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmParams) =
       gemm_pair_kernel<kMx, false>;
+  int threads = C::THREADS, smem = C::SMEM_BYTES;
   if constexpr (!kMx) {
     if (p.out_q) kern = gemm_pair_kernel<false, true>;
+    if (qa) {
+      if (p.out_q) return NVFP4_ERR_INVALID_ARG;
+      kern = gemm_pair_kernel<false, false, true>;
+      threads = C::THREADS_QA;
+      smem = C::SMEM_BYTES_QA;
+      p.qa_x = static_cast<const uint16_t*>(qa->x);
+      p.qa_ldx = qa->ldx;
+      p.qa_wide = (reinterpret_cast<uintptr_t>(qa->x) & 31u) == 0 && (qa->ldx % 16) == 0;
+      p.qa_codes = static_cast<uint8_t*>(const_cast<void*>(a_codes));
+      p.qa_sf = static_cast<uint8_t*>(const_cast<void*>(a_sf));
+      p.qa_g = const_cast<float*>(g_a);
+      p.qa_amax = qa->amax;
+      p.qa_ready = qa->counters;
+    }
   }
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return launch_status(e);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  // the quantize-and-GEMM kernel is a programmatic dependent of the amax pass
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = qa ? 2 : 1;
   // as many resident pairs as the device holds at once, never more than tiles
-  static int max_pairs[64] = {0};
+  static int max_pairs[2][64] = {{0}};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return launch_status(cudaGetLastError());
-  if (dev < 64 && max_pairs[dev] == 0) {
+  int* mp = &max_pairs[qa ? 1 : 0][dev < 64 ? dev : 0];
+  if (dev >= 64 || *mp == 0) {
     cfg.gridDim = dim3(2 * (device_sm_count() / 2));
     int clusters = 0;
     e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
     if (e != cudaSuccess || clusters < 1) return launch_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
-    max_pairs[dev] = clusters;
+    *mp = clusters;
   }
   const int tiles = p.tiles_m * p.tiles_n;
-  const int pairs = tiles < max_pairs[dev < 64 ? dev : 0] ? tiles : max_pairs[dev < 64 ? dev : 0];
+  const int pairs = tiles < *mp ? tiles : *mp;
   cfg.gridDim = dim3(2 * pairs);
   e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmSFA, tmSFB, tmD, p);
   return launch_status(e);
@@ -981,6 +1249,21 @@ nvfp4_status launch_gemm_q(const void* a_codes, const void* a_sf, const float* g
     if (e != cudaSuccess) return launch_status(e);
   }
   return dispatch_gemm<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd_bytes, NVFP4_OUT_BF16, &q, s);
+}
+
+// The quantize-and-GEMM kernel takes its tiles row block by row block, so a
+// row block's tiles read all of B's codes: it is used where those stay in L2
+// (and where the CTA-pair kernel would run at all: M, N > 128).
+bool quant_a_fusable(int64_t M, int64_t N, int64_t K) {
+  return M > 128 && N > 128 && N * (K / 2) <= (int64_t{64} << 20);
+}
+
+nvfp4_status launch_gemm_quant_a_fused(const void* a_bf16, int64_t lda, const float* amax_dev, void* a_codes,
+                                       void* a_sf, float* g_a, int* counters, const void* b_codes,
+                                       const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K,
+                                       void* d, int64_t ldd, nvfp4_out_dtype out, cudaStream_t s) {
+  const QuantA qa{a_bf16, lda, amax_dev, counters};
+  return run_gemm_pair<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, nullptr, s, &qa);
 }
 
 nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,

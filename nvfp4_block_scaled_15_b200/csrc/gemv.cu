@@ -390,12 +390,6 @@ struct GemvFusedParams {
   int* status;
 };
 
-__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Count this contributor's arrival on a tagged counter; returns the number
 // of earlier arrivals of the same call (0 or 1).
 __device__ __forceinline__ int tagged_arrive(unsigned long long* c, uint32_t tag) {
@@ -892,9 +886,17 @@ static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
 
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) { return gemv_ws_layout(M, N, K).total; }
 
-// Tags of the prologue-free GEMV's fix-up counters: unique per call within
-// the process (never 0, so a zeroed counter is never taken for this call's).
-static std::atomic<uint32_t> g_gemv_tag{0};
+// Tags of the prologue-free GEMV's fix-up counters in a caller's workspace:
+// unique per launch within the process and never 0, so a zeroed counter, or
+// one left by an earlier launch in the same workspace, is never taken for
+// this launch's.
+static std::atomic<uint32_t> g_launch_tag{0};
+
+uint32_t next_launch_tag() {
+  uint32_t tag = g_launch_tag.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (tag == 0) tag = g_launch_tag.fetch_add(1, std::memory_order_relaxed) + 1;   // skip 0 on wrap
+  return tag;
+}
 
 static nvfp4_status launch_gemv_fused(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
                                       const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy,
@@ -910,9 +912,7 @@ static nvfp4_status launch_gemv_fused(const void* x, int64_t M, int64_t ldx, con
   p.g_w = g_w;
   p.partials = reinterpret_cast<float*>(base + L.part);
   p.counters = reinterpret_cast<unsigned long long*>(base + L.cnt);
-  uint32_t tag = g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1;
-  if (tag == 0) tag = g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1;   // skip 0 on wrap
-  p.tag = tag;
+  p.tag = next_launch_tag();
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ldy = ldy;
   p.M = static_cast<int>(M);

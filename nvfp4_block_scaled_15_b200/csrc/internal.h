@@ -30,6 +30,11 @@ inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
 // Launchers implemented in the .cu files (arguments already validated).
 nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s);
+// The amax pass taking rows last to first (so the first rows are the ones
+// still in L2 afterwards), for a consumer that reads them first to last.  It
+// does not clear *amax_dev: the caller zeroes it first.
+nvfp4_status launch_amax_reversed(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev,
+                                  cudaStream_t s);
 nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,
                              nvfp4_sf_layout layout, float* g_dev, const float* amax_dev, cudaStream_t s);
 // Quantize pass with stochastic rounding of the codes (Philox4x32-10 bits).
@@ -64,11 +69,23 @@ struct QuantOut {
 nvfp4_status launch_gemm_q(const void* a_codes, const void* a_sf, const float* g_a, const void* b_codes,
                            const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* d,
                            int64_t ldd_bytes, const QuantOut& q, cudaStream_t s);
+// One kernel that quantizes a bf16 A (global scale from amax_dev, computed
+// by an earlier pass on the stream) into codes / tensor-core scales / g_a and
+// runs the block-scaled GEMM on them as the rows become ready.  counters:
+// ceil(M / 256) int row-block counters, zero when the kernel starts.  Only for
+// shapes quant_a_fusable() accepts.
+bool quant_a_fusable(int64_t M, int64_t N, int64_t K);
+nvfp4_status launch_gemm_quant_a_fused(const void* a_bf16, int64_t lda, const float* amax_dev, void* a_codes,
+                                       void* a_sf, float* g_a, int* counters, const void* b_codes,
+                                       const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K,
+                                       void* d, int64_t ldd, nvfp4_out_dtype out, cudaStream_t s);
 nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,
                             int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out,
                             cudaStream_t s);
 nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
                          const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s);
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// Per-launch tag of workspace counters (never 0).
+uint32_t next_launch_tag();
 
 }  // namespace nvfp4

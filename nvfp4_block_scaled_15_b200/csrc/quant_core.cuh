@@ -33,6 +33,24 @@ __device__ __forceinline__ uint32_t abs_max_bits8(const uint4 v) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
+// One 16-element bf16 block (32 B, 16-B aligned) as 8 words, read once and
+// not kept in L1: one 256-bit load when it is 32-B aligned (wide), else two
+// 128-bit loads.
+__device__ __forceinline__ void load_bf16_block(const uint16_t* p, uint32_t (&w)[8], bool wide) {
+  if (wide) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+  } else {
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p + 8));
+  }
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

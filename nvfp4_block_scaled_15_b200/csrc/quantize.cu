@@ -30,6 +30,8 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 }
 
 // Pass 1: max |x|.  grid.x strides over rows, grid.y over row segments.
+// kReversed: rows are taken last to first.
+template <bool kReversed>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                         int64_t ldx, unsigned* __restrict__ amax_bits) {
   // the quantize pass (a programmatic dependent) may take SMs as these CTAs leave
@@ -37,7 +39,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
   const int chunks = k >> 3;
   const int c0 = blockIdx.y * kSegChunks + threadIdx.x;
   uint32_t m = 0;
-  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+  for (int i = blockIdx.x; i < rows; i += gridDim.x) {
+    const int r = kReversed ? rows - 1 - i : i;
     const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ldx);
     uint4 v[kUnroll];
 #pragma unroll
@@ -647,16 +650,30 @@ float hadamard_norm(int n) { return static_cast<float>(1.0 / std::sqrt(static_ca
 
 }  // namespace
 
-nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(amax_dev, 0, sizeof(float), s);
-  if (e != cudaSuccess) return launch_status(e);
+template <bool kReversed>
+static nvfp4_status run_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s,
+                             bool clear) {
+  if (clear) {
+    cudaError_t e = cudaMemsetAsync(amax_dev, 0, sizeof(float), s);
+    if (e != cudaSuccess) return launch_status(e);
+  }
   if (rows == 0 || k == 0) return NVFP4_OK;
   const int segs = static_cast<int>((k / 8 + kSegChunks - 1) / kSegChunks);
   const int64_t want = static_cast<int64_t>(device_sm_count()) * 8 / segs;
   const int gx = static_cast<int>(rows < want ? rows : (want > 0 ? want : 1));
-  amax_kernel<<<dim3(gx, segs), kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
-                                                  static_cast<int>(k), ldx, reinterpret_cast<unsigned*>(amax_dev));
+  amax_kernel<kReversed><<<dim3(gx, segs), kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<int>(rows),
+                                                             static_cast<int>(k), ldx,
+                                                             reinterpret_cast<unsigned*>(amax_dev));
   return launch_status(cudaGetLastError());
+}
+
+nvfp4_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev, cudaStream_t s) {
+  return run_amax<false>(x, rows, k, ldx, amax_dev, s, true);
+}
+
+nvfp4_status launch_amax_reversed(const void* x, int64_t rows, int64_t k, int64_t ldx, float* amax_dev,
+                                  cudaStream_t s) {
+  return run_amax<true>(x, rows, k, ldx, amax_dev, s, false);
 }
 
 nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx, void* codes, void* sf,

@@ -58,6 +58,8 @@ _SIGS = {
     "nvfp4_workspace_bytes": ([_i32, _i64, _i64, _i64], _sz),
     "nvfp4_gemv_batched": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _sz, _vp], _i32),
     "nvfp4_gemm_quant_a": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp], _i32),
+    "nvfp4_gemm_quant_a_amax": ([_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp],
+                                _i32),
     "nvfp4_gemv_batched_noalloc": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp], _i32),
     "nvfp4_mxfp4_sf_bytes": ([_i64, _i64, _i32], _sz),
     "nvfp4_mxfp4_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
@@ -187,6 +189,12 @@ def nvfp4_gemm_quant_a(a, lda, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, w
                        stream=None) -> None:
     _check(_lib.nvfp4_gemm_quant_a(_p(a), lda, _p(b_codes), _p(b_sf), _p(g_b), m, n, k, _p(d), ldd, out_dtype,
                                    _p(workspace), ws_bytes, _s(stream)), "nvfp4_gemm_quant_a")
+
+
+def nvfp4_gemm_quant_a_amax(a, lda, amax, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, workspace, ws_bytes,
+                            stream=None) -> None:
+    _check(_lib.nvfp4_gemm_quant_a_amax(_p(a), lda, _p(amax), _p(b_codes), _p(b_sf), _p(g_b), m, n, k, _p(d), ldd,
+                                        out_dtype, _p(workspace), ws_bytes, _s(stream)), "nvfp4_gemm_quant_a_amax")
 
 
 def nvfp4_mxfp4_sf_bytes(rows: int, k: int, layout: int) -> int:
@@ -337,15 +345,32 @@ def gemv_batched(x: torch.Tensor, w: Quantized, out: torch.Tensor | None = None,
 
 
 def gemm_quant_a(a: torch.Tensor, b: Quantized, out_dtype=torch.bfloat16, out=None, workspace=None,
-                 stream=None) -> torch.Tensor:
+                 stream=None, amax: torch.Tensor | None = None) -> torch.Tensor:
+    """D = A_q @ B_q^T with a bf16 A quantized inside the call; amax: A's tensor
+    amax already on the device (1-element fp32), which skips the amax pass."""
     m, k = a.shape
     n = b.rows
     ws_bytes = nvfp4_workspace_bytes(OP_GEMM_QUANT_A, m, n, k)
     ws = workspace if workspace is not None else torch.empty(ws_bytes, dtype=torch.uint8, device=a.device)
     od = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
     d = out if out is not None else torch.empty((m, n), dtype=out_dtype, device=a.device)
-    nvfp4_gemm_quant_a(a, a.stride(0), b.codes, b.sf, b.g, m, n, k, d, d.stride(0), od, ws, ws.numel(), stream)
+    if amax is None:
+        nvfp4_gemm_quant_a(a, a.stride(0), b.codes, b.sf, b.g, m, n, k, d, d.stride(0), od, ws, ws.numel(), stream)
+    else:
+        nvfp4_gemm_quant_a_amax(a, a.stride(0), amax, b.codes, b.sf, b.g, m, n, k, d, d.stride(0), od, ws,
+                                ws.numel(), stream)
     return d
+
+
+def quant_a_workspace_views(ws: torch.Tensor, m: int, k: int):
+    """A's codes [m, k/2], its tensor-core scales and g_a (1-element fp32) inside a
+    gemm_quant_a workspace (the layout include/nvfp4.h states)."""
+    codes_bytes = m * (k // 2)
+    sf_off = (codes_bytes + 255) // 256 * 256
+    sf_bytes = nvfp4_sf_bytes(m, k, SF_TCGEN05)
+    g_off = sf_off + (sf_bytes + 255) // 256 * 256
+    return (ws[:codes_bytes].view(m, k // 2), ws[sf_off:sf_off + sf_bytes],
+            ws[g_off:g_off + 4].view(torch.float32))
 
 
 class MXQuantized:
