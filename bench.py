@@ -3,13 +3,14 @@
 
 One step = the prefill linear-layer path on the 8192 x 8192 x 8192 workload
 (activations bf16 [8192, 8192] N(0,1) with 0.5% outlier channels x30,
-weights N(0, 0.02)): quantize the activations (amax pass + quantize pass,
-scales written in the tensor-core layout) and run the block-scaled GEMM
-against the pre-quantized weights, bf16 output.  value = 2*M*N*K per step
+weights N(0, 0.02)): quantize the activations and run the block-scaled GEMM
+against the pre-quantized weights, bf16 output: the amax pass, then one
+kernel whose extra warps quantize A (scales in the tensor-core layout) row
+block by row block while its tensor cores multiply the blocks already done.  value = 2*M*N*K per step
 over the device time of the step, summed over ranks (weak scaling: every
 rank runs its own replica; the path needs no exchange).
 
-Also reported on rank 0: the GEMM kernel's roofline (live CUDA events),
+Also reported on rank 0: that kernel's roofline (live CUDA events),
 end-to-end throughput through host buffers and SM clocks during the timed
 region; at N = 1 also the quantize-bandwidth, rotated and stochastic
 quantize, decode-GEMV, long-K, MXFP4 and requantizing-GEMM workloads, and
@@ -53,7 +54,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/GEMV/long-K sub-benchmarks")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--part", choices=["quantize", "hadamard", "stochastic", "gemv", "longk", "gemm", "mxquantize", "mxgemm", "requant"],
+    ap.add_argument("--part", choices=["quantize", "hadamard", "stochastic", "gemv", "longk", "gemm", "quantgemm",
+                                       "mxquantize", "mxgemm", "requant"],
                     default=None,
                     help="run one workload alone, --steps times (for profiling); prints its timing")
     return ap.parse_args()
@@ -250,8 +252,9 @@ def run_reference(args, rank):
 
 
 def config_block(n_gpus):
-    return {"workload": "prefill GEMM 8192x8192x8192: activation quantize (amax + quantize, tcgen05 scale "
-                        "layout) + block-scaled NVFP4 GEMM, weights pre-quantized, bf16 out",
+    return {"workload": "prefill GEMM 8192x8192x8192: activation quantize (amax pass, then quantization "
+                        "inside the GEMM kernel, tcgen05 scale layout) + block-scaled NVFP4 GEMM, weights "
+                        "pre-quantized, bf16 out",
             "M": M, "N": N, "K": K, "activations": "bf16 N(0,1), 0.5% outlier channels x30, seed 4",
             "weights": "bf16 N(0,0.02), seed 5", "l2": "flushed before every step (256 MiB write)",
             "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"}
@@ -303,16 +306,23 @@ def main():
     qw = nv.quantize(w, nv.SF_TCGEN05)
     qa = nv.empty_quantized(M, K, nv.SF_TCGEN05, dev)
     d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws_bytes = nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, M, N, K)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        nv.quantize(a, nv.SF_TCGEN05, out=qa)
-        nv.gemm(qa, qw, out=d)
+    # The step: A's amax pass (prepare), then the quantize-and-GEMM kernel
+    # (run), an event between them so the kernel is timed on its own.
+    def prepare():
+        nv.nvfp4_gemm_quant_a_prepare(a, K, M, N, K, ws, ws_bytes)
+
+    def run():
+        nv.nvfp4_gemm_quant_a_run(a, K, qw.codes, qw.sf, qw.g, M, N, K, d, N, nv.OUT_BF16, ws, ws_bytes)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
-        step()
+        prepare()
+        run()
     torch.cuda.synchronize(dev)
     assert nv.nvfp4_check_device_status() == nv.OK
 
@@ -326,9 +336,9 @@ def main():
     for e0, e1, e2 in ev:
         flush.zero_()
         e0.record(stream)
-        nv.quantize(a, nv.SF_TCGEN05, out=qa)
+        prepare()
         e1.record(stream)
-        nv.gemm(qa, qw, out=d)
+        run()
         e2.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -337,8 +347,8 @@ def main():
     sampler.stop()
     status = nv.nvfp4_check_device_status()
     step_ms = [e0.elapsed_time(e2) for e0, e1, e2 in ev]
-    quant_ms = [e0.elapsed_time(e1) for e0, e1, e2 in ev]
-    gemm_ms = [e1.elapsed_time(e2) for e0, e1, e2 in ev]
+    amax_ms = [e0.elapsed_time(e1) for e0, e1, e2 in ev]
+    fused_ms = [e1.elapsed_time(e2) for e0, e1, e2 in ev]
     ms = statistics.mean(step_ms)
     if world > 1:
         ms = max_over_ranks(ms, dist, dev)
@@ -347,35 +357,47 @@ def main():
     # end to end through the public API with pinned host buffers
     e2e = None
     if rank == 0:
-        e2e = bench_e2e(nv, torch, dev, a_bits, qw, qa, min(args.steps, 30))
+        e2e = bench_e2e(nv, torch, dev, a_bits, qw, min(args.steps, 30))
 
     result = None
     if rank == 0:
-        gemm_avg = statistics.mean(gemm_ms)
-        achieved = FLOPS_STEP / (gemm_avg * 1e-3) / 1e12
-        traffic = profile_traffic("gemm_prefill_8192.md", GEMM_SOURCES)
+        fused_avg = statistics.mean(fused_ms)
+        achieved = FLOPS_STEP / (fused_avg * 1e-3) / 1e12
+        traffic = profile_traffic("quant_gemm_prefill_8192.md", GEMM_SOURCES)
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic", "config": config_block(world),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp4_peak, "traffic": traffic,
-                         "kernel": "gemm_pair_kernel (tcgen05.mma.cta_group::2 kind::mxf4nvf4, 256x256 tiles, 8192^3)",
+                         "kernel": "gemm_pair_kernel<quantize A> (extra warps quantize the bf16 A row block by "
+                                   "row block; tcgen05.mma.cta_group::2 kind::mxf4nvf4, 256x256 tiles, 8192^3)",
                          "peak_source": f"{peaks_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} "
                                         "(nominal FP4:BF16 dense ratio)",
-                         "algorithmic": "2*M*N*K = 1.0995e12 FLOP per launch"},
+                         "algorithmic": "2*M*N*K = 1.0995e12 FLOP per launch (the quantization of A inside the "
+                                        "kernel is not counted)"},
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 2 * args.steps,
             "clocks": sampler.summary(t0, t1),
             "wall_ms_per_step": (t1 - t0) * 1e3 / args.steps,
-            "step_breakdown_ms": {"quantize_activations": statistics.mean(quant_ms), "gemm": gemm_avg},
+            "step_breakdown_ms": {"amax_pass": statistics.mean(amax_ms), "quantize_and_gemm": fused_avg},
             "device_status": nv.nvfp4_status_string(status),
         }
     if rank == 0 and parts_inputs is not None:
         parts_inputs["prefill"] = (a, w)
         result["parts"] = bench_parts(nv, torch, dev, flush, parts_inputs, hbm_peak, fp4_peak, peaks_src)
-        result["parts"]["gemm_only"] = {"tflops": result["roofline"]["achieved"],
-                                        "frac_fp4_peak": result["roofline"]["frac"]}
+        # the same step as two kernels after the amax pass (quantize pass, then
+        # the plain GEMM), and the plain GEMM alone
+        ms_q = _timed(torch, dev, flush, lambda: nv.quantize(a, nv.SF_TCGEN05, out=qa), 20)
+        ms_g = _timed(torch, dev, flush, lambda: nv.gemm(qa, qw, out=d), 20)
+        ms_two = _timed(torch, dev, flush, lambda: (nv.quantize(a, nv.SF_TCGEN05, out=qa), nv.gemm(qa, qw, out=d)), 20)
+        result["parts"]["prefill_step_two_kernels"] = {
+            "ms": ms_two, "tflops": FLOPS_STEP / (ms_two * 1e-3) / 1e12, "quantize_ms": ms_q, "gemm_ms": ms_g,
+            "note": "amax + quantize passes, then gemm_pair_kernel; median of 20, L2 flushed"}
+        result["parts"]["gemm_only"] = {
+            "ms": ms_g, "tflops": FLOPS_STEP / (ms_g * 1e-3) / 1e12,
+            "frac_fp4_peak": FLOPS_STEP / (ms_g * 1e-3) / 1e12 / fp4_peak,
+            "traffic": profile_traffic("gemm_prefill_8192.md", GEMM_SOURCES)}
     if rank == 0 and world == 1 and not args.no_cpu:
         sample = OracleSample(a_bits, w_bits, rows=8192, cols=2048)
         sec = time_oracle(sample)
@@ -391,10 +413,10 @@ def main():
         dist.destroy_process_group()
 
 
-def bench_e2e(nv, torch, dev, a_bits, qw, qa, steps):
+def bench_e2e(nv, torch, dev, a_bits, qw, steps):
     """The step through host buffers: every step copies A [8192, 8192] bf16 from
-    pinned host memory, quantizes it, runs the GEMM and copies D back to pinned
-    host memory.  Steps are double-buffered on three streams (upload, compute,
+    pinned host memory, quantizes and multiplies it (nvfp4_gemm_quant_a) and
+    copies D back to pinned host memory.  Steps are double-buffered on three streams (upload, compute,
     download), as a serving loop overlaps them: step i+1's upload and step
     i-1's download run while step i computes, each buffer reused only after
     the work that read it has finished."""
@@ -402,7 +424,8 @@ def bench_e2e(nv, torch, dev, a_bits, qw, qa, steps):
     d_host = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     a_dev = [torch.empty((M, K), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     d_dev = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    qas = [qa, nv.empty_quantized(M, K, nv.SF_TCGEN05, dev)]
+    ws_bytes = nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, M, N, K)
+    wss = [torch.empty(ws_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     up, comp, down = (torch.cuda.Stream(dev) for _ in range(3))
     uploaded = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
@@ -420,8 +443,7 @@ def bench_e2e(nv, torch, dev, a_bits, qw, qa, steps):
                 comp.wait_event(uploaded[b])
                 if i >= 2:
                     comp.wait_event(downloaded[b])      # d_dev[b] copied out
-                nv.quantize(a_dev[b], nv.SF_TCGEN05, out=qas[b], stream=comp)
-                nv.gemm(qas[b], qw, out=d_dev[b], stream=comp)
+                nv.gemm_quant_a(a_dev[b], qw, out=d_dev[b], workspace=wss[b], stream=comp)
                 computed[b].record(comp)
             with torch.cuda.stream(down):
                 down.wait_event(computed[b])
@@ -708,6 +730,12 @@ def run_part(args):
         out["ms"] = _timed(torch, dev, flush, lambda: nv.nvfp4_gemm_requant(
             qa.codes, qa.sf, qa.g, qw.codes, qw.sf, qw.g, M, N, K, h.g, h.codes, N // 2, h.sf, nv.SF_TCGEN05,
             h.amax), args.steps)
+    elif args.part == "quantgemm":
+        qw = nv.quantize(to_dev(w_bits), nv.SF_TCGEN05)
+        a = to_dev(a_bits)
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, M, N, K), dtype=torch.uint8, device=dev)
+        out["ms"] = _timed(torch, dev, flush, lambda: nv.gemm_quant_a(a, qw, out=d, workspace=ws), args.steps)
     elif args.part == "mxgemm":
         qa = nv.mxfp4_quantize(to_dev(a_bits), nv.SF_TCGEN05)
         qw = nv.mxfp4_quantize(to_dev(w_bits), nv.SF_TCGEN05)

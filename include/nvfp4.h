@@ -358,6 +358,23 @@ NVFP4_API nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const
                                 nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gemm_quant_a in two calls on one stream, the same A and workspace:
+ * _prepare zeroes what the second call counts on and runs the amax pass of A
+ * into the workspace (it reads no B and writes no D); _run quantizes A and
+ * multiplies.  _prepare then _run computes exactly what nvfp4_gemm_quant_a
+ * computes; work may be enqueued between them if it leaves A and the
+ * workspace alone.  A _run without a _prepare since the last _run on that
+ * workspace is an error the library cannot detect: D may then come from a
+ * stale amax or from rows of A not yet quantized.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_quant_a_prepare(const void* a_bf16, int64_t lda, int64_t M, int64_t N, int64_t K,
+                                void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+NVFP4_API nvfp4_status nvfp4_gemm_quant_a_run(const void* a_bf16, int64_t lda, const void* b_codes,
+                                const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K,
+                                void* d, int64_t ldd, nvfp4_out_dtype out_dtype, void* workspace,
+                                size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
  * nvfp4_gemm_quant_a with A's tensor amax already on the device: amax_dev
  * (one fp32, read-only) holds max |A|, e.g. from nvfp4_amax on the same A
  * earlier on the stream; the call skips its own amax pass.  Null amax_dev:

@@ -375,14 +375,18 @@ nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t ldx, cons
 
 namespace {
 
-// Quantize a bf16 A and multiply (amax_given: A's amax already on the device;
-// else computed into the workspace).  Workspace: A's codes, A's tensor-core
+// Quantize a bf16 A and multiply.  Workspace: A's codes, A's tensor-core
 // scales, then the scalars (g_a at byte 0, amax at byte 16) and the
-// quantize-and-GEMM kernel's row-block counters from byte 64.
-nvfp4_status gemm_quant_a_common(const void* a_bf16, int64_t lda, const float* amax_given, const void* b_codes,
-                                 const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d,
-                                 int64_t ldd, nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
-                                 nvfp4_stream_t stream) {
+// quantize-and-GEMM kernel's row-block counters from byte 64.  The prepare
+// phase zeroes the amax (and the counters) and runs the amax pass; the run
+// phase quantizes and multiplies.  kAmaxGiven: A's amax is already on the
+// device (the counters are zeroed, then the run phase).
+enum class QaMode { kAll, kPrepare, kRun, kAmaxGiven };
+
+nvfp4_status gemm_quant_a_common(QaMode mode, const void* a_bf16, int64_t lda, const float* amax_given,
+                                 const void* b_codes, const void* b_sf_tc, const float* g_b_dev, int64_t M, int64_t N,
+                                 int64_t K, void* d, int64_t ldd, nvfp4_out_dtype out_dtype, void* workspace,
+                                 size_t ws_bytes, nvfp4_stream_t stream) {
   nvfp4_status st = check_bf16_input(a_bf16, M, K, lda);
   if (st != NVFP4_OK) return st;
   if (!workspace) return NVFP4_ERR_INVALID_ARG;
@@ -397,26 +401,33 @@ nvfp4_status gemm_quant_a_common(const void* a_bf16, int64_t lda, const float* a
   float* g_a = reinterpret_cast<float*>(scal_bytes);
   float* amax_ws = reinterpret_cast<float*>(scal_bytes + 16);
   int* counters = reinterpret_cast<int*>(scal_bytes + 64);
-  st = check_gemm_operands(a_codes, a_sf, g_a, b_codes, b_sf_tc, g_b_dev, M, N, K, d);
-  if (st != NVFP4_OK) return st;
-  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
-  if (ldd < N) return NVFP4_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(d) & (out_dtype == NVFP4_OUT_F32 ? 3u : 1u)) != 0) return NVFP4_ERR_MISALIGNED;
+  if (mode != QaMode::kPrepare) {
+    st = check_gemm_operands(a_codes, a_sf, g_a, b_codes, b_sf_tc, g_b_dev, M, N, K, d);
+    if (st != NVFP4_OK) return st;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+    if (ldd < N) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d) & (out_dtype == NVFP4_OUT_F32 ? 3u : 1u)) != 0) return NVFP4_ERR_MISALIGNED;
+  }
   if ((st = check_arch()) != NVFP4_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool fused = quant_a_fusable(M, N, K);
-  const float* amax = amax_given ? amax_given : amax_ws;
-  if (fused) {
-    // zero the row-block counters (and the amax when this call computes it) in one memset
-    const size_t first = amax_given ? 64 : 16;
-    const size_t end = 64 + 4 * static_cast<size_t>((M + 255) / 256);
-    cudaError_t e = cudaMemsetAsync(scal_bytes + first, 0, end - first, s);
+  const size_t counters_end = 64 + 4 * static_cast<size_t>((M + 255) / 256);
+  if (mode == QaMode::kAll || mode == QaMode::kPrepare) {
+    if (fused) {
+      // zero the amax and the row-block counters in one memset; the
+      // quantizers take the first rows first, so the amax pass leaves those in L2
+      cudaError_t e = cudaMemsetAsync(scal_bytes + 16, 0, counters_end - 16, s);
+      if (e != cudaSuccess) return launch_status(e);
+      st = launch_amax_reversed(a_bf16, M, K, lda, amax_ws, s);
+    } else {
+      st = launch_amax(a_bf16, M, K, lda, amax_ws, s);
+    }
+    if (st != NVFP4_OK || mode == QaMode::kPrepare) return st;
+  } else if (mode == QaMode::kAmaxGiven && fused) {
+    cudaError_t e = cudaMemsetAsync(scal_bytes + 64, 0, counters_end - 64, s);
     if (e != cudaSuccess) return launch_status(e);
-    // the quantizers take the first rows first: leave those in L2
-    if (!amax_given && (st = launch_amax_reversed(a_bf16, M, K, lda, amax_ws, s)) != NVFP4_OK) return st;
-  } else if (!amax_given && (st = launch_amax(a_bf16, M, K, lda, amax_ws, s)) != NVFP4_OK) {
-    return st;
   }
+  const float* amax = mode == QaMode::kAmaxGiven ? amax_given : amax_ws;
   if (fused)
     return launch_gemm_quant_a_fused(a_bf16, lda, amax, a_codes, a_sf, g_a, counters, b_codes, b_sf_tc, g_b_dev, M,
                                      N, K, d, ldd, out_dtype, s);
@@ -433,8 +444,22 @@ nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_c
                                 const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
                                 nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
                                 nvfp4_stream_t stream) {
-  return gemm_quant_a_common(a_bf16, lda, nullptr, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype, workspace,
-                             ws_bytes, stream);
+  return gemm_quant_a_common(QaMode::kAll, a_bf16, lda, nullptr, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd,
+                             out_dtype, workspace, ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_quant_a_prepare(const void* a_bf16, int64_t lda, int64_t M, int64_t N, int64_t K,
+                                        void* workspace, size_t ws_bytes, nvfp4_stream_t stream) {
+  return gemm_quant_a_common(QaMode::kPrepare, a_bf16, lda, nullptr, nullptr, nullptr, nullptr, M, N, K, nullptr, N,
+                             NVFP4_OUT_BF16, workspace, ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_quant_a_run(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,
+                                    const float* g_b_dev, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
+                                    nvfp4_out_dtype out_dtype, void* workspace, size_t ws_bytes,
+                                    nvfp4_stream_t stream) {
+  return gemm_quant_a_common(QaMode::kRun, a_bf16, lda, nullptr, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd,
+                             out_dtype, workspace, ws_bytes, stream);
 }
 
 nvfp4_status nvfp4_gemm_quant_a_amax(const void* a_bf16, int64_t lda, const float* amax_dev, const void* b_codes,
@@ -442,8 +467,8 @@ nvfp4_status nvfp4_gemm_quant_a_amax(const void* a_bf16, int64_t lda, const floa
                                      void* d, int64_t ldd, nvfp4_out_dtype out_dtype, void* workspace,
                                      size_t ws_bytes, nvfp4_stream_t stream) {
   if (!amax_dev) return NVFP4_ERR_INVALID_ARG;
-  return gemm_quant_a_common(a_bf16, lda, amax_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype,
-                             workspace, ws_bytes, stream);
+  return gemm_quant_a_common(QaMode::kAmaxGiven, a_bf16, lda, amax_dev, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd,
+                             out_dtype, workspace, ws_bytes, stream);
 }
 
 nvfp4_status nvfp4_check_device_status(nvfp4_stream_t stream) {

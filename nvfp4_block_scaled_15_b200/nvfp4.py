@@ -58,6 +58,8 @@ _SIGS = {
     "nvfp4_workspace_bytes": ([_i32, _i64, _i64, _i64], _sz),
     "nvfp4_gemv_batched": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _sz, _vp], _i32),
     "nvfp4_gemm_quant_a": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp], _i32),
+    "nvfp4_gemm_quant_a_prepare": ([_vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _i32),
+    "nvfp4_gemm_quant_a_run": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp], _i32),
     "nvfp4_gemm_quant_a_amax": ([_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _sz, _vp],
                                 _i32),
     "nvfp4_gemv_batched_noalloc": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _vp], _i32),
@@ -189,6 +191,17 @@ def nvfp4_gemm_quant_a(a, lda, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, w
                        stream=None) -> None:
     _check(_lib.nvfp4_gemm_quant_a(_p(a), lda, _p(b_codes), _p(b_sf), _p(g_b), m, n, k, _p(d), ldd, out_dtype,
                                    _p(workspace), ws_bytes, _s(stream)), "nvfp4_gemm_quant_a")
+
+
+def nvfp4_gemm_quant_a_prepare(a, lda, m, n, k, workspace, ws_bytes, stream=None) -> None:
+    _check(_lib.nvfp4_gemm_quant_a_prepare(_p(a), lda, m, n, k, _p(workspace), ws_bytes, _s(stream)),
+           "nvfp4_gemm_quant_a_prepare")
+
+
+def nvfp4_gemm_quant_a_run(a, lda, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, workspace, ws_bytes,
+                           stream=None) -> None:
+    _check(_lib.nvfp4_gemm_quant_a_run(_p(a), lda, _p(b_codes), _p(b_sf), _p(g_b), m, n, k, _p(d), ldd, out_dtype,
+                                       _p(workspace), ws_bytes, _s(stream)), "nvfp4_gemm_quant_a_run")
 
 
 def nvfp4_gemm_quant_a_amax(a, lda, amax, b_codes, b_sf, g_b, m, n, k, d, ldd, out_dtype, workspace, ws_bytes,

@@ -82,6 +82,13 @@ def test_argument_errors_return_before_any_device_work(nv):
     assert raw("nvfp4_gemv_batched", fake, 33, 64, fake, fake, fake, 128, 64, fake, 128, fake, 1 << 30, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert raw("nvfp4_gemv_batched", fake, 4, 64, fake, fake, fake, 128, 64, fake, 128, fake, 16, None) == nv.ERR_WORKSPACE
     assert raw("nvfp4_gemm_quant_a", fake, 64, fake, fake, fake, 8, 8, 64, fake, 8, 0, fake, 16, None) == nv.ERR_WORKSPACE
+    assert raw("nvfp4_gemm_quant_a_prepare", fake, 64, 8, 8, 64, fake, 16, None) == nv.ERR_WORKSPACE
+    assert raw("nvfp4_gemm_quant_a_prepare", fake, 96, 8, 8, 96, fake, 1 << 20, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert raw("nvfp4_gemm_quant_a_run", fake, 64, fake, fake, fake, 8, 8, 64, fake, 8, 0, fake, 16, None) == nv.ERR_WORKSPACE
+    assert raw("nvfp4_gemm_quant_a_run", fake, 64, fake, fake, fake, 8, 8, 64, fake, 4, 0, fake, 1 << 20, None) == nv.ERR_INVALID_ARG
+    qa_amax = "nvfp4_gemm_quant_a_amax"
+    assert raw(qa_amax, fake, 64, None, fake, fake, fake, 8, 8, 64, fake, 8, 0, fake, 1 << 20, None) == nv.ERR_INVALID_ARG
+    assert raw(qa_amax, fake, 64, fake, fake, fake, fake, 8, 8, 64, fake, 8, 0, fake, 16, None) == nv.ERR_WORKSPACE
     assert raw("nvfp4_swizzle_sf", fake, 4, 48, fake, None) == nv.ERR_UNSUPPORTED_SHAPE
     qs = "nvfp4_quantize_stochastic"
     assert raw(qs, fake, 4, 48, 48, fake, fake, 1, fake, fake, 0, 1, 2, None) == nv.ERR_UNSUPPORTED_SHAPE

@@ -1,8 +1,8 @@
-"""Quantize-and-multiply (nvfp4_gemm_quant_a, nvfp4_gemm_quant_a_amax): a bf16
-A quantized inside the call, then the block-scaled GEMM.  Where one kernel
-does both (M, N > 128, B's codes <= 64 MiB), its codes, scales, g_a and D must
-equal, bit for bit, those of the quantize pass followed by the GEMM, and both
-must agree with the oracle."""
+"""Quantize-and-multiply (nvfp4_gemm_quant_a and its _prepare / _run and
+_amax forms): a bf16 A quantized inside the call, then the block-scaled GEMM.
+Where one kernel does both (M, N > 128, B's codes <= 64 MiB), its codes,
+scales, g_a and D must equal, bit for bit, those of the quantize pass followed
+by the GEMM, and both must agree with the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -115,10 +115,29 @@ def test_quant_a_amax_given_equals_own_amax(lib):
     assert torch.equal(d1.view(torch.int32), d2.view(torch.int32))
 
 
+def test_quant_a_prepare_then_run_equals_one_call(lib):
+    """_prepare then _run (with unrelated work enqueued between them) gives
+    what one nvfp4_gemm_quant_a call gives, bit for bit, on the fused path and
+    on the two-kernel path (N <= 128)."""
+    for m, n, k in ((1000, 520, 1088), (300, 96, 512)):
+        a, a_dev = _a_input(m, k, 0, seed=m)
+        w = inputs.gaussian_bf16((n, k), seed=n, std=0.02)
+        qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+        d1 = lib.gemm_quant_a(a_dev, qw, out_dtype=torch.float32)
+        ws = torch.empty(lib.nvfp4_workspace_bytes(lib.OP_GEMM_QUANT_A, m, n, k), dtype=torch.uint8, device="cuda")
+        d2 = torch.empty((m, n), dtype=torch.float32, device="cuda")
+        lib.nvfp4_gemm_quant_a_prepare(a_dev, k, m, n, k, ws, ws.numel())
+        other = torch.randn(1 << 20, device="cuda").sum()          # unrelated work between the calls
+        lib.nvfp4_gemm_quant_a_run(a_dev, k, qw.codes, qw.sf, qw.g, m, n, k, d2, n, lib.OUT_F32, ws, ws.numel())
+        assert lib.nvfp4_check_device_status() == lib.OK
+        assert torch.isfinite(other)
+        assert torch.equal(d1.view(torch.int32), d2.view(torch.int32))
+
+
 def test_quant_a_workspace_reused_across_inputs(lib):
-    """Five calls on one workspace with a different A each time: the row-block
-    counters carry a per-call tag, so no call starts its GEMM on rows left by
-    the previous call; each result equals the two-kernel path's."""
+    """Five calls on one workspace with a different A each time: each call
+    zeroes the row-block counters first, so no call starts its GEMM on rows
+    left by the previous call; each result equals the two-kernel path's."""
     m, n, k = 1536, 512, 2048
     w = inputs.gaussian_bf16((n, k), seed=8, std=0.02)
     qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
