@@ -989,10 +989,11 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
     // ------------------- A quantizers (quantize-and-GEMM) -------------------
     // Units (row r, blocks c * QA_UNIT_BLOCKS ..) numbered row-major and
     // taken in order (a start-up unit, then every nqw-th), so the row blocks
-    // complete roughly first to last, the order the row-major tiles need them.  Each unit: the quantize pass's rule (block
-    // scales RN_e4m3(RN(RN(amax_b g) / 6)), codes RN_e2m1(RN(RN(x g) / s)));
-    // rows past M (up to the 128-row group) get zero scales.  After a unit
-    // the warp counts it on its row block's counter with release semantics.
+    // complete roughly first to last, the order the row-major tiles need
+    // them.  Each unit: the quantize pass's rule (block scales
+    // RN_e4m3(RN(RN(amax_b g) / 6)), codes RN_e2m1(RN(RN(x g) / s))); rows
+    // past M (up to the 128-row group) get zero scales.  After a unit the
+    // warp counts it on its row block's counter with release semantics.
     const int qw = warp - (2 + C::EPI_WARPS);
     bool valid;
     const float g = global_scale_from_amax(*p.qa_amax, valid);
