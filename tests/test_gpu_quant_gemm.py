@@ -99,6 +99,25 @@ def test_quant_a_bf16_out_prefill_full_size(lib):
     check_bf16(host_bf16_bits(d)[rows, cols], d_ref, s_ref, alpha)
 
 
+@pytest.mark.parametrize("n", [260, 264], ids=lambda v: f"n{v}")
+def test_quant_a_bf16_into_wider_output(lib, n):
+    """bf16 D written into a wider, taller buffer (row pitch n + 40): N = 260
+    ends inside a 16-B chunk (direct stores from the 64-column drain), N = 264
+    on a chunk boundary (TMA stores); equal to the two-kernel path, nothing
+    outside the M x N window changes."""
+    m, k = 300, 512
+    _, a_dev = _a_input(m, k, 0, seed=n)
+    w = inputs.gaussian_bf16((n, k), seed=n + 1, std=0.02)
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    big = torch.full((m + 8, n + 40), -7.0, dtype=torch.bfloat16, device="cuda")
+    lib.gemm_quant_a(a_dev, qw, out=big[:m, :n])
+    _, d2 = _two_kernel(lib, a_dev, qw, torch.bfloat16)
+    assert lib.nvfp4_check_device_status() == lib.OK
+    assert torch.equal(big[:m, :n].contiguous().view(torch.int16), d2.view(torch.int16))
+    assert torch.all(big[:m, n:] == -7.0)
+    assert torch.all(big[m:, :] == -7.0)
+
+
 def test_quant_a_amax_given_equals_own_amax(lib):
     """nvfp4_gemm_quant_a_amax with the amax from nvfp4_amax gives what
     nvfp4_gemm_quant_a gives with its own amax pass."""
