@@ -562,16 +562,18 @@ __device__ __forceinline__ int64_t qa_startup_units(int64_t units, int grid, int
 }
 
 // Quantizer warp: 16-element blocks b0 + 32 j (j < QA_BLOCKS) of A row r into
-// w (zeros past the row's end or for rows past M).
+// w (zeros past the row's end or for rows past M).  A is read once: the
+// loads are marked evict-first in L2, where B and A's codes are reused.
 __device__ __forceinline__ void qa_load(const GemmParams& p, int r, int b0, int kb, bool wide,
                                         uint32_t (&w)[QA_BLOCKS][8]) {
   const bool real = r < p.M;
   const uint16_t* xr = p.qa_x + static_cast<int64_t>(r) * p.qa_ldx;
+  const uint64_t pol = l2_evict_first_policy();
 #pragma unroll
   for (int j = 0; j < QA_BLOCKS; ++j) {
     const int b = b0 + 32 * j;
     if (real && b < kb) {
-      load_bf16_block(xr + b * 16, w[j], wide);
+      load_bf16_block_hint(xr + b * 16, w[j], wide, pol);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[j][i] = 0u;
