@@ -350,6 +350,11 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M,
  *   amax_a 16 bytes after it and row-block counters from byte 64 there,
  *   which the call zeroes itself.  It needs no clearing; calls sharing a
  *   workspace must not overlap.
+ * Concurrency: the one-kernel form's CTAs wait for rows that other CTAs of
+ *   the same launch quantize, so it needs its whole grid resident to run at
+ *   speed.  Run these calls on one stream; two of them overlapping on the
+ *   device may wait on each other until the wait limit and report
+ *   NVFP4_ERR_TIMEOUT.
  * K % 64 == 0.
  */
 NVFP4_API nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,
