@@ -20,3 +20,22 @@ def lib():
     """The CUDA library, built in-tree; GPU tests fail loudly if it is missing."""
     from nvfp4_block_scaled_15_b200 import nvfp4
     return nvfp4
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Per test: bf16 outputs that passed only by the carried pre-cast bound."""
+    parity = sys.modules.get("parity")
+    log = getattr(parity, "CARRIED_LOG", None) if parity else None
+    if not log:
+        return
+    per = {}
+    for test, n, size in log:
+        c, t = per.get(test, (0, 0))
+        per[test] = (c + n, t + size)
+    total_c = sum(c for c, _ in per.values())
+    total_t = sum(t for _, t in per.values())
+    terminalreporter.write_sep("-", "bf16 outputs passing only by the carried pre-cast bound")
+    for test, (c, t) in sorted(per.items()):
+        if c:
+            terminalreporter.write_line(f"{test}: {c} of {t}")
+    terminalreporter.write_line(f"all bf16 checks: {total_c} of {total_t} outputs ({len(per)} tests)")

@@ -9,12 +9,20 @@ Acceptance (written here once, used by every GEMM/GEMV test):
     |D - D_ref| <= 2^-20 * alpha * S + ulp_bf16(D)/2 (the pre-cast bound
     carried through one rounding to bf16).
 """
+import os
+
 import numpy as np
 import torch
 
 from oracle import nvfp4_oracle as O
 
 BOUND = 2.0 ** -20
+
+# Largest share of a bf16 output that may pass by the carried pre-cast bound
+# alone (more than 1 ulp from bf16_rne(D_ref)).  Each check's count is
+# asserted against it and logged; conftest prints the log after the run.
+CARRIED_LIMIT = 1e-3
+CARRIED_LOG = []        # (test id, outputs passing only by the carried bound, outputs checked)
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -43,8 +51,11 @@ def check_f32(d_gpu: np.ndarray, d_ref: np.ndarray, s_ref: np.ndarray, alpha) ->
         f"{bad[0].size} fp32 outputs outside 2^-20*alpha*S; worst ratio {np.max(err / np.maximum(lim, 1e-300)):.3g}")
 
 
-def check_bf16(y_bits: np.ndarray, d_ref: np.ndarray, s_ref: np.ndarray, alpha) -> int:
-    """Returns how many elements needed the carried pre-cast bound."""
+def check_bf16(y_bits: np.ndarray, d_ref: np.ndarray, s_ref: np.ndarray, alpha,
+               carried_limit: float = CARRIED_LIMIT) -> int:
+    """Asserts the bf16 acceptance rule on every element, and that at most
+    ``carried_limit`` of them (rounded down) pass by the carried bound alone.
+    Returns that count (also appended to CARRIED_LOG)."""
     ref_bits = O.f64_to_bf16_rne(d_ref)
     ulps = np.abs(O.bf16_ordinal(y_bits) - O.bf16_ordinal(ref_bits))
     y = O.bf16_to_f32(y_bits).astype(np.float64)
@@ -55,4 +66,9 @@ def check_bf16(y_bits: np.ndarray, d_ref: np.ndarray, s_ref: np.ndarray, alpha) 
     bad = np.nonzero(~ok)
     assert bad[0].size == 0, (
         f"{bad[0].size} bf16 outputs off; e.g. got {y[bad][:4]} want {d_ref[bad][:4]} ulps {ulps[bad][:4]}")
-    return int(np.count_nonzero((ulps > 1) & carried))
+    n_carried = int(np.count_nonzero((ulps > 1) & carried))
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    CARRIED_LOG.append((test, n_carried, int(y.size)))
+    assert n_carried <= int(carried_limit * y.size), (
+        f"{n_carried} of {y.size} bf16 outputs pass only by the carried pre-cast bound")
+    return n_carried
