@@ -25,6 +25,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -58,6 +59,11 @@ def parse_args():
                                        "mxquantize", "mxgemm", "requant"],
                     default=None,
                     help="run one workload alone, --steps times (for profiling); prints its timing")
+    ap.add_argument("--record-traffic", nargs=4, metavar=("NAME", "RAW_CSV", "LAUNCHES", "SOURCES"),
+                    help="store DRAM bytes per launch of an ncu capture in profiles/traffic.json: NAME, the "
+                         "CSV of 'ncu -i REPORT --page raw --csv', the number of captured launches, and the "
+                         "kernel's csrc files, comma-separated; the capture command follows as --traffic-command")
+    ap.add_argument("--traffic-command", default="", help="the ncu command of --record-traffic's capture")
     return ap.parse_args()
 
 
@@ -69,32 +75,67 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash(files):
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and with whitespace runs collapsed:
+    edits to comments or layout do not change it."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_code_hash(files):
     h = hashlib.sha256()
     for name in files:
-        with open(os.path.join(ROOT, "nvfp4_block_scaled_15_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_15_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(summary_name, src_files):
-    """DRAM bytes per launch from a committed ncu summary (``source_hash:`` and
-    ``dram_bytes_per_launch:`` lines), if it matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", summary_name)
-    if not os.path.exists(path):
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def profile_traffic(name):
+    """DRAM bytes per launch of a kernel from one ncu capture, kept in
+    profiles/traffic.json by ``--record-traffic``; None when the kernel's code
+    (comments and layout aside) changed after the capture."""
+    if not os.path.exists(TRAFFIC_JSON):
         return None
-    info = {}
-    with open(path) as f:
-        for line in f:
-            if ":" in line and not line.startswith(("|", "#", " ")):
-                key, _, val = line.partition(":")
-                info[key.strip()] = val.strip()
-    if info.get("source_hash") != kernel_source_hash(src_files):
+    with open(TRAFFIC_JSON) as f:
+        entry = json.load(f).get(name)
+    if not entry or entry.get("code_hash") != kernel_code_hash(entry["sources"]):
         return None
-    try:
-        return int(info["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    return int(entry["dram_bytes_per_launch"])
+
+
+def record_traffic(name, raw_csv, sources, launches, command):
+    """Store one capture's DRAM traffic per launch (dram__bytes_read.sum +
+    dram__bytes_write.sum, averaged over the captured launches) from the CSV
+    that ``ncu -i REPORT --page raw --csv`` prints, with the code hash of the
+    kernel's sources at capture time."""
+    import csv
+    with open(raw_csv, newline="") as f:
+        rows = list(csv.reader(f))
+    head = next(r for r in rows if "dram__bytes_read.sum" in r)
+    i_r, i_w = head.index("dram__bytes_read.sum"), head.index("dram__bytes_write.sum")
+    units_row = rows[rows.index(head) + 1]
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    vals = []
+    for r in rows[rows.index(head) + 2:]:
+        if len(r) > max(i_r, i_w) and r[i_r]:
+            vals.append(float(r[i_r].replace(",", "")) * scale[units_row[i_r]]
+                        + float(r[i_w].replace(",", "")) * scale[units_row[i_w]])
+    if len(vals) != launches:
+        raise SystemExit(f"{len(vals)} launches in {raw_csv}, expected {launches}")
+    data = {}
+    if os.path.exists(TRAFFIC_JSON):
+        with open(TRAFFIC_JSON) as f:
+            data = json.load(f)
+    data[name] = {"dram_bytes_per_launch": int(round(sum(vals) / len(vals))), "sources": sources,
+                  "code_hash": kernel_code_hash(sources), "launches": launches, "command": command}
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return data[name]
 
 
 # ---------------------------------------------------------------------------
@@ -271,6 +312,10 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
+    if args.record_traffic:
+        name, raw_csv, launches, sources = args.record_traffic
+        print(json.dumps(record_traffic(name, raw_csv, sources.split(","), int(launches), args.traffic_command)))
+        return
     if args.part:
         run_part(args)
         return
@@ -363,7 +408,7 @@ def main():
     if rank == 0:
         fused_avg = statistics.mean(fused_ms)
         achieved = FLOPS_STEP / (fused_avg * 1e-3) / 1e12
-        traffic = profile_traffic("quant_gemm_prefill_8192.md", GEMM_SOURCES)
+        traffic = profile_traffic("quant_gemm_prefill_8192")
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -397,7 +442,7 @@ def main():
         result["parts"]["gemm_only"] = {
             "ms": ms_g, "tflops": FLOPS_STEP / (ms_g * 1e-3) / 1e12,
             "frac_fp4_peak": FLOPS_STEP / (ms_g * 1e-3) / 1e12 / fp4_peak,
-            "traffic": profile_traffic("gemm_prefill_8192.md", GEMM_SOURCES)}
+            "traffic": profile_traffic("gemm_prefill_8192")}
     if rank == 0 and world == 1 and not args.no_cpu:
         sample = OracleSample(a_bits, w_bits, rows=8192, cols=2048)
         sec = time_oracle(sample)

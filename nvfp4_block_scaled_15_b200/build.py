@@ -21,8 +21,12 @@ NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC,-fvisibility=hidden",
     "--expt-relaxed-constexpr",
-    # IEEE division and no fused contractions in the quantizer: its codes are
-    # compared bit for bit with the CPU definition.
+    # IEEE division by default.  Contraction of a*b+c into an FMA stays
+    # allowed (-fmad=true) for the GEMM and GEMV epilogues; every fp32 step
+    # of the quantizers whose rounding is part of the definition is written
+    # with an explicit round-to-nearest intrinsic (__fmul_rn, __fadd_rn,
+    # __fmaf_rn, __fdiv_rn, or the packed .rn PTX forms), which the compiler
+    # never contracts, so their codes match the CPU definition bit for bit.
     "-prec-div=true", "-fmad=true",
 ]
 

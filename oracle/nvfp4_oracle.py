@@ -27,8 +27,8 @@ Definition (fp32 operation order is part of the definition):
      NVFP4 output: steps 3-5 on v with g := g_d (g_d is the output's
      encode scale, given by the caller); amax_d = max |v|
 
-Readings taken where the pages are silent or disagree are listed in the design doc
-of the repository; each function below states the one it uses.
+Where the pages are silent or disagree, each function below states the
+reading it takes.
 
 Pins (tests/test_oracle_pins.py) tie every function to the pages or to
 mathematics outside this file.  ``swizzle_sf_tcgen05`` is a data layout the
