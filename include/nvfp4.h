@@ -298,10 +298,18 @@ NVFP4_API size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_
  * weight stream dominates (decode is memory-bound: "NVIDIA NVFP4 与
  * Micro-Scaling" section 六).  y: out, bf16 [M, N], pitch ldy.
  * workspace: device scratch of nvfp4_workspace_bytes(NVFP4_OP_GEMV_BATCHED, M, N, K)
- *   bytes (quantized x, its scales and g, fp32 partial sums, tile counters);
- *   every call re-initialises what it reads, or marks it with a tag of its
- *   own, so the workspace needs no clearing, before the first call or
- *   between calls.  Calls sharing a workspace must not overlap on the device.
+ *   bytes (quantized x, its scales and g, fp32 partial sums, tile counters).
+ *   It needs no clearing, before the first call or between calls:
+ *     - M > 4: the call's first kernel rewrites the quantized x and zeroes
+ *       the counters;
+ *     - M <= 4: each counter holds a 48-bit tag drawn per launch beside its
+ *       count, and a counter with another tag counts as zero, so stale bytes
+ *       are taken for this launch's only by a 2^-48 chance; every launch that
+ *       completes returns the counters it used to zero, so a CUDA graph that
+ *       replays one launch (one tag) starts each replay from zeros;
+ *     - partial sums are written before they are read.
+ *   After a call that reported NVFP4_ERR_TIMEOUT, zero the workspace before
+ *   reusing it.  Calls sharing a workspace must not overlap on the device.
  * K % 64 == 0, 1 <= M <= 32.
  */
 NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t ldx, const void* w_codes,
@@ -310,10 +318,11 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t
 
 /*
  * nvfp4_gemv_batched without a workspace argument, for callers that cannot
- * allocate device memory: code that must not call the allocator (inside a
- * CUDA graph capture, on a real-time path after start-up), or a plug-in whose
- * host framework hands it only input and output buffers.  The pages have no
- * counterpart of this entry point; it computes exactly what
+ * allocate device memory: a plug-in whose host framework owns all device
+ * memory and hands it only input and output buffers, or a real-time path
+ * that may not call the allocator once it has started (an allocation can
+ * block, synchronise the device or fail when memory is short).  The pages
+ * have no counterpart of this entry point; it computes exactly what
  * nvfp4_gemv_batched computes.
  *   Scratch: a fixed 4 MiB array inside the library, present on every GPU
  *     that loads it until the process exits.  Shapes whose workspace
@@ -324,9 +333,10 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t
  *     up the scratch's device address; make that first call before any stream
  *     capture.  Nothing is allocated or freed, then or later.
  *   Sharing: every call on a device uses the same scratch and overwrites what
- *     the previous call left there (each call clears, or marks with a tag of
- *     its own, what must start at zero).  Calls that overlap on the device
- *     race: serialise them, e.g. on one stream.
+ *     the previous call left there; what must start at zero is cleared by the
+ *     call (M > 4) or tagged per launch and returned to zero at its end
+ *     (M <= 4), as for nvfp4_gemv_batched's workspace.  Calls that overlap on
+ *     the device race: serialise them, e.g. on one stream.
  * Other arguments, constraints and errors as nvfp4_gemv_batched.
  */
 NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M, int64_t ldx, const void* w_codes,
@@ -339,22 +349,25 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M,
  * then multiplied by pre-quantized B as in nvfp4_gemm ("NVIDIA NVFP4 与
  * Micro-Scaling" section 三: activations quantized with a per-tensor global
  * scale and per-block micro-scales, then the block-scaled product).
- *   When M > 128, N > 128 and B's codes (N * K / 2 bytes) are at most 64 MiB,
- *   one kernel does both after the amax pass: extra warps quantize A row by
- *   row while the tensor cores multiply the row blocks already done.  Other
- *   shapes run the quantize pass and the GEMM as two kernels.  Both give the
- *   same codes, scales, g_a and D bit for bit.
+ *   When M > 128 and N > 128 (and K <= 262144), one kernel does both after
+ *   the amax pass: extra warps quantize A in units (one row, 4096 elements
+ *   of K) while the tensor cores multiply the parts already done.  Where B's
+ *   codes (N * K / 2 bytes) are at most 64 MiB the tiles go row block by row
+ *   block and A is quantized row by row; larger B (long K) takes the tiles
+ *   m-fastest and A chunk by chunk along K, so B is read from DRAM once.
+ *   Other shapes run the quantize pass and the GEMM as two kernels.  All
+ *   give the same codes, scales, g_a and D bit for bit.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_QUANT_A, M, N, K) bytes:
  *   A's codes [M, K/2] at byte 0, A's tensor-core scales from
- *   round_up(M * K / 2, 256), then g_a (fp32) at the next 256-byte boundary,
- *   amax_a 16 bytes after it and row-block counters from byte 64 there,
- *   which the call zeroes itself.  It needs no clearing; calls sharing a
- *   workspace must not overlap.
- * Concurrency: the one-kernel form's CTAs wait for rows that other CTAs of
- *   the same launch quantize, so it needs its whole grid resident to run at
- *   speed.  Run these calls on one stream; two of them overlapping on the
- *   device may wait on each other until the wait limit and report
- *   NVFP4_ERR_TIMEOUT.
+ *   round_up(M * K / 2, 256), then at the next 256-byte boundary g_a (fp32),
+ *   amax_a 16 bytes after it, a unit ticket at byte 64 and readiness
+ *   counters (one int per 256-row block and 4096-wide K chunk) from byte 128
+ *   there, which the call zeroes itself.  It needs no clearing; calls
+ *   sharing a workspace must not overlap.
+ * Concurrency: the one-kernel form's warps take units of A from a ticket
+ *   counter, so whichever CTAs are resident quantize what the tiles wait
+ *   for; it runs at speed with its whole grid resident.  Calls that share
+ *   nothing may overlap.
  * K % 64 == 0.
  */
 NVFP4_API nvfp4_status nvfp4_gemm_quant_a(const void* a_bf16, int64_t lda, const void* b_codes, const void* b_sf_tc,

@@ -356,9 +356,12 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 //     amax partials, and each arrives on another (x_ready) once its image
 //     writes are fenced for the tensor core's proxy; the MMA thread waits on
 //     x_ready before its first MMA.
-//   * Fix-up counters carry the call's tag in their high 32 bits, so a
-//     counter left by an earlier call reads as zero and nothing has to clear
-//     them between calls.
+//   * Fix-up counters: (tag << 16) | arrivals, with a 48-bit tag drawn per
+//     launch.  A counter whose tag is not this launch's counts as zero, so
+//     bytes left in the workspace by other use match only by a 2^-48 chance;
+//     and whichever contributor completes a split tile stores 0 back, so a
+//     launch that finishes leaves every counter zero (a replayed graph, whose
+//     launches share one tag, starts from zeros too).
 // ---------------------------------------------------------------------------
 constexpr int GF_MAX_M = 4;                  // rows of x held in registers by the quantizer threads
 constexpr int GF_MAX_K = 8192;
@@ -378,8 +381,8 @@ struct GemvFusedParams {
   const uint8_t* wsf;      // weight scales, tensor-core layout
   const float* g_w;
   float* partials;         // [2 * grid][M][128] fp32 stream-K partial slots
-  unsigned long long* counters;   // [tiles * 4]: (tag << 32) | arrivals
-  uint32_t tag;            // this call's tag (never 0)
+  unsigned long long* counters;   // [tiles * 4]: (tag << 16) | arrivals
+  unsigned long long tag;  // this launch's 48-bit tag (never 0)
   __nv_bfloat16* y;
   int64_t ldy;
   int M, N, K;
@@ -391,14 +394,14 @@ struct GemvFusedParams {
 };
 
 // Count this contributor's arrival on a tagged counter; returns the number
-// of earlier arrivals of the same call (0 or 1).
-__device__ __forceinline__ int tagged_arrive(unsigned long long* c, uint32_t tag) {
+// of earlier arrivals of the same launch (0 or 1).
+__device__ __forceinline__ int tagged_arrive(unsigned long long* c, unsigned long long tag) {
   unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(c);
   for (int attempt = 0; attempt < 64; ++attempt) {
-    const bool same = static_cast<uint32_t>(cur >> 32) == tag;
-    const unsigned long long want = same ? cur + 1ull : ((static_cast<unsigned long long>(tag) << 32) | 1ull);
+    const bool same = (cur >> 16) == tag;
+    const unsigned long long want = same ? cur + 1ull : ((tag << 16) | 1ull);
     const unsigned long long prev = atomicCAS(c, cur, want);
-    if (prev == cur) return same ? static_cast<int>(cur & 0xFFFFFFFFull) : 0;
+    if (prev == cur) return same ? static_cast<int>(cur & 0xFFFFull) : 0;
     cur = prev;
   }
   return 0;   // two contributors per tile cannot contend 64 times; reached only on corruption
@@ -658,8 +661,13 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       float* mine = p.partials + (static_cast<int64_t>(2 * cta + (has_head ? 1 : 0)) * p.M) * BM;
       const float* other = p.partials + (static_cast<int64_t>(has_head ? 2 * (cta + 1) : 2 * (cta - 1) + 1) * p.M) * BM;
       unsigned long long* counter = &p.counters[tile * 4 + quad];
-      const unsigned long long seen = ld_acquire_gpu_u64(counter);
-      if (static_cast<uint32_t>(seen >> 32) == p.tag && (seen & 0xFFFFFFFFull) >= 1ull) {
+      // one load for the warp (lane 0's acquire, broadcast), so all lanes take
+      // the same branch; __syncwarp orders the other lanes' reads after it
+      unsigned long long seen = 0;
+      if (lane == 0) seen = ld_acquire_gpu_u64(counter);
+      seen = __shfl_sync(0xFFFFFFFFu, seen, 0);
+      __syncwarp();
+      if ((seen >> 16) == p.tag && (seen & 0xFFFFull) >= 1ull) {
         if (n < p.N) {
 #pragma unroll
           for (int m = 0; m < GF_MAX_M; ++m)
@@ -668,6 +676,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
               p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
             }
         }
+        if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(counter) = 0ull;   // tile done: reset
         continue;
       }
 #pragma unroll
@@ -688,6 +697,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
               p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(sum * alpha);
             }
         }
+        if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(counter) = 0ull;   // tile done: reset
       }
     }
   }
@@ -865,7 +875,8 @@ __global__ void __launch_bounds__(GP_THREADS) gemv_prologue_kernel(const uint16_
 
 // Workspace of the GEMV: [32, K/2] activation codes | [128, K/16] activation
 // scales | g_x (16 B) | fp32 partial slots [2 * GV_MAX_CTAS][M][128] |
-// counters [tiles * 4] (8 bytes each: the prologue-free kernel tags them).
+// counters [tiles * 4] (8 bytes each: the prologue-free kernel tags them and
+// returns them to zero).
 constexpr int GV_MAX_CTAS = 160;
 
 struct GemvWs {
@@ -886,16 +897,23 @@ static GemvWs gemv_ws_layout(int64_t M, int64_t N, int64_t K) {
 
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K) { return gemv_ws_layout(M, N, K).total; }
 
-// Tags of the prologue-free GEMV's fix-up counters in a caller's workspace:
-// unique per launch within the process and never 0, so a zeroed counter, or
-// one left by an earlier launch in the same workspace, is never taken for
-// this launch's.
-static std::atomic<uint32_t> g_launch_tag{0};
+// Tags of the prologue-free GEMV's fix-up counters: 48 bits, the process's
+// launch count passed through the splitmix64 finaliser (a bijection on 64
+// bits) and cut to 48, never 0.  Consecutive launches get unrelated tags, so
+// counter bytes left in a workspace by other use (small integers, float bit
+// patterns, an earlier launch's values) equal this launch's tag only by a
+// 2^-48 chance.
+static std::atomic<unsigned long long> g_launch_count{0};
 
-uint32_t next_launch_tag() {
-  uint32_t tag = g_launch_tag.fetch_add(1, std::memory_order_relaxed) + 1;
-  if (tag == 0) tag = g_launch_tag.fetch_add(1, std::memory_order_relaxed) + 1;   // skip 0 on wrap
-  return tag;
+unsigned long long next_launch_tag() {
+  for (;;) {
+    unsigned long long z = g_launch_count.fetch_add(1, std::memory_order_relaxed) + 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    const unsigned long long tag = z >> 16;
+    if (tag != 0) return tag;
+  }
 }
 
 static nvfp4_status launch_gemv_fused(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,

@@ -1,9 +1,10 @@
 // Decode GEMV for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc: code running inside a CUDA graph
-// capture that must not allocate, plug-ins and inference runtimes whose
-// memory is owned by a host framework that only hands out input and output
-// buffers, and real-time paths that forbid allocator calls after start-up.
+// Some callers cannot call cudaMalloc: plug-ins and inference runtimes whose
+// device memory is owned by a host framework that only hands them input and
+// output buffers, and real-time paths that forbid allocator calls once they
+// have started (an allocation can block, synchronise the device, or fail
+// when memory runs short).
 // nvfp4_gemv_batched needs a device workspace; this variant uses a fixed
 // scratch array compiled into the library instead, so the caller passes only
 // inputs and outputs.
@@ -79,9 +80,10 @@ extern "C" NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16,
   // The existing GEMV paths, given the fixed scratch as their workspace.
   // Nothing from an earlier call is reused: with M > 4 the prologue rewrites
   // the quantized activations and clears the counters on every call; with
-  // M <= 4 the activations stay in shared memory and the counters carry the
-  // call's tag, so an earlier call's counts read as zero; partial sums are
-  // always written before they are read.
+  // M <= 4 the activations stay in shared memory and the counters carry a
+  // per-launch tag (any other call's counts read as zero) and are returned
+  // to zero by the launch; partial sums are always written before they are
+  // read.
   return launch_gemv(x_bf16, M, ldx, w_codes, w_sf_tc, g_w_dev, N, K, y_bf16, ldy, scratch,
                      reinterpret_cast<cudaStream_t>(stream));
 }

@@ -72,11 +72,13 @@ nvfp4_status launch_gemm_q(const void* a_codes, const void* a_sf, const float* g
 // One kernel that quantizes a bf16 A (global scale from amax_dev, computed
 // by an earlier pass on the stream) into codes / tensor-core scales / g_a and
 // runs the block-scaled GEMM on them as the rows become ready.  counters:
-// ceil(M / 256) int row-block counters, zero when the kernel starts.  Only for
-// shapes quant_a_fusable() accepts.
+// ceil(M / 256) x quant_a_chunks(K) ints ((row block, K chunk) readiness),
+// ticket: one int (the next unit), all zero when the kernel starts.  Only
+// for shapes quant_a_fusable() accepts.
+int quant_a_chunks(int64_t K);
 bool quant_a_fusable(int64_t M, int64_t N, int64_t K);
 nvfp4_status launch_gemm_quant_a_fused(const void* a_bf16, int64_t lda, const float* amax_dev, void* a_codes,
-                                       void* a_sf, float* g_a, int* counters, const void* b_codes,
+                                       void* a_sf, float* g_a, int* counters, int* ticket, const void* b_codes,
                                        const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K,
                                        void* d, int64_t ldd, nvfp4_out_dtype out, cudaStream_t s);
 nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b_codes, const void* b_sf,
@@ -85,7 +87,7 @@ nvfp4_status launch_mx_gemm(const void* a_codes, const void* a_sf, const void* b
 nvfp4_status launch_gemv(const void* x, int64_t M, int64_t ldx, const void* w_codes, const void* w_sf,
                          const float* g_w, int64_t N, int64_t K, void* y, int64_t ldy, void* ws, cudaStream_t s);
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K);
-// Per-launch tag of workspace counters (never 0).
-uint32_t next_launch_tag();
+// Per-launch 48-bit tag of workspace counters (never 0).
+unsigned long long next_launch_tag();
 
 }  // namespace nvfp4

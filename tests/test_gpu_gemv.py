@@ -1,4 +1,9 @@
-"""Decode batched GEMV parity (activations quantized inside the call)."""
+"""Decode batched GEMV parity (activations quantized inside the call).
+
+Two paths serve the call: for M <= 4 and K <= 8192 one kernel whose CTAs
+each quantize the activations (held in registers) into shared memory, and
+otherwise a quantizing prologue followed by the GEMV; the shapes below reach
+both, with ragged N, K not a multiple of 256 and tiles split between CTAs."""
 import numpy as np
 import pytest
 import torch
@@ -10,8 +15,8 @@ from parity import check_bf16, dev_bf16, host_bf16_bits
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("m", [1, 3, 8, 16, 32])
-@pytest.mark.parametrize("n,k", [(1000, 1024), (128, 64), (384, 4096)], ids=lambda v: str(v))
+@pytest.mark.parametrize("m", [1, 3, 5, 8, 13, 16, 17, 32])
+@pytest.mark.parametrize("n,k", [(1000, 1024), (128, 64), (384, 4096), (640, 2880)], ids=lambda v: str(v))
 def test_gemv_matches_oracle(lib, m, n, k):
     x = inputs.gaussian_bf16((m, k), seed=300 + m)
     w = inputs.gaussian_bf16((n, k), seed=400 + n, std=0.02)
@@ -24,7 +29,7 @@ def test_gemv_matches_oracle(lib, m, n, k):
     check_bf16(host_bf16_bits(y), d_ref, s_ref, alpha)
 
 
-@pytest.mark.parametrize("m", [1, 7, 16])
+@pytest.mark.parametrize("m", [1, 7, 12, 16])
 def test_gemv_tiles_split_between_ctas(lib, m):
     """160 weight tiles on at most 148 CTAs: stream-K ranges split tiles
     between neighbouring CTAs, whose partial sums meet in the workspace.
@@ -98,7 +103,7 @@ def test_gemv_decode_full_size_sampled(lib, m):
     check_bf16(host_bf16_bits(y)[:, cols], d_ref, s_ref, alpha)
 
 
-@pytest.mark.parametrize("m", [1, 4])
+@pytest.mark.parametrize("m", [1, 4, 9, 16])
 def test_gemv_weights_in_l2_repeated(lib, m):
     """All 148 CTAs running (160 weight tiles) with 94 MB of weights resident in
     L2, so the weight stages reach the tensor core while the CTAs are still

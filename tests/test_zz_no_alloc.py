@@ -1,8 +1,9 @@
 """The zero-allocation decode GEMV (nvfp4_gemv_batched_noalloc).
 
-It serves callers that cannot allocate device memory (graph captures that
-must not allocate, plug-ins handed only their inputs and outputs).  It must
-give what nvfp4_gemv_batched gives with a caller-allocated workspace, on
+It serves callers that cannot allocate device memory (plug-ins whose host
+framework owns the device memory and hands them only their inputs and
+outputs, real-time paths that may not call the allocator once started).  It
+must give what nvfp4_gemv_batched gives with a caller-allocated workspace, on
 consecutive calls that reuse the library's fixed scratch, and it must refuse
 shapes that do not fit that scratch.  This file is collected last.
 """
@@ -46,6 +47,32 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, m, n, k):
         # and both against the oracle
         check_bf16(new_bits, d_ref, s_ref, alpha)
         check_bf16(old_bits, d_ref, s_ref, alpha)
+
+
+@pytest.mark.parametrize("m", [1, 4])
+def test_noalloc_decode_size_split_tiles_on_two_calls(lib, m):
+    """The decode workload (W [28672, 8192]: tiles split between CTAs) at
+    M <= 4, the kernel whose fix-up counters live in the shared scratch from
+    one call to the next: two calls in a row, each equal bit for bit to the
+    workspace entry point's output, and 512 sampled columns against the
+    oracle."""
+    x_first, w = inputs.decode_gemv(m)
+    n, k = w.shape
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    gw = O.global_scale(O.amax(w))
+    cols = np.sort(np.random.default_rng(53).choice(n, 512, replace=False))
+    cw, sw = O.quantize_with_scale(w[cols], gw)
+    for x in (x_first, inputs.gaussian_bf16((m, k), seed=811 + m)):
+        xd = dev_bf16(x)
+        y_new = _noalloc(lib, xd, qw)
+        y_old = lib.gemv_batched(xd, qw)
+        torch.cuda.synchronize()
+        assert lib.nvfp4_check_device_status() == lib.OK
+        new_bits = host_bf16_bits(y_new)
+        assert np.array_equal(new_bits, host_bf16_bits(y_old))
+        px, sx, gx, _ = O.quantize(x)
+        d_ref, s_ref, alpha = O.gemm_ref(px, sx, gx, O.pack_codes(cw), sw, gw)
+        check_bf16(new_bits[:, cols], d_ref, s_ref, alpha)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
