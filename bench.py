@@ -651,8 +651,21 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
         torch.cuda.synchronize(dev)
         ms_g = g0.elapsed_time(g1) / (2 * calls)
         del graph
+        # one call per event pair, without an L2 flush: the three weight copies
+        # (396 MB, more than L2) in rotation keep every call's weights cold
+        ts = []
+        for i in range(21):
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+            c1.record(stream)
+            ts.append((c0, c1))
+        torch.cuda.synchronize(dev)
+        ms_c = statistics.median(c0.elapsed_time(c1) for c0, c1 in ts)
         thr[f"M={m}"] = {"ms_per_call": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak,
-                         "graph_ms_per_call": ms_g, "graph_frac_hbm": algo / ms_g / 1e6 / hbm_peak}
+                         "graph_ms_per_call": ms_g, "graph_frac_hbm": algo / ms_g / 1e6 / hbm_peak,
+                         "cold_rotated_ms_per_call": ms_c,
+                         "cold_rotated_frac_hbm": algo / ms_c / 1e6 / hbm_peak}
     out["gemv_28672x8192_back_to_back"] = thr
     del wq, wqs
 

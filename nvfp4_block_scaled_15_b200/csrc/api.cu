@@ -117,7 +117,11 @@ nvfp4_status check_bf16_input(const void* x, int64_t rows, int64_t k, int64_t ld
 
 // Scalar tail of the quantize-and-multiply workspace: g_a, the amax and one
 // 32-bit counter per 256-row block of A from byte 64.
-size_t quant_a_scalar_bytes(int64_t M) { return static_cast<size_t>(round_up(64 + 4 * ((M + 255) / 256), 256)); }
+// g_a at 0, amax_a at 16, the unit ticket at 64, the (row block, K chunk)
+// counters from 128.
+size_t quant_a_scalar_bytes(int64_t M, int64_t K) {
+  return static_cast<size_t>(round_up(128 + 4 * ((M + 255) / 256) * quant_a_chunks(K), 256));
+}
 
 }  // namespace
 
@@ -350,7 +354,7 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
   if (op == NVFP4_OP_GEMM_QUANT_A) {
     const size_t codes = static_cast<size_t>(round_up(M * (K / 2), 256));
     const size_t sf = static_cast<size_t>(round_up(nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05), 256));
-    return codes + sf + quant_a_scalar_bytes(M);
+    return codes + sf + quant_a_scalar_bytes(M, K);
   }
   return 0;
 }
@@ -400,7 +404,8 @@ nvfp4_status gemm_quant_a_common(QaMode mode, const void* a_bf16, int64_t lda, c
   uint8_t* scal_bytes = a_sf + round_up(nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05), 256);
   float* g_a = reinterpret_cast<float*>(scal_bytes);
   float* amax_ws = reinterpret_cast<float*>(scal_bytes + 16);
-  int* counters = reinterpret_cast<int*>(scal_bytes + 64);
+  int* ticket = reinterpret_cast<int*>(scal_bytes + 64);
+  int* counters = reinterpret_cast<int*>(scal_bytes + 128);
   if (mode != QaMode::kPrepare) {
     st = check_gemm_operands(a_codes, a_sf, g_a, b_codes, b_sf_tc, g_b_dev, M, N, K, d);
     if (st != NVFP4_OK) return st;
@@ -411,11 +416,11 @@ nvfp4_status gemm_quant_a_common(QaMode mode, const void* a_bf16, int64_t lda, c
   if ((st = check_arch()) != NVFP4_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool fused = quant_a_fusable(M, N, K);
-  const size_t counters_end = 64 + 4 * static_cast<size_t>((M + 255) / 256);
+  const size_t counters_end = 128 + 4 * static_cast<size_t>((M + 255) / 256) * quant_a_chunks(K);
   if (mode == QaMode::kAll || mode == QaMode::kPrepare) {
     if (fused) {
-      // zero the amax and the row-block counters in one memset; the
-      // quantizers take the first rows first, so the amax pass leaves those in L2
+      // zero the amax, the ticket and the readiness counters in one memset;
+      // the quantizers take the first rows first, so the amax pass leaves those in L2
       cudaError_t e = cudaMemsetAsync(scal_bytes + 16, 0, counters_end - 16, s);
       if (e != cudaSuccess) return launch_status(e);
       st = launch_amax_reversed(a_bf16, M, K, lda, amax_ws, s);
@@ -429,8 +434,8 @@ nvfp4_status gemm_quant_a_common(QaMode mode, const void* a_bf16, int64_t lda, c
   }
   const float* amax = mode == QaMode::kAmaxGiven ? amax_given : amax_ws;
   if (fused)
-    return launch_gemm_quant_a_fused(a_bf16, lda, amax, a_codes, a_sf, g_a, counters, b_codes, b_sf_tc, g_b_dev, M,
-                                     N, K, d, ldd, out_dtype, s);
+    return launch_gemm_quant_a_fused(a_bf16, lda, amax, a_codes, a_sf, g_a, counters, ticket, b_codes, b_sf_tc,
+                                     g_b_dev, M, N, K, d, ldd, out_dtype, s);
   if ((st = launch_quantize(a_bf16, M, K, lda, a_codes, a_sf, NVFP4_SF_TCGEN05, g_a, amax, s)) != NVFP4_OK)
     return st;
   return launch_gemm(a_codes, a_sf, g_a, b_codes, b_sf_tc, g_b_dev, M, N, K, d, ldd, out_dtype, s);

@@ -109,8 +109,15 @@ struct GemmParams {
   // Quantize-and-GEMM kernel only: A arrives as bf16 rows (qa_x, pitch
   // qa_ldx elements; qa_wide: 32-B aligned blocks) and is quantized in the
   // kernel into qa_codes / qa_sf (tensor-core layout) with the global scale
-  // from qa_amax (also written to qa_g); qa_ready holds one counter per
-  // 256-row block of A, zero at launch: the rows of the block quantized.
+  // from qa_amax (also written to qa_g).  The work is cut into units (one
+  // row, QA_UNIT_BLOCKS blocks of 16 along K: one K chunk), qa_upr chunks per
+  // row; warps take units in ticket order from qa_ticket.  qa_ready holds one
+  // counter per (256-row block, K chunk), [tiles_m][qa_upr], zero at launch:
+  // the rows of the block whose chunk is quantized.  Row blocks form groups
+  // of qa_group; tiles go group by group, m-fastest inside a group, and units
+  // group by group, chunk by chunk along K inside a group, so a group's
+  // first tiles start once its first chunk is quantized, and B is read from
+  // DRAM about once per group.
   const uint16_t* qa_x;
   int64_t qa_ldx;
   int qa_wide;
@@ -119,6 +126,9 @@ struct GemmParams {
   float* qa_g;
   const float* qa_amax;
   int* qa_ready;
+  int* qa_ticket;
+  int qa_upr;
+  int qa_group;
 };
 
 __host__ __device__ __forceinline__ int round_up_int(int a, int b) { return (a + b - 1) / b * b; }
@@ -529,18 +539,18 @@ struct PairCfg {
   static_assert(SMEM_BYTES_QA <= 232448, "shared memory budget");
 };
 
-// Wait (bounded) until all units of 256-row block tm of A are quantized
-// (upr units per row), then order the TMA loads that follow after the
-// quantizers' stores.
-__device__ __forceinline__ bool wait_rows_quantized(const GemmParams& p, int tm, int rows_pad, int upr,
-                                                    volatile int* abort_flag) {
-  const int want = min(256, rows_pad - tm * 256) * upr;
-  const int* c = p.qa_ready + tm;
-  if (ld_acquire_gpu(c) < want) {
+// Wait (bounded) until chunk c of every row of 256-row block tm of A is
+// quantized, then order the TMA loads that follow after the quantizers'
+// stores.
+__device__ __forceinline__ bool wait_chunk_quantized(const GemmParams& p, int tm, int c, int rows_pad,
+                                                     volatile int* abort_flag) {
+  const int want = min(256, rows_pad - tm * 256);
+  const int* ctr = p.qa_ready + static_cast<int64_t>(tm) * p.qa_upr + c;
+  if (ld_acquire_gpu(ctr) < want) {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
       __nanosleep(64);
-      if (ld_acquire_gpu(c) >= want) break;
+      if (ld_acquire_gpu(ctr) >= want) break;
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > p.wait_limit_ns) {
         *abort_flag = 1;
@@ -553,12 +563,41 @@ __device__ __forceinline__ bool wait_rows_quantized(const GemmParams& p, int tm,
   return true;
 }
 
-// Units quantized at start-up, one per quantizer and epilogue warp of the
-// grid (the epilogue warps have nothing to drain before the first tile):
-// enough for the first row blocks the first tiles need.
-__device__ __forceinline__ int64_t qa_startup_units(int64_t units, int grid, int epi_warps) {
-  const int64_t h = static_cast<int64_t>(grid) * (QA_WARPS + epi_warps);
-  return units < h ? units : h;
+// Row and K chunk of unit u: groups of qa_group row blocks in turn, inside
+// a group chunk by chunk, inside a chunk row by row.  With one row block per
+// group the units go row by row (a row's chunks together), the order in
+// which the row-block-by-row-block tiles need them.
+__device__ __forceinline__ void qa_unit(const GemmParams& p, int u, int rows_pad, int& r, int& c) {
+  if (p.qa_group == 1) {
+    r = u / p.qa_upr;
+    c = u - r * p.qa_upr;
+    return;
+  }
+  const int group_rows = p.qa_group * 256;
+  const int per_group = group_rows * p.qa_upr;
+  const int g = u / per_group;
+  const int ul = u - g * per_group;
+  const int rows_in = min(group_rows, rows_pad - g * group_rows);
+  c = ul / rows_in;
+  r = g * group_rows + (ul - c * rows_in);
+}
+
+// Tile t's row block and column block: groups of qa_group row blocks in
+// turn, m-fastest inside a group.
+__device__ __forceinline__ void qa_tile(const GemmParams& p, int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+  const int per_group = p.qa_group * tiles_n;
+  const int g = t / per_group;
+  const int tl = t - g * per_group;
+  const int tms = min(p.qa_group, tiles_m - g * p.qa_group);
+  tm = g * p.qa_group + tl % tms;
+  tn = tl / tms;
+}
+
+// Publish unit (r, c): its bytes are read next by TMA loads of any CTA.
+__device__ __forceinline__ void qa_publish(const GemmParams& p, int r, int c) {
+  fence_proxy_async_global();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) red_release_add_gpu(p.qa_ready + static_cast<int64_t>(r >> 8) * p.qa_upr + c, 1);
 }
 
 // Quantizer warp: 16-element blocks b0 + 32 j (j < QA_BLOCKS) of A row r into
@@ -634,6 +673,7 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* qa_table = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(full) + 256);   // kQA only
+  int* qa_start = reinterpret_cast<int*>(tmem_slot + 2);       // kQA: first ticket of this CTA's start-up batch
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -654,6 +694,10 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
     mbar_init(ovl_free, 2 * 4);                // the 4 warps per CTA that hold the shared columns
     mbar_init(mma_done, 1);
     *abort_flag = 0;
+    // One ticket batch for the CTA's first units (one per quantizer and
+    // epilogue warp): one atomic per CTA instead of one per warp at the start.
+    // The tickets were zeroed before the amax pass this kernel depends on.
+    if constexpr (kQA) *qa_start = atomicAdd(p.qa_ticket, QA_WARPS + C::EPI_WARPS);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -690,20 +734,36 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
-      int ready_tm = -1;                        // kQA: A rows known quantized up to this row block
-      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
-        const int tm = kQA ? t / tiles_n : t % tiles_m;
-        const int tn = kQA ? t - tm * tiles_n : t / tiles_m;
+      int ready_tm = -1;                        // kQA: row block whose chunks in ready_mask are known quantized
+      uint64_t ready_mask = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && !*abort_flag && ok; t += npairs) {
+        int tm, tn;
+        if constexpr (kQA) {
+          qa_tile(p, t, tiles_m, tiles_n, tm, tn);
+        } else {
+          tm = t % tiles_m;
+          tn = t / tiles_m;
+        }
         const int m_cta = tm * 256 + static_cast<int>(rank) * 128;
         const int n0 = tn * C::BN;
         if constexpr (kQA) {
-          if (tm > ready_tm) {
-            if (!wait_rows_quantized(p, tm, rows_pad, (p.K / 16 + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS, abort_flag))
-              break;
+          if (tm != ready_tm) {
             ready_tm = tm;
+            ready_mask = 0;
           }
         }
         for (int kt = 0; kt < num_kt; ++kt) {
+          if constexpr (kQA) {
+            const int c = kt / (QA_UNIT_BLOCKS * 16 / BK);     // the K chunk this stage reads
+            if (!((ready_mask >> c) & 1u)) {
+              if (!wait_chunk_quantized(p, tm, c, rows_pad, abort_flag)) {
+                ok = false;
+                break;
+              }
+              ready_mask |= uint64_t{1} << c;
+            }
+          }
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_limit_ns, p.status)) break;
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
@@ -834,21 +894,19 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
       alpha = kMx ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(*p.g_a, *p.g_b));
     }
     if constexpr (kQA) {
-      // start-up: this warp's unit of the first row blocks of A
+      // start-up: one unit of A per epilogue warp (nothing to drain before
+      // the first accumulator), so the first tiles' units come from every warp
       bool valid;
       const float g = global_scale_from_amax(*p.qa_amax, valid);
       const int kb = p.K >> 4;
-      const int upr = (kb + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS;
-      const int64_t units = static_cast<int64_t>(rows_pad) * upr;
-      const int64_t u = static_cast<int64_t>(blockIdx.x) * (QA_WARPS + C::EPI_WARPS) + QA_WARPS + ew;
-      if (u < qa_startup_units(units, static_cast<int>(gridDim.x), C::EPI_WARPS)) {
-        const int r = static_cast<int>(u / upr), c0 = static_cast<int>(u % upr) * QA_UNIT_BLOCKS;
+      const int u = *qa_start + QA_WARPS + ew;
+      if (u < rows_pad * p.qa_upr) {
+        int r, c;
+        qa_unit(p, u, rows_pad, r, c);
         uint32_t w[QA_BLOCKS][8];
-        qa_load(p, r, c0 + lane, kb, p.qa_wide != 0, w);
-        qa_quantize_store(p, r, c0 + lane, kb, g, valid, qa_table, w);
-        fence_proxy_async_global();
-        __syncwarp();
-        if (lane == 0) red_release_add_gpu(p.qa_ready + (r >> 8), 1);
+        qa_load(p, r, c * QA_UNIT_BLOCKS + lane, kb, p.qa_wide != 0, w);
+        qa_quantize_store(p, r, c * QA_UNIT_BLOCKS + lane, kb, g, valid, qa_table, w);
+        qa_publish(p, r, c);
       }
     }
     const float gd = kQ ? *p.g_d : 0.0f;
@@ -858,8 +916,13 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
     int j = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++j) {
       const int b = j & 1;
-      const int tm = kQA ? t / tiles_n : t % tiles_m;
-      const int tn = kQA ? t - tm * tiles_n : t / tiles_m;
+      int tm, tn;
+      if constexpr (kQA) {
+        qa_tile(p, t, tiles_m, tiles_n, tm, tn);
+      } else {
+        tm = t % tiles_m;
+        tn = t / tiles_m;
+      }
       if (!mbar_wait_bounded(acc_full, static_cast<uint32_t>(j & 1), abort_flag, p.wait_limit_ns, p.status)) break;
       tc_fence_after();
       uint32_t v[HALF];
@@ -989,13 +1052,13 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
     if constexpr (kQ) publish_amax(p, amax_run);
   } else if constexpr (kQA) {
     // ------------------- A quantizers (quantize-and-GEMM) -------------------
-    // Units (row r, blocks c * QA_UNIT_BLOCKS ..) numbered row-major and
-    // taken in order (a start-up unit, then every nqw-th), so the row blocks
-    // complete roughly first to last, the order the row-major tiles need
-    // them.  Each unit: the quantize pass's rule (block scales
-    // RN_e4m3(RN(RN(amax_b g) / 6)), codes RN_e2m1(RN(RN(x g) / s))); rows
-    // past M (up to the 128-row group) get zero scales.  After a unit the
-    // warp counts it on its row block's counter with release semantics.
+    // Units taken in ticket order (qa_unit maps a ticket to a row and a K
+    // chunk), so units complete roughly in the order the tiles need them,
+    // whichever CTAs are resident.  Each unit: the quantize pass's rule
+    // (block scales RN_e4m3(RN(RN(amax_b g) / 6)), codes
+    // RN_e2m1(RN(RN(x g) / s))); rows past M (up to the 128-row group) get
+    // zero scales.  After a unit the warp counts it on its (row block, chunk)
+    // counter with release semantics.
     const int qw = warp - (2 + C::EPI_WARPS);
     bool valid;
     const float g = global_scale_from_amax(*p.qa_amax, valid);
@@ -1004,32 +1067,47 @@ __global__ void __launch_bounds__(kQA ? PairCfg<kMx>::THREADS_QA : PairCfg<kMx>:
       if (!valid) record_status(p.status, kDevRange);
     }
     const int kb = p.K >> 4;
-    const int upr = (kb + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS;   // units per row
-    const int64_t units = static_cast<int64_t>(rows_pad) * upr;
-    const int nqw = static_cast<int>(gridDim.x) * QA_WARPS;
+    const int units = rows_pad * p.qa_upr;
     const bool wide = p.qa_wide != 0;
     // Pipelined over units: the next unit's loads go out before this one is
-    // published, so the release waits while they are in flight.
-    // Units [0, S) are the start-up units, one per quantizer and epilogue
-    // warp; this warp then takes S + gw, S + gw + nqw, ...
-    const int64_t S = qa_startup_units(units, static_cast<int>(gridDim.x), C::EPI_WARPS);
-    const int64_t gw = static_cast<int64_t>(blockIdx.x) * QA_WARPS + qw;
+    // published, so the release waits while they are in flight.  After its
+    // start-up unit a warp takes tickets two at a time (consecutive units:
+    // with one row block per group, a row's two halves), and one pair ahead
+    // (lane 0 holds the raw value), so the atomic's round trip overlaps the
+    // work instead of preceding the loads.
     uint32_t w[QA_BLOCKS][8];
-    int64_t u = static_cast<int64_t>(blockIdx.x) * (QA_WARPS + C::EPI_WARPS) + qw;
-    if (u >= S) u = S + gw;
-    int r = static_cast<int>(u / upr), c0 = static_cast<int>(u % upr) * QA_UNIT_BLOCKS;
-    if (u < units) qa_load(p, r, c0 + lane, kb, wide, w);
+    int tk_ahead = 0;
+    if (lane == 0) tk_ahead = atomicAdd(p.qa_ticket, 2);
+    int u = *qa_start + qw;                     // this warp's unit of the CTA's start-up batch
+    int pending = -1;                           // the second unit of the current pair
+    int r = 0, c = 0;
+    if (u < units) {
+      qa_unit(p, u, rows_pad, r, c);
+      qa_load(p, r, c * QA_UNIT_BLOCKS + lane, kb, wide, w);
+    }
     while (u < units && !*abort_flag) {
-      qa_quantize_store(p, r, c0 + lane, kb, g, valid, qa_table, w);
-      const int64_t un = u < S ? S + gw : u + nqw;
-      const int rn = static_cast<int>(un / upr), cn = static_cast<int>(un % upr) * QA_UNIT_BLOCKS;
-      if (un < units) qa_load(p, rn, cn + lane, kb, wide, w);
-      fence_proxy_async_global();   // the unit's bytes are read next by TMA loads
-      __syncwarp();
-      if (lane == 0) red_release_add_gpu(p.qa_ready + (r >> 8), 1);
+      qa_quantize_store(p, r, c * QA_UNIT_BLOCKS + lane, kb, g, valid, qa_table, w);
+      // tickets are handed out in increasing order: once one is past the
+      // last unit, so is every later one, and no taken unit is left undone
+      int un;
+      if (pending >= 0) {
+        un = pending;
+        pending = -1;
+      } else {
+        un = __shfl_sync(0xFFFFFFFFu, tk_ahead, 0);
+        if (un + 1 < units) pending = un + 1;
+        // no unit is left past this pair when un + 1 >= units: stop there
+        if (lane == 0) tk_ahead = un + 1 < units ? atomicAdd(p.qa_ticket, 2) : units;
+      }
+      int rn = 0, cn = 0;
+      if (un < units) {
+        qa_unit(p, un, rows_pad, rn, cn);
+        qa_load(p, rn, cn * QA_UNIT_BLOCKS + lane, kb, wide, w);
+      }
+      qa_publish(p, r, c);
       u = un;
       r = rn;
-      c0 = cn;
+      c = cn;
     }
   }
 
@@ -1095,6 +1173,8 @@ struct QuantA {
   int64_t ldx;
   const float* amax;
   int* counters;
+  int* ticket;
+  int group;
 };
 
 template <bool kMx>
@@ -1154,6 +1234,9 @@ nvfp4_status run_gemm_pair(const void* a_codes, const void* a_sf, const float* g
       p.qa_g = const_cast<float*>(g_a);
       p.qa_amax = qa->amax;
       p.qa_ready = qa->counters;
+      p.qa_ticket = qa->ticket;
+      p.qa_upr = quant_a_chunks(K);
+      p.qa_group = qa->group;
     }
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1254,18 +1337,37 @@ nvfp4_status launch_gemm_q(const void* a_codes, const void* a_sf, const float* g
   return dispatch_gemm<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd_bytes, NVFP4_OUT_BF16, &q, s);
 }
 
-// The quantize-and-GEMM kernel takes its tiles row block by row block, so a
-// row block's tiles read all of B's codes: it is used where those stay in L2
-// (and where the CTA-pair kernel would run at all: M, N > 128).
+// K chunks of one A row in the quantize-and-GEMM kernel (units of
+// QA_UNIT_BLOCKS blocks of 16).
+int quant_a_chunks(int64_t K) {
+  return static_cast<int>((K / 16 + QA_UNIT_BLOCKS - 1) / QA_UNIT_BLOCKS);
+}
+
+// The quantize-and-GEMM kernel runs where the CTA-pair kernel would (M, N >
+// 128), with at most 64 K chunks per row (the producer's readiness mask)
+// and unit tickets that fit an int.
 bool quant_a_fusable(int64_t M, int64_t N, int64_t K) {
-  return M > 128 && N > 128 && N * (K / 2) <= (int64_t{64} << 20);
+  const int64_t rows_pad = (M + 127) / 128 * 128;
+  return M > 128 && N > 128 && quant_a_chunks(K) <= 64 && rows_pad * quant_a_chunks(K) < (int64_t{1} << 30);
+}
+
+// Row blocks per group of the quantize-and-GEMM kernel.  Where B's codes
+// (N * K / 2 bytes) stay in L2, one: tiles go row block by row block and
+// every row block reuses B from L2.  Larger B (the long-K workload) would
+// then stream from DRAM once per row block, so the row blocks form about
+// four groups: B is read about four times, and the first tiles still wait
+// only for the first chunk of a quarter of A.
+int quant_a_group(int64_t M, int64_t N, int64_t K) {
+  if (N * (K / 2) <= (int64_t{64} << 20)) return 1;
+  const int tiles_m = static_cast<int>((M + 255) / 256);
+  return (tiles_m + 3) / 4;
 }
 
 nvfp4_status launch_gemm_quant_a_fused(const void* a_bf16, int64_t lda, const float* amax_dev, void* a_codes,
-                                       void* a_sf, float* g_a, int* counters, const void* b_codes,
+                                       void* a_sf, float* g_a, int* counters, int* ticket, const void* b_codes,
                                        const void* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K,
                                        void* d, int64_t ldd, nvfp4_out_dtype out, cudaStream_t s) {
-  const QuantA qa{a_bf16, lda, amax_dev, counters};
+  const QuantA qa{a_bf16, lda, amax_dev, counters, ticket, quant_a_group(M, N, K)};
   return run_gemm_pair<false>(a_codes, a_sf, g_a, b_codes, b_sf, g_b, M, N, K, d, ldd, out, nullptr, s, &qa);
 }
 

@@ -64,10 +64,13 @@ def test_workspace_bytes(nv):
     assert nv.nvfp4_workspace_bytes(nv.OP_GEMV_BATCHED, 33, 128, 128) == 0     # M > 32
     assert nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, 4096, 8192, 28672) >= 4096 * 14336
     assert nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, 16, 16, 100) == 0      # K % 64
-    # A codes, A's tensor-core scales, then g_a, amax_a and one int counter per 256-row block
-    for m, n, k in ((8192, 8192, 8192), (300, 260, 512), (1, 1, 64), (20000, 4096, 1024)):
+    # A codes, A's tensor-core scales, then g_a, amax_a, the unit ticket and one int
+    # counter per (256-row block, K chunk of 4096)
+    for m, n, k in ((8192, 8192, 8192), (300, 260, 512), (1, 1, 64), (20000, 4096, 1024), (4096, 8192, 28672)):
         rup = lambda v: (v + 255) // 256 * 256
-        want = rup(m * k // 2) + rup(nv.nvfp4_sf_bytes(m, k, nv.SF_TCGEN05)) + rup(64 + 4 * ((m + 255) // 256))
+        chunks = -(-k // 4096)
+        want = (rup(m * k // 2) + rup(nv.nvfp4_sf_bytes(m, k, nv.SF_TCGEN05))
+                + rup(128 + 4 * ((m + 255) // 256) * chunks))
         assert nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, m, n, k) == want
 
 

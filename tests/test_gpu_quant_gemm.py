@@ -1,12 +1,15 @@
 """Quantize-and-multiply (nvfp4_gemm_quant_a and its _prepare / _run and
 _amax forms): a bf16 A quantized inside the call, then the block-scaled GEMM.
-Where one kernel does both (M, N > 128, B's codes <= 64 MiB), its codes,
-scales, g_a and D must equal, bit for bit, those of the quantize pass followed
-by the GEMM, and both must agree with the oracle."""
+Where one kernel does both (M, N > 128), its codes, scales, g_a and D must
+equal, bit for bit, those of the quantize pass followed by the GEMM, and both
+must agree with the oracle.  Both of its schedules are covered: tiles row
+block by row block (B's codes within 64 MiB) and m-fastest tiles with A
+quantized chunk by chunk along K (larger B, the long-K workload)."""
 import numpy as np
 import pytest
 import torch
 
+import oracle_pool
 from oracle import nvfp4_oracle as O
 from nvfp4_block_scaled_15_b200 import inputs
 from parity import check_bf16, check_f32, dev_bf16, f32_scalar, host_bf16_bits, host_u8
@@ -20,6 +23,7 @@ SHAPES = [
     (777, 300, 4096, 8),     # A rows 16-B but not 32-B aligned: 128-bit loads
     (2048, 4096, 8192, 0),   # a full 8192-wide row per quantizer pass, 256 tiles (more than one wave)
     (4352, 384, 12288, 0),   # 17 row blocks, K beyond one pass per row
+    (600, 8488, 16384, 8),   # B's codes > 64 MiB: m-fastest tiles, units chunk by chunk along K; ragged M and N
 ]
 
 
@@ -79,13 +83,18 @@ def test_quant_a_against_oracle_and_two_kernel_path(lib, m, n, k, pad):
 def test_quant_a_bf16_out_prefill_full_size(lib):
     """Prefill workload 8192^3 through the quantize-and-multiply call: the
     whole bf16 D, A's codes and scales equal the two-kernel path's bit for bit;
-    256 sampled outputs against the oracle."""
+    every code byte and scale of A, and 256 sampled outputs, against the
+    oracle."""
     a, w = inputs.prefill_gemm()
     qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
     a_dev = dev_bf16(a)
     d, qa = _check_same_as_two_kernel(lib, a_dev, qw, a.shape[0], a.shape[1], torch.bfloat16)
     assert torch.isfinite(d).all()
-    ga = O.global_scale(O.amax(a))
+    # every code byte and block scale of A (the quantize-and-GEMM kernel's, equal to qa's) against the oracle
+    ca_all, sa_all, ga, _ = oracle_pool.quantize(a)
+    assert f32_scalar(qa.g) == ga
+    assert np.array_equal(host_u8(qa.codes), ca_all)
+    assert np.array_equal(host_u8(qa.sf), O.swizzle_sf_tcgen05(sa_all))
     gw = O.global_scale(O.amax(w))
     rng = np.random.default_rng(41)
     rows = rng.choice(a.shape[0], 256)
@@ -187,3 +196,57 @@ def test_quant_a_non_finite_input(lib):
     assert float(g.item()) == 0.0
     assert not codes.any() and not sf.any()
     assert torch.isnan(d).all()
+
+
+def test_quant_a_long_k_full_size(lib):
+    """Long-K workload: A [4096, 28672] = a*silu(b) quantized inside the call
+    (the m-fastest schedule: W's codes are 117 MB), W [8192, 28672] N(0, 0.02)
+    pre-quantized.  The whole bf16 D, A's codes and scales equal the
+    two-kernel path's bit for bit; every code byte and scale of A, and 256
+    sampled outputs, against the oracle."""
+    a, w = inputs.long_k()
+    qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+    d, qa = _check_same_as_two_kernel(lib, dev_bf16(a), qw, a.shape[0], a.shape[1], torch.bfloat16)
+    assert torch.isfinite(d).all()
+    ca_all, sa_all, ga, _ = oracle_pool.quantize(a)
+    assert f32_scalar(qa.g) == ga
+    assert np.array_equal(host_u8(qa.codes), ca_all)
+    assert np.array_equal(host_u8(qa.sf), O.swizzle_sf_tcgen05(sa_all))
+    gw = O.global_scale(O.amax(w))
+    rng = np.random.default_rng(29)
+    rows = rng.choice(a.shape[0], 256)
+    cols = rng.choice(w.shape[0], 256)
+    uc = np.unique(cols)
+    cw, sw = O.quantize_with_scale(w[uc], gw)
+    d_ref, s_ref, alpha = O.gemm_ref_entries(ca_all, sa_all, ga, O.pack_codes(cw), sw, gw,
+                                             rows, np.searchsorted(uc, cols))
+    check_bf16(host_bf16_bits(d)[rows, cols], d_ref, s_ref, alpha)
+
+
+def test_quant_a_two_streams_at_once(lib):
+    """Two quantize-and-GEMM calls on two streams, three times over: their
+    CTAs compete for the SMs, so each call has CTAs that start only after
+    others of the same launch finished.  Warps take units of A from a ticket
+    counter, so the resident CTAs quantize what their tiles wait for: both
+    calls finish without a wait running out, with the single-call results."""
+    m, n, k = 2048, 4096, 8192
+    outs, refs, args = [], [], []
+    for seed in (501, 502):
+        a, _ = _a_input(m, k, 0, seed=seed)
+        w = inputs.gaussian_bf16((n, k), seed=seed + 1, std=0.02)
+        qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
+        a_dev = dev_bf16(a)
+        refs.append(lib.gemm_quant_a(a_dev, qw))
+        ws = torch.empty(lib.nvfp4_workspace_bytes(lib.OP_GEMM_QUANT_A, m, n, k), dtype=torch.uint8, device="cuda")
+        args.append((a_dev, qw, ws))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for _ in range(3):
+        outs = []
+        for st, (a_dev, qw, ws) in zip(streams, args):
+            with torch.cuda.stream(st):
+                outs.append(lib.gemm_quant_a(a_dev, qw, workspace=ws, stream=st))
+        torch.cuda.synchronize()
+        assert lib.nvfp4_check_device_status() == lib.OK
+        for d, ref in zip(outs, refs):
+            assert torch.equal(d.view(torch.int16), ref.view(torch.int16))
