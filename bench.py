@@ -679,8 +679,14 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
     ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMM_QUANT_A, am, nn, k), dtype=torch.uint8, device=dev)
     ms = _timed(torch, dev, flush, lambda: nv.gemm_quant_a(ad, wq, out=dd, workspace=ws), 10)
     fl = 2.0 * am * nn * k
-    out["long_k_4096x8192x28672"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_fp4_peak": fl / ms / 1e9 / fp4_peak}
-    del wq, ad, dd, ws
+    # the same work as two kernels after the amax pass: the quantize pass, then the plain GEMM
+    qa_l = nv.empty_quantized(am, k, nv.SF_TCGEN05, dev)
+    ms_two = _timed(torch, dev, flush, lambda: (nv.quantize(ad, nv.SF_TCGEN05, out=qa_l), nv.gemm(qa_l, wq, out=dd)),
+                    10)
+    out["long_k_4096x8192x28672"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_fp4_peak": fl / ms / 1e9 / fp4_peak,
+                                     "kernel": "amax pass + quantize-and-GEMM kernel (grouped schedule)",
+                                     "two_kernels_ms": ms_two, "two_kernels_tflops": fl / ms_two / 1e9}
+    del wq, ad, dd, ws, qa_l
 
     # MXFP4 (E8M0 scale per 32, no global scale): one-pass quantize of the
     # same [16384, 8192] input and the 8192^3 GEMM on MXFP4 operands
