@@ -300,9 +300,9 @@ NVFP4_API size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_
  * workspace: device scratch of nvfp4_workspace_bytes(NVFP4_OP_GEMV_BATCHED, M, N, K)
  *   bytes (quantized x, its scales and g, fp32 partial sums, tile counters).
  *   It needs no clearing, before the first call or between calls:
- *     - M > 4: the call's first kernel rewrites the quantized x and zeroes
+ *     - M > 8: the call's first kernel rewrites the quantized x and zeroes
  *       the counters;
- *     - M <= 4: each counter holds a 48-bit tag drawn per launch beside its
+ *     - M <= 8: each counter holds a 48-bit tag drawn per launch beside its
  *       count, and a counter with another tag counts as zero, so stale bytes
  *       are taken for this launch's only by a 2^-48 chance; every launch that
  *       completes returns the counters it used to zero, so a CUDA graph that
@@ -334,8 +334,8 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched(const void* x_bf16, int64_t M, int64_t
  *     capture.  Nothing is allocated or freed, then or later.
  *   Sharing: every call on a device uses the same scratch and overwrites what
  *     the previous call left there; what must start at zero is cleared by the
- *     call (M > 4) or tagged per launch and returned to zero at its end
- *     (M <= 4), as for nvfp4_gemv_batched's workspace.  Calls that overlap on
+ *     call (M > 8) or tagged per launch and returned to zero at its end
+ *     (M <= 8), as for nvfp4_gemv_batched's workspace.  Calls that overlap on
  *     the device race: serialise them, e.g. on one stream.
  * Other arguments, constraints and errors as nvfp4_gemv_batched.
  */

@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Decode GEMV without a prologue (M <= 4, K <= 8192): every CTA quantizes the
+// Decode GEMV without a prologue (M <= 8, K <= 8192): every CTA quantizes the
 // activations itself, at its start, into a resident operand image in shared
 // memory, so the quantized activations never pass through global memory.
 //   * Image: for each 256-wide K stage one 8-row x 128-B tile of codes in the
@@ -350,12 +350,16 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 //     8-row-group stride, i.e. as copies of rows 0..7: they only feed output
 //     columns >= 8, which are never stored.
 //   * The weight ring holds only weights and their scales.
-//   * The four epilogue warps build the image (zero it, amax of x, global
-//     scale, codes and scales of every block) before they turn to the
-//     epilogue.  They meet on an mbarrier (x_sync) after the zeroing and the
-//     amax partials, and each arrives on another (x_ready) once its image
-//     writes are fenced for the tensor core's proxy; the MMA thread waits on
-//     x_ready before its first MMA.
+//   * Sixteen warps build the image (zero it, amax of x, global scale, codes
+//     and scales of every block): the four epilogue warps, which then turn
+//     to the epilogue, and twelve that only do this.  Each thread holds one
+//     16-element block of every row of x in registers (x is read once).  They
+//     meet on an mbarrier (x_sync) after the zeroing and the amax partials,
+//     and each arrives on another (x_ready) once its image writes are fenced
+//     for the tensor core's proxy; the MMA thread waits on x_ready before its
+//     first MMA.  The per-CTA cost grows with M (each CTA quantizes all of x,
+//     read from L2 while the weight stream saturates HBM); up to M = 8 it is
+//     below that of the two-kernel path's hand-off.
 //   * Fix-up counters: (tag << 16) | arrivals, with a 48-bit tag drawn per
 //     launch.  A counter whose tag is not this launch's counts as zero, so
 //     bytes left in the workspace by other use match only by a 2^-48 chance;
@@ -363,17 +367,19 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 //     launch that finishes leaves every counter zero (a replayed graph, whose
 //     launches share one tag, starts from zeros too).
 // ---------------------------------------------------------------------------
-constexpr int GF_MAX_M = 4;                  // rows of x held in registers by the quantizer threads
+constexpr int GF_MAX_M = 8;                  // rows of x held in registers by the quantizer threads
 constexpr int GF_MAX_K = 8192;
-constexpr int GF_BLOCKS = GF_MAX_K / 16 / (GV_EPI_WARPS * 32);   // 16-element blocks per thread and row
+constexpr int GF_QWARPS = 16;                // the 4 epilogue warps and 12 more quantize x
+constexpr int GF_THREADS = (2 + GF_QWARPS) * 32;
+constexpr int GF_BLOCKS = GF_MAX_K / 16 / (GF_QWARPS * 32);      // 16-element blocks per thread and row
 constexpr int GF_STAGES = 8;
 constexpr int GF_STAGE_BYTES = GV_A_BYTES + 4 * SF_ATOM;          // weights + their scales
 constexpr int GF_XIMG_BYTES = (GF_MAX_K / BK) * 1024;             // 8 rows x 128 B per K stage
 constexpr int GF_XSF_BYTES = (GF_MAX_K / MMA_K) * 128;            // 8 rows x 16 B per MMA-K step
-constexpr int GF_SMEM_BYTES = GF_STAGES * GF_STAGE_BYTES + GF_XIMG_BYTES + GF_XSF_BYTES + 1024 + 256 + 1024;
-constexpr int GF_QTHREADS = GV_EPI_WARPS * 32;
+constexpr int GF_SMEM_BYTES = GF_STAGES * GF_STAGE_BYTES + GF_XIMG_BYTES + GF_XSF_BYTES + 1024 + 512 + 1024;
+constexpr int GF_QTHREADS = GF_QWARPS * 32;
 static_assert(GF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(GF_BLOCKS % 2 == 0, "blocks are quantized in pairs");
+static_assert((GF_MAX_M * GF_BLOCKS) % 2 == 0, "blocks are quantized in pairs");
 
 struct GemvFusedParams {
   const uint16_t* x;
@@ -407,7 +413,7 @@ __device__ __forceinline__ int tagged_arrive(unsigned long long* c, unsigned lon
   return 0;   // two contributors per tile cannot contend 64 times; reached only on corruption
 }
 
-__global__ void __launch_bounds__(GV_THREADS, 1)
+__global__ void __launch_bounds__(GF_THREADS, 1)
     gemv_fused_kernel(const __grid_constant__ CUtensorMap tmW, const GemvFusedParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -423,7 +429,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
   uint64_t* x_ready = x_sync + 1;           // the activation image is written and fenced
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* red = tmem_slot + 2;                                     // [GV_EPI_WARPS] amax partials
+  uint32_t* red = tmem_slot + 2;                                     // [GF_QWARPS] amax partials
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -556,7 +562,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       for (int i = qt; i < (GF_XIMG_BYTES + GF_XSF_BYTES) / 16; i += GF_QTHREADS) z[i] = make_uint4(0u, 0u, 0u, 0u);
       fill_scale_table_from(table, qt, GF_QTHREADS);
     }
-    // x, read once into registers: thread qt takes blocks j = qt + 128 i of
+    // x, read once into registers: thread qt takes blocks j = qt + 512 i of
     // every row, block j being x's block (j + rot) % kb.  The rotation differs
     // from CTA to CTA, so the 148 CTAs, which all read the whole of x, do not
     // all ask the same L2 lines for the same data at the same moment.
@@ -589,7 +595,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     (void)mbar_wait_bounded(x_sync, 0, abort_flag, p.wait_limit_ns, p.status);
     uint32_t all = 0;
 #pragma unroll
-    for (int i = 0; i < GV_EPI_WARPS; ++i) all = max(all, red[i]);
+    for (int i = 0; i < GF_QWARPS; ++i) all = max(all, red[i]);
     bool valid;
     float g = global_scale_from_amax(__uint_as_float(all << 16), valid);
     if (blockIdx.x == 0 && qt == 0 && !valid) record_status(p.status, kDevRange);
@@ -597,32 +603,30 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     // block b of row r lands in K stage b / 16, 16-B chunk (b % 16) / 2
     // (swizzled with r), half b % 2, and its scale in MMA-K step b / 4
     if (valid) {
+      // the thread's (row, block) entries f = r * GF_BLOCKS + i, two at a time
+      auto store = [&](int r, int j, uint2 c, uint32_t sc) {
+        if (j >= kb) return;
+        const int b = j + rot < kb ? j + rot : j + rot - kb;
+        *reinterpret_cast<uint2*>(ximg + (b >> 4) * 1024 + r * 128 + ((((b & 15) >> 1) ^ r) << 4) + (b & 1) * 8) = c;
+        xsfimg[(b >> 2) * 128 + r * 16 + (b & 3)] = static_cast<uint8_t>(sc);
+      };
 #pragma unroll
-      for (int r = 0; r < GF_MAX_M; ++r) {
-        if (r >= p.M) break;
-#pragma unroll
-        for (int i = 0; i < GF_BLOCKS; i += 2) {
-          const int j0 = qt + GF_QTHREADS * i, j1 = j0 + GF_QTHREADS;
-          uint2 c0, c1;
-          uint32_t s0, s1;
-          quantize_two_blocks(w[r][i], w[r][i + 1], g, table, c0, c1, s0, s1);
-          if (j0 < kb) {
-            const int b = j0 + rot < kb ? j0 + rot : j0 + rot - kb;
-            *reinterpret_cast<uint2*>(ximg + (b >> 4) * 1024 + r * 128 + ((((b & 15) >> 1) ^ r) << 4) + (b & 1) * 8) = c0;
-            xsfimg[(b >> 2) * 128 + r * 16 + (b & 3)] = static_cast<uint8_t>(s0);
-          }
-          if (j1 < kb) {
-            const int b = j1 + rot < kb ? j1 + rot : j1 + rot - kb;
-            *reinterpret_cast<uint2*>(ximg + (b >> 4) * 1024 + r * 128 + ((((b & 15) >> 1) ^ r) << 4) + (b & 1) * 8) = c1;
-            xsfimg[(b >> 2) * 128 + r * 16 + (b & 3)] = static_cast<uint8_t>(s1);
-          }
-        }
+      for (int f = 0; f < GF_MAX_M * GF_BLOCKS; f += 2) {
+        const int r0 = f / GF_BLOCKS, i0 = f % GF_BLOCKS;
+        const int r1 = (f + 1) / GF_BLOCKS, i1 = (f + 1) % GF_BLOCKS;
+        if (r0 >= p.M) break;
+        uint2 c0, c1;
+        uint32_t s0, s1;
+        quantize_two_blocks(w[r0][i0], w[r1][i1], g, table, c0, c1, s0, s1);
+        store(r0, qt + GF_QTHREADS * i0, c0, s0);
+        if (r1 < p.M) store(r1, qt + GF_QTHREADS * i1, c1, s1);
       }
     }
     fence_proxy_async_shared();                 // generic-proxy writes, read by the tensor core
     mbar_arrive(x_ready);
 
-    // ---- epilogue and stream-K fix-up (as gemv_kernel, tagged counters) ----
+    // ---- epilogue and stream-K fix-up (warps 2..5; as gemv_kernel, tagged counters) ----
+    if (warp < 2 + GV_EPI_WARPS) {
     const int quad = warp & 3;
     const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.g_w, valid ? g : 0.0f));
     const int cta = blockIdx.x;
@@ -699,6 +703,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         }
         if (lane == 0) *reinterpret_cast<volatile unsigned long long*>(counter) = 0ull;   // tile done: reset
       }
+    }
     }
   }
 
@@ -946,7 +951,7 @@ static nvfp4_status launch_gemv_fused(const void* x, int64_t M, int64_t ldx, con
   if (grid > GV_MAX_CTAS) grid = GV_MAX_CTAS;
   cudaError_t e = cudaFuncSetAttribute(gemv_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GF_SMEM_BYTES);
   if (e != cudaSuccess) return launch_status(e);
-  gemv_fused_kernel<<<grid, GV_THREADS, GF_SMEM_BYTES, s>>>(tmW, p);
+  gemv_fused_kernel<<<grid, GF_THREADS, GF_SMEM_BYTES, s>>>(tmW, p);
   return launch_status(cudaGetLastError());
 }
 

@@ -78,9 +78,9 @@ extern "C" NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16,
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch)) != NVFP4_OK) return st;
   // The existing GEMV paths, given the fixed scratch as their workspace.
-  // Nothing from an earlier call is reused: with M > 4 the prologue rewrites
+  // Nothing from an earlier call is reused: with M > 8 the prologue rewrites
   // the quantized activations and clears the counters on every call; with
-  // M <= 4 the activations stay in shared memory and the counters carry a
+  // M <= 8 the activations stay in shared memory and the counters carry a
   // per-launch tag (any other call's counts read as zero) and are returned
   // to zero by the launch; partial sums are always written before they are
   // read.

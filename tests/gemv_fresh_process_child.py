@@ -8,7 +8,7 @@ against the oracle:
     words are all 1 (stale small counts) before the call;
   * nvfp4_gemv_batched_noalloc, M = 1, 4, 8, 20, 1, 16, 4 interleaved: the
     library's fixed scratch, which each call leaves to the next (an M = 20
-    or M = 8 or 16 call, two kernels, leaves 32-bit counts where the M <= 4
+    or M = 16 call, two kernels, leaves 32-bit counts where the M <= 8
     kernel keeps its 64-bit tagged counters).
 Usage: python gemv_fresh_process_child.py OUT.npz
 """

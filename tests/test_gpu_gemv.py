@@ -1,6 +1,6 @@
 """Decode batched GEMV parity (activations quantized inside the call).
 
-Two paths serve the call: for M <= 4 and K <= 8192 one kernel whose CTAs
+Two paths serve the call: for M <= 8 and K <= 8192 one kernel whose CTAs
 each quantize the activations (held in registers) into shared memory, and
 otherwise a quantizing prologue followed by the GEMV; the shapes below reach
 both, with ragged N, K not a multiple of 256 and tiles split between CTAs."""
@@ -103,7 +103,7 @@ def test_gemv_decode_full_size_sampled(lib, m):
     check_bf16(host_bf16_bits(y)[:, cols], d_ref, s_ref, alpha)
 
 
-@pytest.mark.parametrize("m", [1, 4, 9, 16])
+@pytest.mark.parametrize("m", [1, 4, 8, 9, 16])
 def test_gemv_weights_in_l2_repeated(lib, m):
     """All 148 CTAs running (160 weight tiles) with 94 MB of weights resident in
     L2, so the weight stages reach the tensor core while the CTAs are still

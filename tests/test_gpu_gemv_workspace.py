@@ -1,6 +1,6 @@
 """The GEMV's workspace contract, at the decode workload's full size.
 
-The stream-K fix-up counters of the one-kernel path (M <= 4) are never
+The stream-K fix-up counters of the one-kernel path (M <= 8) are never
 cleared by a separate step: each carries a per-launch tag, and each launch returns the
 counters it used to zero.  These tests check, against the oracle on every
 output, that

@@ -52,7 +52,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, m, n, k):
 @pytest.mark.parametrize("m", [1, 4])
 def test_noalloc_decode_size_split_tiles_on_two_calls(lib, m):
     """The decode workload (W [28672, 8192]: tiles split between CTAs) at
-    M <= 4, the kernel whose fix-up counters live in the shared scratch from
+    M <= 8, the kernel whose fix-up counters live in the shared scratch from
     one call to the next: two calls in a row, each equal bit for bit to the
     workspace entry point's output, and 512 sampled columns against the
     oracle."""
