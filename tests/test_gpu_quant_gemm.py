@@ -23,7 +23,8 @@ SHAPES = [
     (777, 300, 4096, 8),     # A rows 16-B but not 32-B aligned: 128-bit loads
     (2048, 4096, 8192, 0),   # a full 8192-wide row per quantizer pass, 256 tiles (more than one wave)
     (4352, 384, 12288, 0),   # 17 row blocks, K beyond one pass per row
-    (600, 8488, 16384, 8),   # B's codes > 64 MiB: m-fastest tiles, units chunk by chunk along K; ragged M and N
+    (600, 8488, 16384, 8),   # B's codes > 64 MiB (one group of 3 row blocks); ragged M and N
+    (2100, 8488, 16384, 0),  # B's codes > 64 MiB: 9 row blocks in 3 groups of 3, the last row block 52 rows
 ]
 
 
