@@ -353,8 +353,11 @@ NVFP4_API nvfp4_status nvfp4_gemv_batched_noalloc(const void* x_bf16, int64_t M,
  *   the amax pass: extra warps quantize A in units (one row, 4096 elements
  *   of K) while the tensor cores multiply the parts already done.  Where B's
  *   codes (N * K / 2 bytes) are at most 64 MiB the tiles go row block by row
- *   block and A is quantized row by row; larger B (long K) takes the tiles
- *   m-fastest and A chunk by chunk along K, so B is read from DRAM once.
+ *   block and A is quantized row by row (B stays in L2); for larger B (long
+ *   K) the 256-row blocks form about four groups, taken in turn, with the
+ *   tiles m-fastest inside a group and A quantized chunk by chunk along K, so
+ *   B is read from DRAM about four times and the first tiles wait for one
+ *   chunk of a quarter of A.
  *   Other shapes run the quantize pass and the GEMM as two kernels.  All
  *   give the same codes, scales, g_a and D bit for bit.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_QUANT_A, M, N, K) bytes:
