@@ -83,9 +83,10 @@ def test_quant_a_against_oracle_and_two_kernel_path(lib, m, n, k, pad):
 
 def test_quant_a_bf16_out_prefill_full_size(lib):
     """Prefill workload 8192^3 through the quantize-and-multiply call: the
-    whole bf16 D, A's codes and scales equal the two-kernel path's bit for bit;
-    every code byte and scale of A, and 256 sampled outputs, against the
-    oracle."""
+    whole bf16 D, A's codes and scales equal the two-kernel path's bit for bit
+    (whose D tests/test_gpu_gemm.py::test_gemm_prefill_full_size checks
+    against the oracle on every output); every code byte and scale of A, and
+    256 sampled outputs, against the oracle."""
     a, w = inputs.prefill_gemm()
     qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
     a_dev = dev_bf16(a)
@@ -203,8 +204,8 @@ def test_quant_a_long_k_full_size(lib):
     """Long-K workload: A [4096, 28672] = a*silu(b) quantized inside the call
     (the m-fastest schedule: W's codes are 117 MB), W [8192, 28672] N(0, 0.02)
     pre-quantized.  The whole bf16 D, A's codes and scales equal the
-    two-kernel path's bit for bit; every code byte and scale of A, and 256
-    sampled outputs, against the oracle."""
+    two-kernel path's bit for bit; every code byte and scale of A and W, and
+    every one of the 33,554,432 outputs, against the oracle."""
     a, w = inputs.long_k()
     qw = lib.quantize(dev_bf16(w), lib.SF_TCGEN05)
     d, qa = _check_same_as_two_kernel(lib, dev_bf16(a), qw, a.shape[0], a.shape[1], torch.bfloat16)
@@ -213,15 +214,10 @@ def test_quant_a_long_k_full_size(lib):
     assert f32_scalar(qa.g) == ga
     assert np.array_equal(host_u8(qa.codes), ca_all)
     assert np.array_equal(host_u8(qa.sf), O.swizzle_sf_tcgen05(sa_all))
-    gw = O.global_scale(O.amax(w))
-    rng = np.random.default_rng(29)
-    rows = rng.choice(a.shape[0], 256)
-    cols = rng.choice(w.shape[0], 256)
-    uc = np.unique(cols)
-    cw, sw = O.quantize_with_scale(w[uc], gw)
-    d_ref, s_ref, alpha = O.gemm_ref_entries(ca_all, sa_all, ga, O.pack_codes(cw), sw, gw,
-                                             rows, np.searchsorted(uc, cols))
-    check_bf16(host_bf16_bits(d)[rows, cols], d_ref, s_ref, alpha)
+    pw, sw, gw, _ = oracle_pool.quantize(w)
+    assert f32_scalar(qw.g) == gw and np.array_equal(host_u8(qw.codes), pw)
+    d_ref, s_ref, alpha = oracle_pool.gemm_ref(ca_all, sa_all, ga, pw, sw, gw)
+    check_bf16(host_bf16_bits(d), d_ref, s_ref, alpha)
 
 
 def test_quant_a_two_streams_at_once(lib):
