@@ -95,17 +95,23 @@ def kernel_code_hash(files):
 TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def profile_traffic(name):
-    """DRAM bytes per launch of a kernel from one ncu capture, kept in
-    profiles/traffic.json by ``--record-traffic``; None when the kernel's code
-    (comments and layout aside) changed after the capture."""
+def profile_entry(name):
+    """One ncu capture's figures for a kernel, kept in profiles/traffic.json by
+    ``--record-traffic``; None when the kernel's code (comments and layout
+    aside) changed after the capture."""
     if not os.path.exists(TRAFFIC_JSON):
         return None
     with open(TRAFFIC_JSON) as f:
         entry = json.load(f).get(name)
     if not entry or entry.get("code_hash") != kernel_code_hash(entry["sources"]):
         return None
-    return int(entry["dram_bytes_per_launch"])
+    return entry
+
+
+def profile_traffic(name):
+    """DRAM bytes per launch of a kernel from its ncu capture (or None)."""
+    entry = profile_entry(name)
+    return None if entry is None else int(entry["dram_bytes_per_launch"])
 
 
 def record_traffic(name, raw_csv, sources, launches, command):
@@ -121,10 +127,16 @@ def record_traffic(name, raw_csv, sources, launches, command):
     units_row = rows[rows.index(head) + 1]
     scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
     vals = []
+    pct = {"tensor_pipe_busy_pct": "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed",
+           "dram_throughput_pct": "gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed"}
+    pct_vals = {k: [] for k in pct}
     for r in rows[rows.index(head) + 2:]:
         if len(r) > max(i_r, i_w) and r[i_r]:
             vals.append(float(r[i_r].replace(",", "")) * scale[units_row[i_r]]
                         + float(r[i_w].replace(",", "")) * scale[units_row[i_w]])
+            for k, metric in pct.items():
+                if metric in head and r[head.index(metric)]:
+                    pct_vals[k].append(float(r[head.index(metric)].replace(",", "")))
     if len(vals) != launches:
         raise SystemExit(f"{len(vals)} launches in {raw_csv}, expected {launches}")
     data = {}
@@ -133,6 +145,9 @@ def record_traffic(name, raw_csv, sources, launches, command):
             data = json.load(f)
     data[name] = {"dram_bytes_per_launch": int(round(sum(vals) / len(vals))), "sources": sources,
                   "code_hash": kernel_code_hash(sources), "launches": launches, "command": command}
+    for k, v in pct_vals.items():
+        if len(v) == launches:
+            data[name][k] = round(sum(v) / len(v), 2)
     with open(TRAFFIC_JSON, "w") as f:
         json.dump(data, f, indent=1, sort_keys=True)
         f.write("\n")
@@ -409,7 +424,8 @@ def main():
     if rank == 0:
         fused_avg = statistics.mean(fused_ms)
         achieved = FLOPS_STEP / (fused_avg * 1e-3) / 1e12
-        traffic = profile_traffic("quant_gemm_prefill_8192")
+        prof = profile_entry("quant_gemm_prefill_8192")
+        traffic = None if prof is None else int(prof["dram_bytes_per_launch"])
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -417,6 +433,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp4_peak, "traffic": traffic,
                          "frac_of_nominal_dense_fp4": achieved / NOMINAL_FP4_TFLOPS,
+                         "tensor_pipe_busy_pct_ncu": None if prof is None else prof.get("tensor_pipe_busy_pct"),
                          "kernel": "gemm_pair_kernel<quantize A> (extra warps quantize the bf16 A row block by "
                                    "row block; tcgen05.mma.cta_group::2 kind::mxf4nvf4, 256x256 tiles, 8192^3)",
                          "peak_source": f"{peaks_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} "
@@ -444,7 +461,8 @@ def main():
         result["parts"]["gemm_only"] = {
             "ms": ms_g, "tflops": FLOPS_STEP / (ms_g * 1e-3) / 1e12,
             "frac_fp4_peak": FLOPS_STEP / (ms_g * 1e-3) / 1e12 / fp4_peak,
-            "traffic": profile_traffic("gemm_prefill_8192")}
+            "traffic": profile_traffic("gemm_prefill_8192"),
+            "tensor_pipe_busy_pct_ncu": (profile_entry("gemm_prefill_8192") or {}).get("tensor_pipe_busy_pct")}
     if rank == 0 and world == 1 and not args.no_cpu:
         sample = OracleSample(a_bits, w_bits, rows=8192, cols=2048)
         sec = time_oracle(sample)
