@@ -24,9 +24,10 @@ NVCC_FLAGS = [
     # IEEE division by default.  Contraction of a*b+c into an FMA stays
     # allowed (-fmad=true) for the GEMM and GEMV epilogues; every fp32 step
     # of the quantizers whose rounding is part of the definition is written
-    # with an explicit round-to-nearest intrinsic (__fmul_rn, __fadd_rn,
-    # __fmaf_rn, __fdiv_rn, or the packed .rn PTX forms), which the compiler
-    # never contracts, so their codes match the CPU definition bit for bit.
+    # with an explicit rounding intrinsic (__fmul_rn, __fadd_rn, __fmaf_rn,
+    # __fdiv_rn, the round-up __fadd_ru of the stochastic rounding, or the
+    # packed .rn PTX forms), which the compiler never contracts, so their
+    # codes match the CPU definition bit for bit.
     "-prec-div=true", "-fmad=true",
 ]
 

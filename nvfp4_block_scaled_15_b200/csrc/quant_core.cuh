@@ -201,27 +201,29 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 // Stochastic rounding of two values onto the E2M1 grid, with 16-bit random
 // integers (element x's in bits 0..15 of r, y's in bits 16..31): a magnitude
 // a lies between neighbours lo and hi = lo + step (step 0.5 below 2, 1 below
-// 4, 2 below 6); it rounds up when r < f * 2^16, f = (a - lo) / step; a >= 6
-// gives 6; the sign of u is kept.  Every step is exact in fp32: v = a / step
-// is a power-of-two scaling, floor(v) and v - floor(v) are exact, and
-// f * 2^16 and r are exact, so the comparison is the real one.  The
-// multiplies, the fraction and the step product run on the packed fp32x2
-// units.
+// 4, 2 below 6); it rounds up when R < f * 2^16, f = (a - lo) / step; a >= 6
+// gives 6; the sign of u is kept.
+//
+// On the fp32 bits.  From 1 up, the grid keeps one mantissa bit: lo is a's
+// bits with the low 22 mantissa bits cleared, and f * 2^16 = rem / 64 for
+// rem those 22 bits, so "up" is rem > 64 R, which is exactly when
+// rem + (2^22 - 1 - 64 R) carries into bit 22.  Adding that constant and
+// clearing the low 22 bits therefore gives lo or hi (the carry runs into the
+// exponent where hi starts the next binade).  Below 1 the grid has step 0.5,
+// which is the same one-bit grid shifted by 1: b = a + 1 rounded up.  Only
+// ceil(f * 2^16) decides "R < f * 2^16" for an integer R, and rounding the
+// sum up to b's ulp (2^-23, finer than f's 2^-17 granularity) keeps that
+// ceiling, so b's bits decide exactly; 1 is subtracted afterwards (exact).
+// Values from 6 up land on 6, 8 or more, which the conversion's satfinite
+// turns into 6.
 __device__ __forceinline__ float2 e2m1_round_stochastic2(float2 u, uint32_t r) {
   const float ax = fabsf(u.x), ay = fabsf(u.y);
-  const float2 inv = make_float2(ax < 2.0f ? 2.0f : (ax < 4.0f ? 1.0f : 0.5f),
-                                 ay < 2.0f ? 2.0f : (ay < 4.0f ? 1.0f : 0.5f));
-  const float2 v = __fmul2_rn(make_float2(ax, ay), inv);
-  const float2 fl = make_float2(floorf(v.x), floorf(v.y));
-  const float2 thr = __fmul2_rn(__ffma2_rn(fl, make_float2(-1.0f, -1.0f), v), make_float2(65536.0f, 65536.0f));
-  const float2 up = make_float2(static_cast<float>(r & 0xFFFFu) < thr.x ? 1.0f : 0.0f,
-                                static_cast<float>(r >> 16) < thr.y ? 1.0f : 0.0f);
-  // step = 1 / inv exactly: for a power of two 2^e, 2^-e has bits 0x7F000000 - bits(2^e);
-  // a >= 6 gives 6 through the minimum (a in [6, 8) lands on 6 or 8), inf included
-  const float2 step = make_float2(__uint_as_float(0x7F000000u - __float_as_uint(inv.x)),
-                                  __uint_as_float(0x7F000000u - __float_as_uint(inv.y)));
-  const float2 m = __fmul2_rn(__fadd2_rn(fl, up), step);
-  return make_float2(copysignf(fminf(m.x, 6.0f), u.x), copysignf(fminf(m.y, 6.0f), u.y));
+  const float2 c = make_float2(ax < 1.0f ? 1.0f : 0.0f, ay < 1.0f ? 1.0f : 0.0f);
+  const uint32_t bx = __float_as_uint(__fadd_ru(ax, c.x)), by = __float_as_uint(__fadd_ru(ay, c.y));
+  const uint32_t kx = 0x3FFFFFu - ((r & 0xFFFFu) << 6), ky = 0x3FFFFFu - ((r >> 16) << 6);
+  const float2 t = make_float2(__uint_as_float((bx + kx) & 0xFFC00000u), __uint_as_float((by + ky) & 0xFFC00000u));
+  const float2 m = __fadd2_rn(t, make_float2(-c.x, -c.y));
+  return make_float2(copysignf(m.x, u.x), copysignf(m.y, u.y));
 }
 
 // 16 codes of one bf16 block for the scale entry e = {sd, RN(1/sd)} with

@@ -366,24 +366,129 @@ __device__ __forceinline__ float rotated_absmax(const uint32_t (&w)[8], int n) {
   return m;
 }
 
+// Orders n >= 32 with the thread's two blocks adjacent (p0 = elements
+// 32j .. 32j + 15 of the segment, p1 = 32j + 16 .. 32j + 31): stage h = 16
+// pairs p0 with p1 inside the thread, and a stage h >= 32 pairs lanes tid and
+// tid ^ (h/32), one cross-lane stage fewer than with one block per lane.
+__device__ __forceinline__ void fwht_pair_stage16(float2 (&p0)[8], float2 (&p1)[8]) {
+  const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 a = p0[i], b = p1[i];
+    p0[i] = __fadd2_rn(a, b);
+    p1[i] = __ffma2_rn(b, m1, a);
+  }
+}
+
+// Stages h = 32, 64, ... below h_end across lanes (lane mask lm = h/32), the
+// sign rule of fwht_cross_lanes.
+__device__ __forceinline__ void fwht_pair_cross_lanes(float2 (&p0)[8], float2 (&p1)[8], int h_end) {
+#pragma unroll
+  for (int lm = 1; lm < 16; lm <<= 1) {
+    if (32 * lm < h_end) {
+      const float sg = (threadIdx.x & lm) ? -1.0f : 1.0f;
+      const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 o0 = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p0[i].x, lm),
+                                      __shfl_xor_sync(0xFFFFFFFFu, p0[i].y, lm));
+        const float2 o1 = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p1[i].x, lm),
+                                      __shfl_xor_sync(0xFFFFFFFFu, p1[i].y, lm));
+        p0[i] = __ffma2_rn(p0[i], s2, o0);
+        p1[i] = __ffma2_rn(p1[i], s2, o1);
+      }
+    }
+  }
+}
+
+// y = x H for the thread's two adjacent blocks (n >= 32), c = fp32(1/sqrt(n)).
+__device__ __forceinline__ void rotate_pair(const uint32_t (&w0)[8], const uint32_t (&w1)[8], int n, float c,
+                                            float2 (&p0)[8], float2 (&p1)[8]) {
+  bf16_block_to_f32(w0, p0);
+  bf16_block_to_f32(w1, p1);
+  fwht_in_thread(p0, 16);
+  fwht_in_thread(p1, 16);
+  fwht_pair_stage16(p0, p1);
+  fwht_pair_cross_lanes(p0, p1, n);
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    p0[i] = __fmul2_rn(p0[i], c2);
+    p1[i] = __fmul2_rn(p1[i], c2);
+  }
+}
+
+// max |y / c| over the thread's two adjacent blocks (n >= 32), the last stage
+// folded into the maximum as in rotated_absmax.  For n = 32 it is stage 16,
+// inside the thread; beyond, the lane with bit lm clear takes the pair's
+// positions 0..15 (its p0 and the partner's), the partner positions 16..31,
+// so each lane sends 16 values.
+__device__ __forceinline__ float rotated_absmax_pair(const uint32_t (&w0)[8], const uint32_t (&w1)[8], int n) {
+  float2 p0[8], p1[8];
+  bf16_block_to_f32(w0, p0);
+  bf16_block_to_f32(w1, p1);
+  fwht_in_thread(p0, 16);
+  fwht_in_thread(p1, 16);
+  float m = 0.0f;
+  if (n == 32) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      m = max3_nan_f32(m, __fadd_rn(fabsf(p0[i].x), fabsf(p1[i].x)), __fadd_rn(fabsf(p0[i].y), fabsf(p1[i].y)));
+    return m;
+  }
+  fwht_pair_stage16(p0, p1);
+  fwht_pair_cross_lanes(p0, p1, n >> 1);
+  const int lm = n >> 6;                        // last stage h = n/2
+  const bool upper = (threadIdx.x & lm) != 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 send = upper ? p0[i] : p1[i];
+    const float2 own = upper ? p1[i] : p0[i];
+    const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, send.x, lm), __shfl_xor_sync(0xFFFFFFFFu, send.y, lm));
+    m = max3_nan_f32(m, __fadd_rn(fabsf(own.x), fabsf(o.x)), __fadd_rn(fabsf(own.y), fabsf(o.y)));
+  }
+  return m;
+}
+
+// Smallest order whose amax pass and stochastic quantize pass take two
+// adjacent blocks per thread (at 128 the amax pass measured 3 % faster, at
+// 256 and 512 8-10 %; at 32 and 64 within noise or slower).
+constexpr int kAdjMinOrder = 128;
+
+// The thread's two blocks of a 512-block segment: b1 = b0 + kThreads (one
+// block per lane in each half), or, with kAdj, b0 = 2 * tid and b1 = b0 + 1.
+template <bool kAdj>
+__device__ __forceinline__ void segment_blocks(int& b0, int& b1) {
+  if (kAdj) {
+    b0 = blockIdx.y * kSegBlocks + 2 * static_cast<int>(threadIdx.x);
+    b1 = b0 + 1;
+  } else {
+    b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
+    b1 = b0 + kThreads;
+  }
+}
+
 // Pass 1 of the rotated quantizer: max |y| over the tensor.  grid.x strides
 // over rows, grid.y over segments of 512 blocks.  The maximum of |y / c|
 // propagates NaN (a NaN or an infinity in y reaches the global amax, and the
 // quantize pass reports it); the one multiply by c at the end gives max |y|
 // exactly, since RN(c v) is monotone in v.
-template <bool kWide>
+template <bool kWide, bool kAdj>
 __global__ void __launch_bounds__(kThreads) hadamard_amax_kernel(const uint16_t* __restrict__ x, int rows, int k,
                                                                  int64_t ldx, int n, float c,
                                                                  unsigned* __restrict__ amax_bits) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int kb = k >> 4;
-  const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
-  const int b1 = b0 + kThreads;
+  int b0, b1;
+  segment_blocks<kAdj>(b0, b1);
   float mf = 0.0f;
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
     uint32_t w0[8], w1[8];
     load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, true, kb, b0, b1, w0, w1);
-    mf = max3_nan_f32(mf, rotated_absmax(w0, n), rotated_absmax(w1, n));
+    if (kAdj)
+      mf = max3_nan_f32(mf, rotated_absmax_pair(w0, w1, n), 0.0f);
+    else
+      mf = max3_nan_f32(mf, rotated_absmax(w0, n), rotated_absmax(w1, n));
   }
   // non-negative floats (NaN as the canonical positive pattern) order as their bits
   uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mf));
@@ -420,17 +525,18 @@ __device__ __forceinline__ uint2 quantize_rotated_block(const float2 (&p)[8], fl
 // the codes, the random words of block b of row r from Philox4x32-10 with
 // key (seed_lo, seed_hi) and counters (2b + h, r, offset_lo, offset_hi), as in
 // quantize_sr_kernel (positions in y).
-template <bool kTcLayout, bool kWide, bool kSR, int kRows>
-__global__ void __launch_bounds__(kThreads)
-    hadamard_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
-                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
-                             const float* __restrict__ amax_in, uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo,
-                             uint32_t off_hi, int* __restrict__ status) {
+template <bool kTcLayout, bool kWide, bool kSR, bool kAdj, int kRows>
+__device__ __forceinline__ void hadamard_quantize_body(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx,
+                                                       int n, float c, uint8_t* __restrict__ codes,
+                                                       uint8_t* __restrict__ sf, float* __restrict__ g_out,
+                                                       const float* __restrict__ amax_in, uint32_t seed_lo,
+                                                       uint32_t seed_hi, uint32_t off_lo, uint32_t off_hi,
+                                                       int* __restrict__ status) {
   __shared__ float2 table[128];
   const int r0 = static_cast<int>(gridDim.x - 1 - blockIdx.x) * kRows;
   const int kb = k >> 4;
-  const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
-  const int b1 = b0 + kThreads;
+  int b0, b1;
+  segment_blocks<kAdj>(b0, b1);
 
   uint32_t w0[kRows][8], w1[kRows][8];         // x and the table before the wait, as in quantize_kernel
 #pragma unroll
@@ -459,6 +565,23 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t ur = static_cast<uint32_t>(r);
     uint2 c0, c1;
     uint32_t s0, s1;
+    if constexpr (kAdj) {                      // both blocks rotated together, then quantized one by one
+      float2 p0[8], p1[8];
+      rotate_pair(w0[j], w1[j], n, c, p0, p1);
+      uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+      if (kSR) {
+        ra = philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi);
+        rb = philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+      }
+      c0 = quantize_rotated_block<kSR>(p0, g, table, s0, ra, rb);
+      if (kSR) {
+        ra = philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi);
+        rb = philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi);
+      }
+      c1 = quantize_rotated_block<kSR>(p1, g, table, s1, ra, rb);
+      store_two_blocks<kTcLayout>(codes, sf, r, r < rows, k, kb, b0, b1, c0, c1, s0, s1);
+      continue;
+    }
     {
       float2 p[8];
       rotate_block(w0[j], n, c, p);
@@ -481,6 +604,28 @@ __global__ void __launch_bounds__(kThreads)
     }
     store_two_blocks<kTcLayout>(codes, sf, r, r < rows, k, kb, b0, b1, c0, c1, s0, s1);
   }
+}
+
+template <bool kTcLayout, bool kWide, bool kSR, int kRows>
+__global__ void __launch_bounds__(kThreads)
+    hadamard_quantize_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
+                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
+                             const float* __restrict__ amax_in, uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo,
+                             uint32_t off_hi, int* __restrict__ status) {
+  hadamard_quantize_body<kTcLayout, kWide, kSR, false, kRows>(x, rows, k, ldx, n, c, codes, sf, g_out, amax_in,
+                                                              seed_lo, seed_hi, off_lo, off_hi, status);
+}
+
+// The stochastic pass with two adjacent blocks per thread, held to 64
+// registers (4 CTAs per SM): uncapped it takes 72 and 3 CTAs per SM.
+template <bool kTcLayout, bool kWide>
+__global__ void __launch_bounds__(kThreads, 4)
+    hadamard_quantize_sr_adj_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, int n, float c,
+                                    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                    float* __restrict__ g_out, const float* __restrict__ amax_in, uint32_t seed_lo,
+                                    uint32_t seed_hi, uint32_t off_lo, uint32_t off_hi, int* __restrict__ status) {
+  hadamard_quantize_body<kTcLayout, kWide, true, true, 1>(x, rows, k, ldx, n, c, codes, sf, g_out, amax_in, seed_lo,
+                                                          seed_hi, off_lo, off_hi, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -607,7 +752,7 @@ cudaError_t launch_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, in
                             status);
 }
 
-template <bool kTc, bool kWide, bool kSR>
+template <bool kTc, bool kWide, bool kSR, bool kAdj>
 cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
                                          int n, float c, uint8_t* codes, uint8_t* sf, float* g_dev,
                                          const float* amax_dev, uint64_t seed, uint64_t offset, int* status) {
@@ -620,6 +765,10 @@ cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if constexpr (kAdj)
+    return cudaLaunchKernelEx(&cfg, hadamard_quantize_sr_adj_kernel<kTc, kWide>, x, rows, k, ldx, n, c, codes, sf,
+                              g_dev, amax_dev, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
+                              static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32), status);
   return cudaLaunchKernelEx(&cfg, hadamard_quantize_kernel<kTc, kWide, kSR, kSR ? 1 : kQuantRows>, x, rows, k, ldx,
                             n, c, codes, sf,
                             g_dev, amax_dev, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
@@ -742,30 +891,54 @@ nvfp4_status launch_hadamard_amax(const void* x, int64_t rows, int64_t k, int64_
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   unsigned* out = reinterpret_cast<unsigned*>(amax_dev);
   const float c = hadamard_norm(n);
-  if (wide)
-    hadamard_amax_kernel<true><<<dim3(gx, segs), kThreads, 0, s>>>(xs, static_cast<int>(rows), static_cast<int>(k),
-                                                                   ldx, n, c, out);
-  else
-    hadamard_amax_kernel<false><<<dim3(gx, segs), kThreads, 0, s>>>(xs, static_cast<int>(rows), static_cast<int>(k),
-                                                                    ldx, n, c, out);
+  const dim3 grid(gx, segs);
+  const int ri = static_cast<int>(rows), ki = static_cast<int>(k);
+  if (n >= kAdjMinOrder) {                      // two adjacent blocks per thread
+    if (wide)
+      hadamard_amax_kernel<true, true><<<grid, kThreads, 0, s>>>(xs, ri, ki, ldx, n, c, out);
+    else
+      hadamard_amax_kernel<false, true><<<grid, kThreads, 0, s>>>(xs, ri, ki, ldx, n, c, out);
+  } else if (wide) {
+    hadamard_amax_kernel<true, false><<<grid, kThreads, 0, s>>>(xs, ri, ki, ldx, n, c, out);
+  } else {
+    hadamard_amax_kernel<false, false><<<grid, kThreads, 0, s>>>(xs, ri, ki, ldx, n, c, out);
+  }
   return launch_status(cudaGetLastError());
 }
 
 namespace {
 
+template <bool kSR, bool kAdj>
+cudaError_t dispatch_hadamard_layout(dim3 grid, bool tc, bool wide, cudaStream_t s, const uint16_t* x, int rows,
+                                     int k, int64_t ldx, int n, float c, uint8_t* codes, uint8_t* sf, float* g_dev,
+                                     const float* amax_dev, uint64_t seed, uint64_t offset, int* status) {
+  if (tc)
+    return wide ? launch_hadamard_quantize_pdl<true, true, kSR, kAdj>(grid, s, x, rows, k, ldx, n, c, codes, sf,
+                                                                      g_dev, amax_dev, seed, offset, status)
+                : launch_hadamard_quantize_pdl<true, false, kSR, kAdj>(grid, s, x, rows, k, ldx, n, c, codes, sf,
+                                                                       g_dev, amax_dev, seed, offset, status);
+  return wide ? launch_hadamard_quantize_pdl<false, true, kSR, kAdj>(grid, s, x, rows, k, ldx, n, c, codes, sf,
+                                                                     g_dev, amax_dev, seed, offset, status)
+              : launch_hadamard_quantize_pdl<false, false, kSR, kAdj>(grid, s, x, rows, k, ldx, n, c, codes, sf,
+                                                                      g_dev, amax_dev, seed, offset, status);
+}
+
+// The stochastic pass takes two adjacent blocks per thread for orders
+// n >= 128 (one cross-lane stage fewer; measured faster there).  The
+// rounded-to-nearest pass keeps one block per lane and two rows per CTA: with
+// adjacent blocks it needs one row per CTA for its registers and measured
+// slower, the loads in flight counting for more than the shuffles saved.
 template <bool kSR>
 cudaError_t dispatch_hadamard_quantize(dim3 grid, bool tc, bool wide, cudaStream_t s, const uint16_t* x, int rows,
                                        int k, int64_t ldx, int n, float c, uint8_t* codes, uint8_t* sf, float* g_dev,
                                        const float* amax_dev, uint64_t seed, uint64_t offset, int* status) {
-  if (tc)
-    return wide ? launch_hadamard_quantize_pdl<true, true, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
-                                                                amax_dev, seed, offset, status)
-                : launch_hadamard_quantize_pdl<true, false, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
-                                                                 amax_dev, seed, offset, status);
-  return wide ? launch_hadamard_quantize_pdl<false, true, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
-                                                               amax_dev, seed, offset, status)
-              : launch_hadamard_quantize_pdl<false, false, kSR>(grid, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
-                                                                amax_dev, seed, offset, status);
+  if constexpr (kSR) {
+    if (n >= kAdjMinOrder)
+      return dispatch_hadamard_layout<true, true>(grid, tc, wide, s, x, rows, k, ldx, n, c, codes, sf, g_dev,
+                                                  amax_dev, seed, offset, status);
+  }
+  return dispatch_hadamard_layout<kSR, false>(grid, tc, wide, s, x, rows, k, ldx, n, c, codes, sf, g_dev, amax_dev,
+                                              seed, offset, status);
 }
 
 }  // namespace

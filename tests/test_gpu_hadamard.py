@@ -53,7 +53,7 @@ def test_hadamard_quantize_matches_oracle(lib, order, rows, k, layout):
     _assert_same(lib, q, ref, layout)
 
 
-@pytest.mark.parametrize("order", [16, 128])
+@pytest.mark.parametrize("order", [16, 32, 128])
 def test_hadamard_quantize_odd_pitch_and_small_k(lib, order):
     """Rows whose pitch is off the 32-B grid take the 128-bit load path."""
     rows, k, ld = 37, 512, 520
@@ -140,7 +140,7 @@ def test_full_size_sampled_rows(lib, order):
     assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape)[rows], sf_ref)
 
 
-@pytest.mark.parametrize("order", [1, 16, 128, 512])
+@pytest.mark.parametrize("order", [1, 16, 32, 128, 512])
 @pytest.mark.parametrize("rows,k", [(200, 1536), (3, 12288)])
 @pytest.mark.parametrize("layout", [0, 1], ids=["rowmajor", "tcgen05"])
 def test_rotated_stochastic_matches_oracle(lib, order, rows, k, layout):
