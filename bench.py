@@ -607,6 +607,10 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
                    reps)
     had["order=16_stochastic"] = {"ms": ms_hs, "gbs_two_pass": two_pass / ms_hs / 1e6,
                                   "frac_hbm": two_pass / ms_hs / 1e6 / hbm_peak}
+    ms_hs = _timed(torch, dev, flush, lambda: nv.quantize_hadamard_stochastic(x, 128, 1234, 0, nv.SF_TCGEN05, out=q),
+                   reps)
+    had["order=128_stochastic"] = {"ms": ms_hs, "gbs_two_pass": two_pass / ms_hs / 1e6,
+                                   "frac_hbm": two_pass / ms_hs / 1e6 / hbm_peak}
     out["hadamard_quantize_16384x8192"] = had
     del x, q
     # stochastic rounding of the codes (Philox4x32-10 in the kernel), same input and bytes
@@ -796,6 +800,9 @@ def run_part(args):
         for order in (16, 128):
             out[f"ms_order{order}"] = _timed(torch, dev, flush,
                                              lambda: nv.quantize_hadamard(x, order, nv.SF_TCGEN05, out=q), args.steps)
+        out["ms_order128_stochastic"] = _timed(
+            torch, dev, flush, lambda: nv.quantize_hadamard_stochastic(x, 128, 1234, 0, nv.SF_TCGEN05, out=q),
+            args.steps)
     elif args.part == "stochastic":
         x = to_dev(x_bits)
         q = nv.empty_quantized(*x.shape, nv.SF_TCGEN05, dev)
