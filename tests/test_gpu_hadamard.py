@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle_pool
 from oracle import hadamard_oracle as H
 from oracle import nvfp4_oracle as O
 from nvfp4_block_scaled_15_b200 import inputs
@@ -119,25 +120,18 @@ def test_rotated_gemm_matches_oracle(lib, order):
 
 
 @pytest.mark.parametrize("order", [16, 128])
-def test_full_size_sampled_rows(lib, order):
+def test_full_size_every_byte(lib, order):
     """Quantize-bandwidth workload [16384, 8192] with 1% outlier channels:
-    the amax of y and g exact, 64 sampled rows bit-exact."""
+    the amax of y and g exact, every code byte and scale equal to the
+    oracle's (run over the host cores by rows)."""
     x = inputs.quantize_bandwidth()
     q = lib.quantize_hadamard(dev_bf16(x), order, lib.SF_TCGEN05)
     torch.cuda.synchronize()
     assert lib.nvfp4_check_device_status() == lib.OK
-    rng = np.random.default_rng(19 + order)
-    rows = np.sort(rng.choice(x.shape[0], 64, replace=False))
-    # the amax over all rows, from the oracle's transform in slices
-    amax = np.float32(0.0)
-    for r0 in range(0, x.shape[0], 2048):
-        y = H.fwht_f32(O.bf16_to_f32(x[r0:r0 + 2048]), order)
-        amax = max(amax, np.float32(np.max(np.abs(y))))
-    g = O.global_scale(amax)
+    codes_ref, sf_ref, g, amax = oracle_pool.quantize_hadamard(x, order)
     assert f32_scalar(q.amax) == amax and f32_scalar(q.g) == g
-    codes_ref, sf_ref, _, _ = H.quantize_hadamard(x[rows], order, amax_value=amax)
-    assert np.array_equal(host_u8(q.codes)[rows], codes_ref)
-    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape)[rows], sf_ref)
+    assert np.array_equal(host_u8(q.codes), codes_ref)
+    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape), sf_ref)
 
 
 @pytest.mark.parametrize("order", [1, 16, 32, 128, 512])
@@ -154,17 +148,15 @@ def test_rotated_stochastic_matches_oracle(lib, order, rows, k, layout):
     _assert_same(lib, q, H.quantize_hadamard_sr(x, order, seed, offset), layout)
 
 
-def test_rotated_stochastic_full_size_sampled_rows(lib):
+@pytest.mark.parametrize("order", [16, 128])
+def test_rotated_stochastic_full_size_every_byte(lib, order):
+    """The same workload rotated then rounded stochastically (order 128 takes
+    the two-adjacent-blocks kernels): every byte equal to the oracle's."""
     x = inputs.quantize_bandwidth()
-    q = lib.quantize_hadamard_stochastic(dev_bf16(x), 16, 42, 1, lib.SF_TCGEN05)
+    q = lib.quantize_hadamard_stochastic(dev_bf16(x), order, 42, 1, lib.SF_TCGEN05)
     torch.cuda.synchronize()
     assert lib.nvfp4_check_device_status() == lib.OK
-    amax = np.float32(0.0)
-    for r0 in range(0, x.shape[0], 2048):
-        y = H.fwht_f32(O.bf16_to_f32(x[r0:r0 + 2048]), 16)
-        amax = max(amax, np.float32(np.max(np.abs(y))))
-    assert f32_scalar(q.amax) == amax
-    rows = np.sort(np.random.default_rng(29).choice(x.shape[0], 64, replace=False))
-    codes_ref, sf_ref, _, _ = H.quantize_hadamard_sr(x[rows], 16, 42, 1, amax_value=amax, row_ids=rows)
-    assert np.array_equal(host_u8(q.codes)[rows], codes_ref)
-    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape)[rows], sf_ref)
+    codes_ref, sf_ref, g, amax = oracle_pool.quantize_hadamard_sr(x, order, 42, 1)
+    assert f32_scalar(q.amax) == amax and f32_scalar(q.g) == g
+    assert np.array_equal(host_u8(q.codes), codes_ref)
+    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape), sf_ref)

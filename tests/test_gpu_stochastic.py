@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle_pool
 from oracle import nvfp4_oracle as O
 from oracle import stochastic_oracle as S
 from nvfp4_block_scaled_15_b200 import inputs
@@ -89,20 +90,19 @@ def test_edge_tensor_and_nonfinite(lib):
     assert f32_scalar(q.g) == 0.0 and not host_u8(q.codes).any()
 
 
-def test_full_size_sampled_rows(lib):
-    """Quantize-bandwidth workload [16384, 8192]: g and amax exact, 64 sampled
-    rows bit-exact (the oracle draws those rows' bits by their indices)."""
+def test_full_size_every_byte(lib):
+    """Quantize-bandwidth workload [16384, 8192]: g and amax exact, every code
+    byte and every scale equal to the oracle's (run over the host cores by
+    rows, each row drawing the random integers of its own index)."""
     x = inputs.quantize_bandwidth()
     seed, offset = 0x5EED, 11
     q = lib.quantize_stochastic(dev_bf16(x), seed, offset, lib.SF_TCGEN05)
     torch.cuda.synchronize()
     assert lib.nvfp4_check_device_status() == lib.OK
-    amax = O.amax(x)
-    assert f32_scalar(q.amax) == amax and f32_scalar(q.g) == O.global_scale(amax)
-    rows = np.sort(np.random.default_rng(23).choice(x.shape[0], 64, replace=False))
-    codes_ref, sf_ref, _, _ = S.quantize_sr(x[rows], seed, offset, amax_value=amax, row_ids=rows)
-    assert np.array_equal(host_u8(q.codes)[rows], codes_ref)
-    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape)[rows], sf_ref)
+    codes_ref, sf_ref, g, amax = oracle_pool.quantize_sr(x, seed, offset)
+    assert f32_scalar(q.amax) == amax and f32_scalar(q.g) == g
+    assert np.array_equal(host_u8(q.codes), codes_ref)
+    assert np.array_equal(O.unswizzle_sf_tcgen05(host_u8(q.sf), *x.shape), sf_ref)
 
 
 def test_mean_over_offsets_is_unbiased(lib):

@@ -3,7 +3,9 @@ what the oracle returns when called on the whole problem."""
 import numpy as np
 
 import oracle_pool
+from oracle import hadamard_oracle as H
 from oracle import nvfp4_oracle as O
+from oracle import stochastic_oracle as S
 from nvfp4_block_scaled_15_b200 import inputs
 
 
@@ -25,3 +27,22 @@ def test_pool_gemm_ref_equals_oracle():
     assert alpha2 == alpha
     assert np.all(np.abs(d2 - d) <= 1e-13 * float(alpha) * s)
     assert np.all(np.abs(s2 - s) <= 1e-13 * s)
+
+
+def _same(got, want):
+    assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
+    assert got[2] == want[2] and got[3] == want[3]
+
+
+def test_pool_stochastic_equals_oracle():
+    """Rows in several tasks draw the random integers of their own indices."""
+    x = inputs.activations_with_outliers(2600, 128, seed=47, fraction=0.02, factor=40.0)
+    _same(oracle_pool.quantize_sr(x, 0x1234_5678_9ABC, 5), S.quantize_sr(x, 0x1234_5678_9ABC, 5))
+
+
+def test_pool_rotated_equals_oracle():
+    """The amax of y from the slices' maxima, then the rows by slices."""
+    x = inputs.activations_with_outliers(2600, 256, seed=48, fraction=0.02, factor=40.0)
+    assert oracle_pool.rotated_amax(x, 64) == np.float32(np.max(np.abs(H.fwht_f32(O.bf16_to_f32(x), 64))))
+    _same(oracle_pool.quantize_hadamard(x, 64), H.quantize_hadamard(x, 64))
+    _same(oracle_pool.quantize_hadamard_sr(x, 32, 9, 3), H.quantize_hadamard_sr(x, 32, 9, 3))
