@@ -16,7 +16,9 @@ oracle's definition makes independent:
   * the rotated quantizer: the transform works inside a row, so the amax of
     y is the largest of the slices' maxima (``H.fwht_f32`` on each slice),
     and, given it, ``H.quantize_hadamard`` / ``H.quantize_hadamard_sr`` run
-    on slices of rows.
+    on slices of rows;
+  * MXFP4 (no global scale): rows quantize independently and each output
+    column depends on one weight row, as for NVFP4.
 Workers are started with ``spawn`` (safe after the process has used CUDA).
 """
 from __future__ import annotations
@@ -26,6 +28,7 @@ import os
 import numpy as np
 
 from oracle import hadamard_oracle as H
+from oracle import mxfp4_oracle as MX
 from oracle import nvfp4_oracle as O
 from oracle import stochastic_oracle as S
 
@@ -36,7 +39,7 @@ def _workers() -> int:
     return max(1, min(32, os.cpu_count() or 1))
 
 
-def _quantize_rows(kind, shm_in, shm_codes, shm_sf, rows, k, params, r0, r1):
+def _quantize_rows(kind, shm_in, shm_codes, shm_sf, rows, k, sf_block, params, r0, r1):
     """Codes and row-major scales of rows r0 .. r1 - 1 by the oracle function
     that ``kind`` names, the whole tensor's scale parameters given."""
     from multiprocessing import shared_memory
@@ -46,7 +49,7 @@ def _quantize_rows(kind, shm_in, shm_codes, shm_sf, rows, k, params, r0, r1):
     try:
         x = np.ndarray((rows, k), dtype=np.uint16, buffer=si.buf)
         codes = np.ndarray((rows, k // 2), dtype=np.uint8, buffer=sc.buf)
-        sf = np.ndarray((rows, k // 16), dtype=np.uint8, buffer=ss.buf)
+        sf = np.ndarray((rows, k // sf_block), dtype=np.uint8, buffer=ss.buf)
         ids = np.arange(r0, r1)
         if kind == "nvfp4":
             (g,) = params
@@ -58,6 +61,8 @@ def _quantize_rows(kind, shm_in, shm_codes, shm_sf, rows, k, params, r0, r1):
         elif kind == "hadamard":
             a, order = params
             c, s, _, _ = H.quantize_hadamard(x[r0:r1], order, amax_value=a)
+        elif kind == "mx":
+            c, s = MX.quantize_mx(x[r0:r1])
         elif kind == "hadamard_sr":
             a, order, seed, offset = params
             c, s, _, _ = H.quantize_hadamard_sr(x[r0:r1], order, seed, offset, amax_value=a, row_ids=ids)
@@ -91,23 +96,23 @@ def _pool():
     return ProcessPoolExecutor(max_workers=_workers(), mp_context=mp.get_context("spawn"))
 
 
-def _by_rows(x_bits: np.ndarray, kind: str, params: tuple):
-    """(packed codes [rows, k/2], row-major scales [rows, k/16]) of the whole
-    tensor, computed slice by slice."""
+def _by_rows(x_bits: np.ndarray, kind: str, params: tuple, sf_block: int = 16):
+    """(packed codes [rows, k/2], row-major scales [rows, k/sf_block]) of the
+    whole tensor, computed slice by slice."""
     from multiprocessing import shared_memory
     rows, k = x_bits.shape
     shms = [shared_memory.SharedMemory(create=True, size=max(1, n))
-            for n in (x_bits.nbytes, rows * k // 2, rows * k // 16)]
+            for n in (x_bits.nbytes, rows * k // 2, rows * k // sf_block)]
     try:
         np.ndarray(x_bits.shape, dtype=np.uint16, buffer=shms[0].buf)[:] = x_bits
         with _pool() as ex:
-            futs = [ex.submit(_quantize_rows, kind, shms[0].name, shms[1].name, shms[2].name, rows, k, params,
-                              r0, min(rows, r0 + _ROWS_PER_TASK))
+            futs = [ex.submit(_quantize_rows, kind, shms[0].name, shms[1].name, shms[2].name, rows, k, sf_block,
+                              params, r0, min(rows, r0 + _ROWS_PER_TASK))
                     for r0 in range(0, rows, _ROWS_PER_TASK)]
             for f in futs:
                 f.result()
         codes = np.ndarray((rows, k // 2), dtype=np.uint8, buffer=shms[1].buf).copy()
-        sf = np.ndarray((rows, k // 16), dtype=np.uint8, buffer=shms[2].buf).copy()
+        sf = np.ndarray((rows, k // sf_block), dtype=np.uint8, buffer=shms[2].buf).copy()
         return codes, sf
     finally:
         for s in shms:
@@ -179,6 +184,25 @@ def quantize_hadamard_sr(x_bits: np.ndarray, order: int, seed: int, offset: int)
     a = rotated_amax(x_bits, order)
     codes, sf = _by_rows(x_bits, "hadamard_sr", (a, order, seed, offset))
     return codes, sf, O.global_scale(a), a
+
+
+def quantize_mx(x_bits: np.ndarray):
+    """Same result as ``MX.quantize_mx(x_bits)``: (packed codes, E8M0 scales)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    if _small(x_bits):
+        return MX.quantize_mx(x_bits)
+    return _by_rows(x_bits, "mx", (), sf_block=MX.MX_BLOCK)
+
+
+def gemm_ref_mx(a_packed, a_sf, b_packed, b_sf, cols_per_slice: int = 2048):
+    """Same result as ``MX.gemm_ref_mx`` (D, S), over slices of B's rows."""
+    n = b_packed.shape[0]
+    ds, ss = [], []
+    for c0 in range(0, n, cols_per_slice):
+        d, s = MX.gemm_ref_mx(a_packed, a_sf, b_packed[c0:c0 + cols_per_slice], b_sf[c0:c0 + cols_per_slice])
+        ds.append(d)
+        ss.append(s)
+    return np.concatenate(ds, axis=1), np.concatenate(ss, axis=1)
 
 
 def gemm_ref(a_packed, a_sf, g_a, b_packed, b_sf, g_b, cols_per_slice: int = 2048):

@@ -4,6 +4,7 @@ import numpy as np
 
 import oracle_pool
 from oracle import hadamard_oracle as H
+from oracle import mxfp4_oracle as MX
 from oracle import nvfp4_oracle as O
 from oracle import stochastic_oracle as S
 from nvfp4_block_scaled_15_b200 import inputs
@@ -46,3 +47,14 @@ def test_pool_rotated_equals_oracle():
     assert oracle_pool.rotated_amax(x, 64) == np.float32(np.max(np.abs(H.fwht_f32(O.bf16_to_f32(x), 64))))
     _same(oracle_pool.quantize_hadamard(x, 64), H.quantize_hadamard(x, 64))
     _same(oracle_pool.quantize_hadamard_sr(x, 32, 9, 3), H.quantize_hadamard_sr(x, 32, 9, 3))
+
+
+def test_pool_mxfp4_equals_oracle():
+    x = inputs.activations_with_outliers(2600, 128, seed=49, fraction=0.02, factor=40.0)
+    got, want = oracle_pool.quantize_mx(x), MX.quantize_mx(x)
+    assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
+    pa, sa = MX.quantize_mx(inputs.gaussian_bf16((5, 128), seed=50))
+    pb, sb = want
+    d, s = MX.gemm_ref_mx(pa, sa, pb[:300], sb[:300])
+    d2, s2 = oracle_pool.gemm_ref_mx(pa, sa, pb[:300], sb[:300], cols_per_slice=64)
+    assert np.all(np.abs(d2 - d) <= 1e-13 * s) and np.all(np.abs(s2 - s) <= 1e-13 * s)
