@@ -643,59 +643,22 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
         "quantize_pass_ms": ms_s1, "quantize_pass_frac_hbm": one_pass / ms_s1 / 1e6 / hbm_peak}
     del x, q
 
-    # decode GEMV: W [28672, 8192] pre-quantized, x [M, 8192] quantized in the call
+    # decode GEMV: W [28672, 8192] pre-quantized, x [M, 8192] quantized in the
+    # call.  Three weight copies (396 MB, more than L2) in rotation, so no call
+    # finds its weights in L2 without a flush.
     xg, wg = pin["gemv"]
-    wq = nv.quantize(to_dev(wg), nv.SF_TCGEN05)
     n, k = wg.shape
-    res = {}
+    wqs = [nv.quantize(to_dev(wg), nv.SF_TCGEN05) for _ in range(3)]
+    stream = torch.cuda.current_stream(dev)
+    res, thr = {}, {}
     for m in (1, 8, 16):
         xm = to_dev(xg[:m])
         y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
         ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device=dev)
-        ms = _timed(torch, dev, flush, lambda: nv.gemv_batched(xm, wq, out=y, workspace=ws), reps)
         algo = n * k // 2 + n * k // 16 + m * k * 2 + m * n * 2
-        res[f"M={m}"] = {"ms": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak,
-                         "algorithmic_bytes": algo}
-    out["gemv_28672x8192"] = res
-    # decode throughput: calls back to back (as layers follow one another),
-    # three weight copies in rotation so no call finds its weights in L2
-    wqs = [wq] + [nv.quantize(to_dev(wg), nv.SF_TCGEN05) for _ in range(2)]
-    thr = {}
-    for m in (1, 8, 16):
-        xm = to_dev(xg[:m])
-        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(nv.nvfp4_workspace_bytes(nv.OP_GEMV_BATCHED, m, n, k), dtype=torch.uint8, device=dev)
-        calls = 30
         for i in range(6):
             nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
-        stream = torch.cuda.current_stream(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(calls):
-            nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / calls
-        algo = n * k // 2 + n * k // 16 + m * k * 2 + m * n * 2
-        # the same 30 calls captured once in a CUDA graph and replayed (how a
-        # decode step issues its layers), so no per-launch host work sits between them
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for i in range(calls):
-                nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
-        graph.replay()
-        torch.cuda.synchronize(dev)
-        stream = torch.cuda.current_stream(dev)
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        graph.replay()
-        graph.replay()
-        g1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_g = g0.elapsed_time(g1) / (2 * calls)
-        del graph
-        # one call per event pair, without an L2 flush: the three weight copies
-        # (396 MB, more than L2) in rotation keep every call's weights cold
+        # per call: one call per event pair, the weights cold by rotation
         ts = []
         for i in range(21):
             c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -705,10 +668,44 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
             ts.append((c0, c1))
         torch.cuda.synchronize(dev)
         ms_c = statistics.median(c0.elapsed_time(c1) for c0, c1 in ts)
+        # decode throughput: calls back to back (as layers follow one another)
+        calls = 30
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(calls):
+            nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / calls
+        # the same 30 calls captured once in a CUDA graph and replayed (how a
+        # decode step issues its layers), so no per-launch host work sits between them
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(calls):
+                nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        graph.replay()
+        graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_g = g0.elapsed_time(g1) / (2 * calls)
+        del graph
         thr[f"M={m}"] = {"ms_per_call": ms, "gbs": algo / ms / 1e6, "frac_hbm": algo / ms / 1e6 / hbm_peak,
-                         "graph_ms_per_call": ms_g, "graph_frac_hbm": algo / ms_g / 1e6 / hbm_peak,
-                         "cold_rotated_ms_per_call": ms_c,
-                         "cold_rotated_frac_hbm": algo / ms_c / 1e6 / hbm_peak}
+                         "graph_ms_per_call": ms_g, "graph_frac_hbm": algo / ms_g / 1e6 / hbm_peak}
+        # per call with a 256 MiB L2 flush (a write) before each, last: the
+        # flush's dirty lines are written back while the call streams the
+        # weights (and would be during the next measurement)
+        ms_f = _timed(torch, dev, flush, lambda: nv.gemv_batched(xm, wqs[0], out=y, workspace=ws), reps)
+        res[f"M={m}"] = {"ms": ms_c, "gbs": algo / ms_c / 1e6, "frac_hbm": algo / ms_c / 1e6 / hbm_peak,
+                         "l2": "inputs larger than L2: three weight copies (396 MB) in rotation, no flush",
+                         "ms_l2_flushed": ms_f, "frac_hbm_l2_flushed": algo / ms_f / 1e6 / hbm_peak,
+                         "algorithmic_bytes": algo}
+        for i in range(6):                      # write the flush's dirty lines back before the next M
+            nv.gemv_batched(xm, wqs[i % 3], out=y, workspace=ws)
+    out["gemv_28672x8192"] = res
     # the fixed cost an event pair sees around any one launch on this machine: a
     # one-element torch fill timed the same way as the per-call numbers
     tiny = torch.empty(1, dtype=torch.int32, device=dev)
@@ -722,10 +719,10 @@ def bench_parts(nv, torch, dev, flush, pin, hbm_peak, fp4_peak, peaks_src):
     torch.cuda.synchronize(dev)
     thr["per_call_floor_ms"] = statistics.median(c0.elapsed_time(c1) for c0, c1 in ts)
     thr["note"] = ("ms_per_call: 30 calls between one event pair; graph: the same calls replayed from a CUDA "
-                   "graph; cold_rotated: one call per event pair; all with three weight copies in rotation "
-                   "(396 MB, more than L2); per_call_floor_ms: an event pair around a one-element fill")
+                   "graph; both with three weight copies in rotation (396 MB, more than L2); "
+                   "per_call_floor_ms: an event pair around a one-element fill")
     out["gemv_28672x8192_back_to_back"] = thr
-    del wq, wqs
+    del wqs
 
     # long-K: A [4096, 28672] bf16 quantized in the call, W [8192, 28672] pre-quantized
     al, wl = pin["longk"]
