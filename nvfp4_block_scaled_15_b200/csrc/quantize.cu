@@ -366,7 +366,7 @@ __device__ __forceinline__ float rotated_absmax(const uint32_t (&w)[8], int n) {
   return m;
 }
 
-// Orders n >= 32 with the thread's two blocks adjacent (p0 = elements
+// Orders n >= 64 with the thread's two blocks adjacent (p0 = elements
 // 32j .. 32j + 15 of the segment, p1 = 32j + 16 .. 32j + 31): stage h = 16
 // pairs p0 with p1 inside the thread, and a stage h >= 32 pairs lanes tid and
 // tid ^ (h/32), one cross-lane stage fewer than with one block per lane.
@@ -401,7 +401,7 @@ __device__ __forceinline__ void fwht_pair_cross_lanes(float2 (&p0)[8], float2 (&
   }
 }
 
-// y = x H for the thread's two adjacent blocks (n >= 32), c = fp32(1/sqrt(n)).
+// y = x H for the thread's two adjacent blocks (n >= 64), c = fp32(1/sqrt(n)).
 __device__ __forceinline__ void rotate_pair(const uint32_t (&w0)[8], const uint32_t (&w1)[8], int n, float c,
                                             float2 (&p0)[8], float2 (&p1)[8]) {
   bf16_block_to_f32(w0, p0);
@@ -418,11 +418,10 @@ __device__ __forceinline__ void rotate_pair(const uint32_t (&w0)[8], const uint3
   }
 }
 
-// max |y / c| over the thread's two adjacent blocks (n >= 32), the last stage
-// folded into the maximum as in rotated_absmax.  For n = 32 it is stage 16,
-// inside the thread; beyond, the lane with bit lm clear takes the pair's
-// positions 0..15 (its p0 and the partner's), the partner positions 16..31,
-// so each lane sends 16 values.
+// max |y / c| over the thread's two adjacent blocks (n >= 64), the last stage
+// folded into the maximum as in rotated_absmax: the lane with bit lm clear
+// takes the pair's positions 0..15 (its p0 and the partner's), the partner
+// positions 16..31, so each lane sends 16 values.
 __device__ __forceinline__ float rotated_absmax_pair(const uint32_t (&w0)[8], const uint32_t (&w1)[8], int n) {
   float2 p0[8], p1[8];
   bf16_block_to_f32(w0, p0);
@@ -430,12 +429,6 @@ __device__ __forceinline__ float rotated_absmax_pair(const uint32_t (&w0)[8], co
   fwht_in_thread(p0, 16);
   fwht_in_thread(p1, 16);
   float m = 0.0f;
-  if (n == 32) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      m = max3_nan_f32(m, __fadd_rn(fabsf(p0[i].x), fabsf(p1[i].x)), __fadd_rn(fabsf(p0[i].y), fabsf(p1[i].y)));
-    return m;
-  }
   fwht_pair_stage16(p0, p1);
   fwht_pair_cross_lanes(p0, p1, n >> 1);
   const int lm = n >> 6;                        // last stage h = n/2
@@ -454,6 +447,7 @@ __device__ __forceinline__ float rotated_absmax_pair(const uint32_t (&w0)[8], co
 // adjacent blocks per thread (at 128 the amax pass measured 3 % faster, at
 // 256 and 512 8-10 %; at 32 and 64 within noise or slower).
 constexpr int kAdjMinOrder = 128;
+static_assert(kAdjMinOrder >= 64, "rotated_absmax_pair folds a cross-lane last stage (n >= 64)");
 
 // The thread's two blocks of a 512-block segment: b1 = b0 + kThreads (one
 // block per lane in each half), or, with kAdj, b0 = 2 * tid and b1 = b0 + 1.
