@@ -190,25 +190,25 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint16_t* __re
 }
 
 // Pass 2 with stochastic rounding of the element codes: the same grid,
-// scales and stores as quantize_kernel; the random integers of block b of row
-// r come from Philox4x32-10 with key (seed_lo, seed_hi) and counters
-// (2b + h, r, offset_lo, offset_hi), h = 0, 1.
-template <bool kTcLayout, bool kWide>
+// scales and stores as quantize_kernel, kRows rows per CTA; the random
+// integers of block b of row r come from Philox4x32-10 with key
+// (seed_lo, seed_hi) and counters (2b + h, r, offset_lo, offset_hi), h = 0, 1.
+template <bool kTcLayout, bool kWide, int kRows>
 __global__ void __launch_bounds__(kThreads)
     quantize_sr_kernel(const uint16_t* __restrict__ x, int rows, int k, int64_t ldx, uint8_t* __restrict__ codes,
                        uint8_t* __restrict__ sf, float* __restrict__ g_out, const float* __restrict__ amax_in,
                        uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo, uint32_t off_hi,
                        int* __restrict__ status) {
   __shared__ float2 table[128];
-  const int r = static_cast<int>(gridDim.x - 1 - blockIdx.x);
+  const int r0 = static_cast<int>(gridDim.x - 1 - blockIdx.x) * kRows;
   const int kb = k >> 4;
   const int b0 = blockIdx.y * kSegBlocks + static_cast<int>(threadIdx.x);
   const int b1 = b0 + kThreads;
 
-  const bool real_row = r < rows;
-
-  uint32_t w0[8], w1[8];                       // x and the table before the wait, as in quantize_kernel
-  load_two_blocks<kWide>(x + static_cast<int64_t>(r) * ldx, real_row, kb, b0, b1, w0, w1);
+  uint32_t w0[kRows][8], w1[kRows][8];         // x and the table before the wait, as in quantize_kernel
+#pragma unroll
+  for (int j = 0; j < kRows; ++j)
+    load_two_blocks<kWide>(x + static_cast<int64_t>(r0 + j) * ldx, r0 + j < rows, kb, b0, b1, w0[j], w1[j]);
   fill_scale_table(table);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   bool valid;
@@ -220,20 +220,26 @@ __global__ void __launch_bounds__(kThreads)
   if (!valid) {                                // all-zero codes and scales
     g = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w0[i] = w1[i] = 0u;
+    for (int j = 0; j < kRows; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w0[j][i] = w1[j][i] = 0u;
   }
   __syncthreads();
 
-  uint32_t s0, s1;
-  two_block_scales(w0, w1, g, s0, s1);
-  const uint32_t ur = static_cast<uint32_t>(r);
-  const uint2 c0 = block_codes_sr(w0, g, table[s0 & 0x7Fu],
-                                  philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi),
-                                  philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi));
-  const uint2 c1 = block_codes_sr(w1, g, table[s1 & 0x7Fu],
-                                  philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi),
-                                  philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi));
-  store_two_blocks<kTcLayout>(codes, sf, r, real_row, k, kb, b0, b1, c0, c1, s0, s1);
+#pragma unroll
+  for (int j = 0; j < kRows; ++j) {
+    const int r = r0 + j;
+    uint32_t s0, s1;
+    two_block_scales(w0[j], w1[j], g, s0, s1);
+    const uint32_t ur = static_cast<uint32_t>(r);
+    const uint2 c0 = block_codes_sr(w0[j], g, table[s0 & 0x7Fu],
+                                    philox4x32_10(make_uint4(2u * b0, ur, off_lo, off_hi), seed_lo, seed_hi),
+                                    philox4x32_10(make_uint4(2u * b0 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi));
+    const uint2 c1 = block_codes_sr(w1[j], g, table[s1 & 0x7Fu],
+                                    philox4x32_10(make_uint4(2u * b1, ur, off_lo, off_hi), seed_lo, seed_hi),
+                                    philox4x32_10(make_uint4(2u * b1 + 1u, ur, off_lo, off_hi), seed_lo, seed_hi));
+    store_two_blocks<kTcLayout>(codes, sf, r, r < rows, k, kb, b0, b1, c0, c1, s0, s1);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -769,6 +775,8 @@ cudaError_t launch_hadamard_quantize_pdl(dim3 grid, cudaStream_t s, const uint16
                             static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32), status);
 }
 
+constexpr int kSRRows = 2;                     // rows per CTA of the stochastic quantize pass
+
 template <bool kTc, bool kWide>
 cudaError_t launch_quantize_sr_pdl(dim3 grid, cudaStream_t s, const uint16_t* x, int rows, int k, int64_t ldx,
                                    uint8_t* codes, uint8_t* sf, float* g_dev, const float* amax_dev, uint64_t seed,
@@ -782,7 +790,7 @@ cudaError_t launch_quantize_sr_pdl(dim3 grid, cudaStream_t s, const uint16_t* x,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_sr_kernel<kTc, kWide>, x, rows, k, ldx, codes, sf, g_dev, amax_dev,
+  return cudaLaunchKernelEx(&cfg, quantize_sr_kernel<kTc, kWide, kSRRows>, x, rows, k, ldx, codes, sf, g_dev, amax_dev,
                             static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
                             static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32), status);
 }
@@ -978,7 +986,7 @@ nvfp4_status launch_quantize_sr(const void* x, int64_t rows, int64_t k, int64_t 
   if (grid_rows == 0 || segs == 0)
     return launch_status(launch_quantize_sr_pdl<false, false>(dim3(1, 1), s, xs, 0, 0, ldx, cs, ss, g_dev, amax_dev,
                                                               seed, offset, status));
-  const dim3 grid(static_cast<unsigned>(grid_rows), segs);
+  const dim3 grid(static_cast<unsigned>((grid_rows + kSRRows - 1) / kSRRows), segs);
   const bool wide = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
   cudaError_t e;
   if (layout == NVFP4_SF_TCGEN05)
